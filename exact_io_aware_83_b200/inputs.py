@@ -1,0 +1,91 @@
+"""Seeded synthetic attention inputs shared by the CUDA path's tests, the benchmark and
+the oracle's callers.
+
+This module holds none of the method's arithmetic: it only draws i.i.d. Gaussian
+tensors from a CPU ``torch.Generator`` and rounds them to bf16, so the same seed gives
+the same bytes on every host.  Draw order is q, k, v, then dO.
+
+Workloads (shapes of the pages' GPT-3 2K / 8K-context training runs and of the
+head-dimension-256 and grouped-query variants named on the FlashAttention-2 page):
+
+====================  ==  ===  ===  ====  ===  ======  =========  =====================
+name                  B   Hq   Hkv  N     d    causal  passes     q distribution
+====================  ==  ===  ===  ====  ===  ======  =========  =====================
+tiny_fwd_d64          1   1    1    128   64   no      fwd        N(0,1)
+gpt_2k_causal         8   16   16   2048  128  yes     fwd+bwd    N(0,1)
+long_8k_causal        2   16   16   8192  128  yes     fwd+bwd    N(0,1)
+gqa_4k_causal_fwd     4   32   8    4096  128  yes     fwd        N(0,1)
+d256_4k_stress        2   8    8    4096  256  no      fwd+bwd    N(0,4^2)
+====================  ==  ===  ===  ====  ===  ======  =========  =====================
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    backward: bool
+    q_std: float
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        # The caller passes the softmax scale as fp32; 1/sqrt(128) is not exact in fp32,
+        # so every consumer uses the fp32-rounded value.
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
+
+    def fwd_flops(self) -> float:
+        """4 B Hq N^2 d, halved when causal (the metric's convention)."""
+        f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def bwd_flops(self) -> float:
+        """2.5 x the forward count."""
+        return 2.5 * self.fwd_flops()
+
+
+WORKLOADS = {
+    w.name: w
+    for w in (
+        Workload("tiny_fwd_d64", 1, 1, 1, 128, 64, False, False, 1.0, 1),
+        Workload("gpt_2k_causal", 8, 16, 16, 2048, 128, True, True, 1.0, 2),
+        Workload("long_8k_causal", 2, 16, 16, 8192, 128, True, True, 1.0, 3),
+        Workload("gqa_4k_causal_fwd", 4, 32, 8, 4096, 128, True, False, 1.0, 4),
+        Workload("d256_4k_stress", 2, 8, 8, 4096, 256, False, True, 4.0, 5),
+    )
+}
+
+
+def draw(B: int, Hq: int, Hkv: int, N: int, d: int, seed: int, q_std: float = 1.0,
+         with_dout: bool = True):
+    """Return bf16 CPU tensors (q, k, v[, dout]) in ``[B, H, N, d]`` layout."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((B, Hq, N, d), generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q = q * q_std
+    k = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hkv, N, d), generator=g, dtype=torch.float32)
+    out = [q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)]
+    if with_dout:
+        do = torch.randn((B, Hq, N, d), generator=g, dtype=torch.float32)
+        out.append(do.to(torch.bfloat16))
+    return tuple(out)
+
+
+def draw_workload(w: Workload, with_dout: bool | None = None):
+    """Inputs of a named workload (dO drawn when the workload has a backward pass)."""
+    if with_dout is None:
+        with_dout = w.backward
+    return draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, w.q_std, with_dout)

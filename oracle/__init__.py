@@ -1,0 +1,110 @@
+"""ctypes front end of the fp64 attention oracle (``attention_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, the smoke check and the benchmark's
+CPU-baseline leg may import this package; the CUDA library and its binding never do.
+
+Every function takes and returns numpy float64 arrays in the ``[B, H, N, d]`` layout
+(LSE / Delta: ``[B, Hq, N]``).  Inputs given in bf16 are upcast exactly by the caller.
+
+Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy example
+of the "Consideration"/FlashAttention article page, finite differences and invariants):
+``oracle_fwd``, ``oracle_bwd`` and ``online_softmax_stats`` all have pins; none is
+"parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ci = ctypes.c_int
+        lib.oracle_fwd.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, ci, ctypes.c_double]
+        lib.oracle_fwd.restype = ci
+        lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                   ci, ci, ci, ci, ci, ci, ctypes.c_double]
+        lib.oracle_bwd.restype = ci
+        lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
+        lib.oracle_online_softmax_stats.restype = ci
+        _LIB = lib
+    return _LIB
+
+
+def _as_f64(a) -> np.ndarray:
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    return a
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def set_threads(n: int) -> None:
+    """Set the OpenMP thread count used by later oracle calls in this process."""
+    os.environ["OMP_NUM_THREADS"] = str(int(n))
+    try:
+        gomp = ctypes.CDLL("libgomp.so.1")
+        gomp.omp_set_num_threads(ctypes.c_int(int(n)))
+    except OSError:
+        pass
+
+
+def _shapes(q, k):
+    B, Hq, N, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, Nk, dk) != (B, N, d):
+        raise ValueError(f"shape mismatch q{q.shape} k{k.shape}")
+    return B, Hq, Hkv, N, d
+
+
+def attention_fwd(q, k, v, causal: bool, scale: float):
+    """O = softmax(scale Q K^T [+ causal mask]) V and the natural-log LSE per row."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    rc = _lib().oracle_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                           B, Hq, Hkv, N, d, int(bool(causal)), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_fwd failed with {rc}")
+    return o, lse
+
+
+def attention_bwd(q, k, v, dout, causal: bool, scale: float):
+    """Exact gradient of <O, dO>: returns dq, dk, dv, lse, delta."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    delta = np.empty((B, Hq, N), dtype=np.float64)
+    rc = _lib().oracle_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                           _ptr(dv), _ptr(lse), _ptr(delta), B, Hq, Hkv, N, d,
+                           int(bool(causal)), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bwd failed with {rc}")
+    return dq, dk, dv, lse, delta
+
+
+def online_softmax_stats(scores, block: int):
+    """(m, l) of the blocked online-softmax recurrence over a 1-D score row."""
+    s = _as_f64(scores).reshape(-1)
+    m = ctypes.c_double()
+    l = ctypes.c_double()
+    rc = _lib().oracle_online_softmax_stats(_ptr(s), s.size, int(block), ctypes.byref(m),
+                                            ctypes.byref(l))
+    if rc != 0:
+        raise RuntimeError(f"oracle_online_softmax_stats failed with {rc}")
+    return m.value, l.value

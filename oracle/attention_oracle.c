@@ -1,0 +1,253 @@
+/*
+ * Plain fp64 CPU oracle for exact scaled-dot-product attention and its gradient.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or load this
+ * file; only the test-suite, the smoke check and the benchmark's CPU-baseline leg do.
+ * It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes (written out from the definition, not from any blocked algorithm):
+ *
+ *   The method is exact: "FlashAttention1" Q&A page, question "key algorithmic
+ *   innovations" (it keeps mathematical equivalence with standard attention), and the
+ *   "flash attention ... deep dive" page, section "Algorithm behind the article" (the
+ *   blocked result is the real answer, not an approximation).  So the oracle is the
+ *   standard attention of that deep-dive page, Steps 1-3 (S = Q K', row softmax,
+ *   output = softmax(S) V), evaluated one query row at a time in fp64:
+ *
+ *     g      = Hq / Hkv, kv(h) = floor(h / g)          (grouped-query heads share K/V)
+ *     J(i)   = {0..N-1}, or {0..i} when causal          (top-left causal mask)
+ *     s_ij   = scale * <q_i, k_j>,  j in J(i)
+ *     m_i    = max_j s_ij,  l_i = sum_j exp(s_ij - m_i)
+ *     LSE_i  = m_i + ln l_i                              (natural log)
+ *     P_ij   = exp(s_ij - LSE_i)
+ *     O_i    = sum_j P_ij v_j
+ *
+ *   The pages never write the backward pass; they only require it to recompute the
+ *   score tiles instead of storing them (next-generation page, "Recomputation").  The
+ *   oracle therefore takes the plain calculus gradient of L = <O, dO>:
+ *
+ *     dP_ij  = <do_i, v_j>
+ *     Delta_i = sum_j P_ij dP_ij
+ *     dS_ij  = P_ij (dP_ij - Delta_i)
+ *     dQ_i   = scale * sum_j dS_ij k_j
+ *     dK_j   = scale * sum_{h: kv(h)=kv} sum_{i: j in J(i)} dS_ij q_i
+ *     dV_j   =         sum_{h: kv(h)=kv} sum_{i: j in J(i)} P_ij do_i
+ *
+ * Layout: every tensor is [B, H, N, d] contiguous (LSE and Delta are [B, Hq, N]).
+ * Every output element is written by exactly one loop iteration with a fixed summation
+ * order, so results do not depend on the OpenMP thread count.
+ *
+ * Return codes: 0 on success, -1 for an invalid argument (nothing written),
+ * -2 when scratch memory cannot be obtained.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <stddef.h>
+
+static int check_args(int B, int Hq, int Hkv, int N, int d)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1) return -1;
+    if (Hq % Hkv != 0) return -1;
+    return 0;
+}
+
+static double dotd(const double *a, const double *b, int d)
+{
+    double acc = 0.0;
+    for (int c = 0; c < d; ++c) acc += a[c] * b[c];
+    return acc;
+}
+
+/* Number of keys row i may attend to: |J(i)|. */
+static int row_extent(int i, int N, int causal)
+{
+    return causal ? i + 1 : N;
+}
+
+/* s_ij for j in J(i) into s[], and the natural-log logsumexp of that row. */
+static double scores_and_lse(const double *qi, const double *kh, int i, int N, int d,
+                             int causal, double scale, double *s)
+{
+    const int J = row_extent(i, N, causal);
+    double m = -INFINITY;
+    for (int j = 0; j < J; ++j) {
+        s[j] = scale * dotd(qi, kh + (size_t)j * d, d);
+        if (s[j] > m) m = s[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < J; ++j) l += exp(s[j] - m);
+    return m + log(l);
+}
+
+/* Forward: O [B,Hq,N,d] and LSE [B,Hq,N]. */
+int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
+               int B, int Hq, int Hkv, int N, int d, int causal, double scale)
+{
+    if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !o || !lse) return -1;
+    const int g = Hq / Hkv;
+    const long long rows = (long long)B * Hq * N;
+    int fail = 0;
+#pragma omp parallel reduction(|: fail)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!s) {
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < rows; ++r) {
+                const int i = (int)(r % N);
+                const long long bh = r / N;
+                const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+                const int kvh = h / g;
+                const double *qi = q + (size_t)r * d;
+                const double *kh = k + ((size_t)b * Hkv + kvh) * (size_t)N * d;
+                const double *vh = v + ((size_t)b * Hkv + kvh) * (size_t)N * d;
+                const double L = scores_and_lse(qi, kh, i, N, d, causal, scale, s);
+                double *oi = o + (size_t)r * d;
+                for (int c = 0; c < d; ++c) oi[c] = 0.0;
+                const int J = row_extent(i, N, causal);
+                for (int j = 0; j < J; ++j) {
+                    const double p = exp(s[j] - L);
+                    const double *vj = vh + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
+                }
+                lse[r] = L;
+            }
+            free(s);
+        }
+    }
+    return fail ? -2 : 0;
+}
+
+/*
+ * Backward: dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d].  lse_out and delta_out ([B,Hq,N])
+ * may be NULL; when given they receive LSE_i and Delta_i.
+ *
+ * Pass 1 runs over query rows (LSE_i, Delta_i, dQ_i); pass 2 runs over key rows and
+ * recomputes s_ij, P_ij and dP_ij for every query row that attends to that key.
+ */
+int oracle_bwd(const double *q, const double *k, const double *v, const double *dout,
+               double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
+               int B, int Hq, int Hkv, int N, int d, int causal, double scale)
+{
+    if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !dout || !dq || !dk || !dv)
+        return -1;
+    const int g = Hq / Hkv;
+    const long long qrows = (long long)B * Hq * N;
+    double *L = (double *)malloc(sizeof(double) * (size_t)qrows);
+    double *D = (double *)malloc(sizeof(double) * (size_t)qrows);
+    if (!L || !D) { free(L); free(D); return -2; }
+    int fail = 0;
+
+    /* Pass 1: per query row. */
+#pragma omp parallel reduction(|: fail)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!s || !dp) {
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < qrows; ++r) {
+                const int i = (int)(r % N);
+                const long long bh = r / N;
+                const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+                const int kvh = h / g;
+                const double *qi = q + (size_t)r * d;
+                const double *doi = dout + (size_t)r * d;
+                const double *kh = k + ((size_t)b * Hkv + kvh) * (size_t)N * d;
+                const double *vh = v + ((size_t)b * Hkv + kvh) * (size_t)N * d;
+                const double Li = scores_and_lse(qi, kh, i, N, d, causal, scale, s);
+                const int J = row_extent(i, N, causal);
+                double Di = 0.0;
+                for (int j = 0; j < J; ++j) {
+                    dp[j] = dotd(doi, vh + (size_t)j * d, d);
+                    Di += exp(s[j] - Li) * dp[j];
+                }
+                double *dqi = dq + (size_t)r * d;
+                for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+                for (int j = 0; j < J; ++j) {
+                    const double dS = exp(s[j] - Li) * (dp[j] - Di);
+                    const double *kj = kh + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) dqi[c] += dS * kj[c];
+                }
+                for (int c = 0; c < d; ++c) dqi[c] *= scale;
+                L[r] = Li;
+                D[r] = Di;
+            }
+        }
+        free(s);
+        free(dp);
+    }
+    if (fail) { free(L); free(D); return -2; }
+
+    /* Pass 2: per key row of each K/V head. */
+    const long long krows = (long long)B * Hkv * N;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long r = 0; r < krows; ++r) {
+        const int j = (int)(r % N);
+        const long long bk = r / N;
+        const int kvh = (int)(bk % Hkv), b = (int)(bk / Hkv);
+        const double *kj = k + (size_t)r * d;
+        const double *vj = v + (size_t)r * d;
+        double *dkj = dk + (size_t)r * d;
+        double *dvj = dv + (size_t)r * d;
+        for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+        for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
+            const size_t head = ((size_t)b * Hq + h) * (size_t)N;
+            const int i0 = causal ? j : 0;
+            for (int i = i0; i < N; ++i) {
+                const double *qi = q + (head + i) * d;
+                const double *doi = dout + (head + i) * d;
+                const double s = scale * dotd(qi, kj, d);
+                const double P = exp(s - L[head + i]);
+                const double dP = dotd(doi, vj, d);
+                const double dS = P * (dP - D[head + i]);
+                for (int c = 0; c < d; ++c) {
+                    dvj[c] += P * doi[c];
+                    dkj[c] += dS * qi[c];
+                }
+            }
+        }
+        for (int c = 0; c < d; ++c) dkj[c] *= scale;
+    }
+
+    if (lse_out)
+        for (long long r = 0; r < qrows; ++r) lse_out[r] = L[r];
+    if (delta_out)
+        for (long long r = 0; r < qrows; ++r) delta_out[r] = D[r];
+    free(L);
+    free(D);
+    return 0;
+}
+
+/*
+ * The online-softmax recurrence of the "FlashAttention1" Q&A page, question
+ * "computation of the softmax function", over one row of scores split into blocks of
+ * `block` entries: for block t with local maximum lm_t and local sum
+ * ls_t = sum exp(s - lm_t),
+ *     m_t = max(m_{t-1}, lm_t)
+ *     l_t = l_{t-1} exp(m_{t-1} - m_t) + ls_t exp(lm_t - m_t)
+ * Returns m and l after the last block through the out-pointers (LSE = m + ln l).
+ * Used by the tests to check that the blocked statistics equal the two-pass ones.
+ */
+int oracle_online_softmax_stats(const double *s, int n, int block, double *m_out,
+                                double *l_out)
+{
+    if (!s || n < 1 || block < 1 || !m_out || !l_out) return -1;
+    double m = -INFINITY, l = 0.0;
+    for (int t0 = 0; t0 < n; t0 += block) {
+        const int t1 = t0 + block < n ? t0 + block : n;
+        double lm = -INFINITY;
+        for (int j = t0; j < t1; ++j)
+            if (s[j] > lm) lm = s[j];
+        double ls = 0.0;
+        for (int j = t0; j < t1; ++j) ls += exp(s[j] - lm);
+        const double mn = lm > m ? lm : m;
+        l = (m == -INFINITY ? 0.0 : l * exp(m - mn)) + ls * exp(lm - mn);
+        m = mn;
+    }
+    *m_out = m;
+    *l_out = l;
+    return 0;
+}

@@ -1,0 +1,321 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each pin is chosen so that a plausible slip in the oracle (a dropped term, a wrong
+sign, a swapped index, K used where V belongs, the wrong K/V head for a query head,
+the causal mask on the wrong side, a missing scale) fails at least one test:
+
+* closed forms: Q = 0 (uniform softmax), V = 1 (rows of P sum to one), a one-hot
+  dominant score, N = 1;
+* the toy 4x4 example printed on the "Consideration is All You Want" page, with values
+  derived by hand (tests/golden/p5_toy_scores.txt);
+* the online-softmax recurrence of the "FlashAttention1" Q&A page and a tiled forward
+  that merges blocks with the rescaling described on the "flash attention deep dive"
+  page ("Intuition"), against the oracle's two-pass rows;
+* scipy's logsumexp for the LSE;
+* central finite differences of L = <O, dO> for the gradient;
+* Delta_i = <dO_i, O_i>, sum_j dK_j = 0, sum_j dV_j = sum_i dO_i;
+* grouped-query attention equals multi-head attention with repeated K/V.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "p5_toy_scores.txt")
+
+
+def _load_golden():
+    scores, vals = [], {}
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            parts = line.split()
+            if len(parts) == 4:
+                scores.append([float(x) for x in parts])
+            else:
+                vals[parts[0]] = float(parts[1])
+    return np.array(scores), vals
+
+
+def _embed_scores(S):
+    """Q = I, K = S^T, V = I, scale 1: then Q K^T = S and O = P."""
+    n = S.shape[0]
+    q = np.eye(n)[None, None]
+    k = S.T.copy()[None, None]
+    v = np.eye(n)[None, None]
+    return q, k, v
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ---------------------------------------------------------------------------- forward
+
+
+def test_toy_example_non_causal():
+    S, gv = _load_golden()
+    q, k, v = _embed_scores(S)
+    o, lse = oracle.attention_fwd(q, k, v, causal=False, scale=1.0)
+    np.testing.assert_allclose(lse[0, 0], gv["lse_full"], rtol=0, atol=1e-13)
+    p_of = {s: gv[f"p_of_{s}"] for s in (1, 2, 3, 4)}
+    expect = np.vectorize(lambda s: p_of[int(s)])(S)
+    np.testing.assert_allclose(o[0, 0], expect, rtol=0, atol=1e-13)
+
+
+def test_toy_example_causal():
+    S, gv = _load_golden()
+    q, k, v = _embed_scores(S)
+    o, lse = oracle.attention_fwd(q, k, v, causal=True, scale=1.0)
+    np.testing.assert_allclose(
+        lse[0, 0], [gv[f"lse_causal_{r}"] for r in "ABCD"], rtol=0, atol=1e-13)
+    # Row A keeps only key A; row B: softmax(2, 1) over keys A, B; keys after the
+    # query get exactly zero weight.
+    assert o[0, 0, 0, 0] == 1.0 and np.all(o[0, 0, 0, 1:] == 0.0)
+    np.testing.assert_allclose(o[0, 0, 1, :2], [math.e / (math.e + 1), 1 / (math.e + 1)],
+                               atol=1e-15)
+    assert np.all(o[0, 0, 1, 2:] == 0.0) and np.all(o[0, 0, 2, 3:] == 0.0)
+
+
+def test_toy_example_online_recurrence_2x2_tiles():
+    S, gv = _load_golden()
+    m, l = oracle.online_softmax_stats(S[0], block=2)
+    assert m == gv["row_A_tile2_m"]
+    assert abs(l - gv["row_A_tile2_l"]) < 1e-14
+    assert abs(m + math.log(l) - gv["lse_full"]) < 1e-13
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_gives_mean_of_values(causal):
+    B, Hq, Hkv, N, d = 2, 4, 2, 9, 5
+    r = _rng(1)
+    q = np.zeros((B, Hq, N, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    o, lse = oracle.attention_fwd(q, k, v, causal, scale=0.3)
+    g = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            for i in range(N):
+                J = i + 1 if causal else N
+                np.testing.assert_allclose(o[b, h, i], v[b, h // g, :J].mean(0), atol=1e-14)
+                assert abs(lse[b, h, i] - math.log(J)) < 1e-14
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_of_p_sum_to_one(causal):
+    r = _rng(2)
+    q = 3 * r.standard_normal((1, 2, 33, 8))
+    k = r.standard_normal((1, 2, 33, 8))
+    v = np.ones((1, 2, 33, 8))
+    o, _ = oracle.attention_fwd(q, k, v, causal, scale=0.5)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_one_hot_dominant_score_selects_value_row(causal):
+    # K = I (N <= d) and q_i = alpha e_t(i): s_ij = scale*alpha*[j == t(i)].  With
+    # scale*alpha = 800 every other weight is exp(-800), which underflows in fp64, so
+    # O_i = v_t(i) and LSE_i = 800 exactly.
+    N, d = 6, 8
+    r = _rng(3)
+    t = [int(r.integers(0, (i + 1) if causal else N)) for i in range(N)]
+    q = np.zeros((1, 1, N, d))
+    for i, ti in enumerate(t):
+        q[0, 0, i, ti] = 1600.0
+    k = np.zeros((1, 1, N, d))
+    k[0, 0, :, :N] = np.eye(N)
+    v = r.standard_normal((1, 1, N, d))
+    o, lse = oracle.attention_fwd(q, k, v, causal, scale=0.5)
+    for i, ti in enumerate(t):
+        np.testing.assert_array_equal(o[0, 0, i], v[0, 0, ti])
+        assert lse[0, 0, i] == 800.0
+
+
+def test_single_token_causal():
+    r = _rng(4)
+    q, k, v = (r.standard_normal((1, 1, 1, 4)) for _ in range(3))
+    o, lse = oracle.attention_fwd(q, k, v, True, scale=0.7)
+    np.testing.assert_array_equal(o[0, 0, 0], v[0, 0, 0])
+    assert abs(lse[0, 0, 0] - 0.7 * float(q[0, 0, 0] @ k[0, 0, 0])) < 1e-15
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_lse_matches_scipy_logsumexp(causal):
+    r = _rng(5)
+    N, d, scale = 40, 16, 0.25
+    q = 4 * r.standard_normal((1, 1, N, d))
+    k = r.standard_normal((1, 1, N, d))
+    v = r.standard_normal((1, 1, N, d))
+    _, lse = oracle.attention_fwd(q, k, v, causal, scale)
+    for i in range(N):
+        J = i + 1 if causal else N
+        s = scale * (k[0, 0, :J] @ q[0, 0, i])
+        assert abs(lse[0, 0, i] - scipy.special.logsumexp(s)) < 1e-12
+
+
+@pytest.mark.parametrize("block", [1, 2, 3, 7, 128, 1000])
+def test_online_softmax_stats_equal_two_pass(block):
+    r = _rng(6)
+    for scale in (1.0, 30.0):
+        s = scale * r.standard_normal(300)
+        m, l = oracle.online_softmax_stats(s, block)
+        assert m == s.max()
+        assert abs((m + math.log(l)) - scipy.special.logsumexp(s)) < 1e-12
+
+
+def _tiled_forward(q, k, v, causal, scale, Br, Bc):
+    """Block-by-block forward: running max, running sum and a running numerator that is
+    rescaled by exp(old max - new max) whenever a key block raises the max; tiles wholly
+    above the diagonal are skipped and the diagonal tile is masked element-wise."""
+    N, d = q.shape
+    o = np.zeros((N, d))
+    lse = np.zeros(N)
+    for r0 in range(0, N, Br):
+        rows = range(r0, min(r0 + Br, N))
+        m = np.full(len(rows), -np.inf)
+        l = np.zeros(len(rows))
+        acc = np.zeros((len(rows), d))
+        for c0 in range(0, N, Bc):
+            if causal and c0 > rows[-1]:
+                break  # tile entirely above the diagonal
+            cols = np.arange(c0, min(c0 + Bc, N))
+            s = scale * (q[list(rows)] @ k[cols].T)
+            if causal:
+                s = np.where(cols[None, :] <= np.array(list(rows))[:, None], s, -np.inf)
+            bm = s.max(axis=1)
+            mn = np.maximum(m, bm)
+            alpha = np.where(np.isneginf(m), 0.0, np.exp(m - mn))
+            p = np.exp(s - mn[:, None])
+            l = l * alpha + p.sum(axis=1)
+            acc = acc * alpha[:, None] + p @ v[cols]
+            m = mn
+        o[list(rows)] = acc / l[:, None]
+        lse[list(rows)] = m + np.log(l)
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Br,Bc", [(1, 1), (2, 2), (3, 5), (16, 16), (128, 128)])
+def test_tiled_online_forward_equals_oracle(causal, Br, Bc):
+    r = _rng(7)
+    N, d, scale = 37, 8, 0.35
+    q = 4 * r.standard_normal((N, d))
+    k = r.standard_normal((N, d))
+    v = r.standard_normal((N, d))
+    o_t, lse_t = _tiled_forward(q, k, v, causal, scale, Br, Bc)
+    o, lse = oracle.attention_fwd(q[None, None], k[None, None], v[None, None], causal, scale)
+    np.testing.assert_allclose(o[0, 0], o_t, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], lse_t, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------------------------- backward
+
+
+def _loss(q, k, v, do, causal, scale):
+    o, _ = oracle.attention_fwd(q, k, v, causal, scale)
+    return float(np.sum(o * do))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(1, 2), (5, 3), (7, 4)])
+def test_gradients_match_central_differences(causal, N, d):
+    r = _rng(100 + N * 10 + d + int(causal))
+    B, Hq, Hkv, scale = 1, 2, 1, 0.6
+    q = r.standard_normal((B, Hq, N, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    do = r.standard_normal((B, Hq, N, d))
+    dq, dk, dv, _, _ = oracle.attention_bwd(q, k, v, do, causal, scale)
+    h = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp = x.copy()
+            xp[idx] += h
+            xm = x.copy()
+            xm[idx] -= h
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], do, causal, scale)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], do, causal, scale)
+            num[idx] = (lp - lm) / (2 * h)
+        err = np.linalg.norm(grad - num) / max(np.linalg.norm(num), 1e-30)
+        assert err < 1e-6 or np.linalg.norm(grad - num) < 1e-8, (name, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_delta_equals_do_dot_o_and_lse_matches_forward(causal):
+    r = _rng(8)
+    B, Hq, Hkv, N, d, scale = 2, 4, 2, 23, 8, 0.3
+    q = r.standard_normal((B, Hq, N, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    do = r.standard_normal((B, Hq, N, d))
+    o, lse_f = oracle.attention_fwd(q, k, v, causal, scale)
+    _, _, _, lse_b, delta = oracle.attention_bwd(q, k, v, do, causal, scale)
+    np.testing.assert_allclose(delta, np.sum(o * do, axis=-1), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(lse_b, lse_f, rtol=0, atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gradient_column_sum_invariants(causal):
+    r = _rng(9)
+    B, Hq, Hkv, N, d, scale = 2, 6, 2, 19, 8, 0.4
+    q = 2 * r.standard_normal((B, Hq, N, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    do = r.standard_normal((B, Hq, N, d))
+    _, dk, dv, _, _ = oracle.attention_bwd(q, k, v, do, causal, scale)
+    g = Hq // Hkv
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    group_do = do.reshape(B, Hkv, g, N, d).sum(axis=(2, 3))
+    np.testing.assert_allclose(dv.sum(axis=2), group_do, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_equals_mha_with_repeated_kv(causal):
+    r = _rng(10)
+    B, Hq, Hkv, N, d, scale = 2, 8, 2, 17, 8, 0.3
+    g = Hq // Hkv
+    q = r.standard_normal((B, Hq, N, d))
+    k = r.standard_normal((B, Hkv, N, d))
+    v = r.standard_normal((B, Hkv, N, d))
+    do = r.standard_normal((B, Hq, N, d))
+    kr, vr = np.repeat(k, g, axis=1), np.repeat(v, g, axis=1)
+    o1, l1 = oracle.attention_fwd(q, k, v, causal, scale)
+    o2, l2 = oracle.attention_fwd(q, kr, vr, causal, scale)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-14)
+    dq1, dk1, dv1, _, _ = oracle.attention_bwd(q, k, v, do, causal, scale)
+    dq2, dk2, dv2, _, _ = oracle.attention_bwd(q, kr, vr, do, causal, scale)
+    np.testing.assert_allclose(dq1, dq2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dk1, dk2.reshape(B, Hkv, g, N, d).sum(2), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dv1, dv2.reshape(B, Hkv, g, N, d).sum(2), rtol=1e-12, atol=1e-12)
+
+
+def test_causal_differs_from_full_only_through_the_mask():
+    # Row N-1 of a causal attention sees every key, so it equals the non-causal row.
+    r = _rng(11)
+    q, k, v = (r.standard_normal((1, 1, 12, 4)) for _ in range(3))
+    oc, lc = oracle.attention_fwd(q, k, v, True, 0.5)
+    of, lf = oracle.attention_fwd(q, k, v, False, 0.5)
+    np.testing.assert_array_equal(oc[0, 0, -1], of[0, 0, -1])
+    assert lc[0, 0, -1] == lf[0, 0, -1]
+    assert not np.allclose(oc[0, 0, 0], of[0, 0, 0])
+
+
+def test_invalid_arguments_are_rejected():
+    q = np.zeros((1, 3, 4, 2))
+    k = np.zeros((1, 2, 4, 2))
+    with pytest.raises(RuntimeError):
+        oracle.attention_fwd(q, k, k, False, 1.0)  # Hq % Hkv != 0
+    with pytest.raises(ValueError):
+        oracle.attention_fwd(q, np.zeros((1, 1, 5, 2)), np.zeros((1, 1, 5, 2)), False, 1.0)
