@@ -1,0 +1,228 @@
+// fa_api.cu - host side of libfa_sm100.so: argument checks, TMA tensor maps, launches.
+//
+// The C entry points are declared (with their contracts) in include/fa.h.  This file is
+// the only translation unit of the library; the kernels are included from the .cuh
+// files beside it.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_common.cuh"
+#include "fa_fwd.cuh"
+#include "fa_fwd_d256.cuh"
+#include "fa_bwd.cuh"
+
+namespace {
+
+using fa::FwdParams;
+
+constexpr int kMaxDevices = 64;
+
+// cuTensorMapEncodeTiled, fetched once through the runtime so the library does not link
+// the driver library directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// Per-device capability check (sm_100) and one-time kernel attribute setup.
+struct DeviceState {
+  std::once_flag once;
+  bool ok = false;
+};
+DeviceState g_dev[kMaxDevices];
+
+template <typename K>
+bool set_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+bool device_ready() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  DeviceState &st = g_dev[dev];
+  std::call_once(st.once, [&] {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return;
+    if (major != 10 || minor != 0) return;  // sm_100a code only
+    bool ok = encode_fn() != nullptr;
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, false>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, true>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, false>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, true>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<false>, fa::FwdD256Layout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<true>, fa::FwdD256Layout::kSmemBytes);
+    ok = ok && fa::bwd_set_attributes();
+    st.ok = ok;
+  });
+  return st.ok;
+}
+
+// 3-D bf16 tensor map over [heads][N][d] with [rows x 64] boxes and 128-byte swizzle.
+bool make_map_bf16(CUtensorMap *m, const void *ptr, int d, int N, long long heads, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return FA_ERR_GQA;
+  // Row indices (b*H + h)*N + i must fit in int32 for the kernels' index arithmetic, and
+  // the grid size in int32.
+  const long long rows = static_cast<long long>(B) * Hq * N;
+  if (rows >= (1ll << 31) || static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_version(void) { return 100; }
+
+const char *fa_status_string(int code) {
+  switch (code) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported size (d must be 64, 128 or 256)";
+    case FA_ERR_GQA: return "Hq must be a multiple of Hkv";
+    case FA_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "workspace missing or too small";
+    case FA_ERR_CUDA: return "CUDA error (no sm_100 device or launch failure)";
+    case FA_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+           int N, int d, int causal, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+
+  const int box_rows = 128;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map_bf16(&tq, q, d, N, static_cast<long long>(B) * Hq, box_rows) ||
+      !make_map_bf16(&tk, k, d, N, static_cast<long long>(B) * Hkv, d == 256 ? 64 : box_rows) ||
+      !make_map_bf16(&tv, v, d, N, static_cast<long long>(B) * Hkv, d == 256 ? 64 : box_rows) ||
+      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, box_rows))
+    return FA_ERR_CUDA;
+
+  FwdParams p;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.nqb = (N + 127) / 128;
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int g = Hq / Hkv;
+
+  if (d == 256) {
+    p.pair_heads = 0;
+    const unsigned units = static_cast<unsigned>(B) * Hq * p.nqb;
+    if (causal)
+      fa::fa_fwd_d256_kernel<true><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
+          tq, tk, tv, to, p);
+    else
+      fa::fa_fwd_d256_kernel<false><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
+          tq, tk, tv, to, p);
+  } else {
+    p.pair_heads = (g % 2 == 0) ? 1 : 0;
+    const unsigned units = p.pair_heads
+                               ? static_cast<unsigned>(B) * (Hq / 2) * p.nqb
+                               : static_cast<unsigned>(B) * Hq * ((p.nqb + 1) / 2);
+    if (d == 64) {
+      if (causal)
+        fa::fa_fwd_kernel<64, true><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(
+            tq, tk, tv, to, p);
+      else
+        fa::fa_fwd_kernel<64, false><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(
+            tq, tk, tv, to, p);
+    } else {
+      if (causal)
+        fa::fa_fwd_kernel<128, true><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(
+            tq, tk, tv, to, p);
+      else
+        fa::fa_fwd_kernel<128, false><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(
+            tq, tk, tv, to, p);
+    }
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  if (check_sizes(B, Hq, Hkv, N, d, 1.0f) != FA_OK) return 0;
+  return fa::bwd_workspace_bytes(B, Hq, N, d);
+}
+
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dout, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+           int B, int Hq, int Hkv, int N, int d, int causal, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(B, Hq, N, d)) return FA_ERR_WORKSPACE;
+  const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, causal,
+                        scale, static_cast<cudaStream_t>(stream), encode_fn());
+}
+
+int fa_device_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpyFromSymbol(&status, fa::g_fa_status, sizeof(int)) != cudaSuccess) return FA_ERR_CUDA;
+  if (status != FA_OK) {
+    const int zero = 0;
+    const unsigned long long zero64 = 0;
+    if (cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(int)) != cudaSuccess ||
+        cudaMemcpyToSymbol(fa::g_fa_status_site, &zero64, sizeof(zero64)) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
+  return status;
+}
+
+}  // extern "C"

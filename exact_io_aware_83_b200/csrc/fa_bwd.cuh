@@ -1,0 +1,624 @@
+// fa_bwd.cuh - backward attention kernels for sm_100a.
+//
+// The pages require only that the backward pass recompute the attention tiles on chip
+// instead of storing them ("The Future of AI ..." page, bullet "Recomputation"; the
+// "FlashAttention1" Q&A, question on integration, item 6).  The gradient itself is the
+// plain calculus of L = <O, dO> for O = softmax(scale Q K^T) V:
+//   P_ij   = exp(scale q_i.k_j - LSE_i)             (recomputed from Q, K and the LSE)
+//   dP_ij  = do_i . v_j
+//   Delta_i = sum_j P_ij dP_ij = do_i . o_i
+//   dS_ij  = P_ij (dP_ij - Delta_i)
+//   dV_j   = sum_i P_ij do_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
+// (dK, dV summed over the query heads that share a K/V head).
+//
+// Three kernels on one stream:
+//  1. fa_bwd_pre:  Delta_i = <dO_i, O_i> (fp32) and a zeroed fp32 dQ accumulator.
+//  2. fa_bwd_main: one CTA per (b, K/V head, 128-key block).  It keeps K_j and V_j in
+//     shared memory and dK_j, dV_j in tensor memory, and walks every (query head of the
+//     group, 64-row query block) that can see the key block:
+//        S^T  = K Q_i^T        (tcgen05, TMEM)      P^T = exp2(S^T scale log2e - LSE2_i)
+//        dP^T = V dO_i^T       (tcgen05, TMEM)      dS^T = P^T (dP^T - Delta_i)
+//        dV  += P^T dO_i       (P^T read from TMEM as the A operand)
+//        dK  += dS^T Q_i       (dS^T from swizzled shared memory, K-major)
+//        dQ_i^T = K^T dS^T     (same dS^T tile read MN-major) -> fp32 TMA reduce-add
+//     Warps 0-3 own one key row each (P^T, dS^T, then the dK/dV epilogue); warps 4-7
+//     drain dQ^T from TMEM into the fp32 accumulator; warp 8 issues the MMAs; warp 9
+//     loads (TMA for K, V, Q_i, dO_i; plain loads for LSE_i and Delta_i).
+//  3. fa_bwd_post: dQ = bf16(scale * dQacc).
+// For d = 256 the two K/V accumulators would need all 512 TMEM columns, so two CTAs
+// share each key block, each owning one 128-column half of dK, dV and dQ (both
+// recompute S^T and dP^T over the full d), with 32-row query blocks so the tiles fit.
+#pragma once
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+// ============================================================================ pre / post
+
+template <int D>
+__global__ void __launch_bounds__(256)
+    fa_bwd_pre_kernel(const __nv_bfloat16 *__restrict__ o, const __nv_bfloat16 *__restrict__ dout,
+                      float *__restrict__ delta, float *__restrict__ dqacc, long long rows) {
+  constexpr int kPer = D / 32;  // bf16 elements per lane
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  if (row >= rows) return;
+  const __nv_bfloat16 *orow = o + row * D + lane * kPer;
+  const __nv_bfloat16 *drow = dout + row * D + lane * kPer;
+  float acc = 0.f;
+  if constexpr (kPer == 2) {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162 *>(orow);
+    const __nv_bfloat162 c = *reinterpret_cast<const __nv_bfloat162 *>(drow);
+    acc = __bfloat162float(a.x) * __bfloat162float(c.x) + __bfloat162float(a.y) * __bfloat162float(c.y);
+  } else {
+    constexpr int kVec = kPer / 4;  // 8-byte vectors
+#pragma unroll
+    for (int v = 0; v < kVec; ++v) {
+      const uint2 a = reinterpret_cast<const uint2 *>(orow)[v];
+      const uint2 c = reinterpret_cast<const uint2 *>(drow)[v];
+      const __nv_bfloat162 *a2 = reinterpret_cast<const __nv_bfloat162 *>(&a);
+      const __nv_bfloat162 *c2 = reinterpret_cast<const __nv_bfloat162 *>(&c);
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        acc += __bfloat162float(a2[e].x) * __bfloat162float(c2[e].x) +
+               __bfloat162float(a2[e].y) * __bfloat162float(c2[e].y);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) delta[row] = acc;
+  float *qrow = dqacc + row * D;
+#pragma unroll
+  for (int c = lane * 4; c < D; c += 128)
+    *reinterpret_cast<float4 *>(qrow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+__global__ void __launch_bounds__(256)
+    fa_bwd_post_kernel(const float *__restrict__ dqacc, __nv_bfloat16 *__restrict__ dq, float scale,
+                       long long n8) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4 *>(dqacc)[2 * i];
+  const float4 c = reinterpret_cast<const float4 *>(dqacc)[2 * i + 1];
+  uint4 w;
+  w.x = pack_bf16x2(a.x * scale, a.y * scale);
+  w.y = pack_bf16x2(a.z * scale, a.w * scale);
+  w.z = pack_bf16x2(c.x * scale, c.y * scale);
+  w.w = pack_bf16x2(c.z * scale, c.w * scale);
+  reinterpret_cast<uint4 *>(dq)[i] = w;
+}
+
+// ============================================================================ main kernel
+
+struct BwdParams {
+  const float *lse;    // [B, Hq, N]
+  const float *delta;  // [B, Hq, N]
+  int B, Hq, Hkv, N;
+  int nkb;             // key blocks of 128
+  float sl2;           // scale * log2(e)
+  float scale;
+};
+
+// D: head dimension (contraction of S^T and dP^T); DH: output columns owned by a CTA
+// (D, or 128 when D = 256); BQ: query rows per step.
+template <int D, int DH, int BQ>
+struct BwdLayout {
+  static constexpr int kKRows = 128;
+  static constexpr int kChunks = D / 64;
+  static constexpr int kKChunk = kKRows * 128;      // [128 x 64] bf16 box
+  static constexpr int kKTile = kChunks * kKChunk;
+  static constexpr int kQChunk = BQ * 128;          // [BQ x 64] bf16 box
+  static constexpr int kQTile = kChunks * kQChunk;
+  static constexpr int kQStages = 2;
+  static constexpr int kDSRowBytes = 128;           // dS^T rows padded to one 128-B swizzle row
+  static constexpr int kDSBytes = kKRows * kDSRowBytes;
+  static constexpr int kDQHalves = (BQ * DH * 4 > 32768) ? 2 : 1;  // dQ staging passes
+  static constexpr int kDQCols = DH / kDQHalves;    // d columns staged per pass
+  static constexpr int kDQBytes = BQ * kDQCols * 4;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKTile;
+  static constexpr int kOffQ = kOffV + kKTile;                // Q ring
+  static constexpr int kOffDO = kOffQ + kQStages * kQTile;    // dO ring
+  static constexpr int kOffDS = kOffDO + kQStages * kQTile;
+  static constexpr int kOffDQ = kOffDS + kDSBytes;
+  static constexpr int kOffVec = kOffDQ + kDQBytes;           // [stage][lse2 | delta][BQ] fp32
+  static constexpr int kVecBytes = kQStages * 2 * BQ * 4;
+  static constexpr int kOffBar = kOffVec + kVecBytes;
+  // mbarriers
+  static constexpr int kBarKV = 0;
+  static constexpr int kBarQFull = 1;
+  static constexpr int kBarQEmpty = kBarQFull + kQStages;
+  static constexpr int kBarS = kBarQEmpty + kQStages;
+  static constexpr int kBarDP = kBarS + 1;
+  static constexpr int kBarP = kBarDP + 1;
+  static constexpr int kBarDS = kBarP + 1;
+  static constexpr int kBarDSEmpty = kBarDS + 1;
+  static constexpr int kBarDQ = kBarDSEmpty + 1;
+  static constexpr int kBarDQEmpty = kBarDQ + 1;
+  static constexpr int kBarFinal = kBarDQEmpty + 1;
+  static constexpr int kBarDrain = kBarFinal + 1;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // tensor memory: dV | dK | S^T | dP^T | dQ^T
+  static constexpr uint32_t kTmDV = 0;
+  static constexpr uint32_t kTmDK = DH;
+  static constexpr uint32_t kTmS = 2 * DH;
+  static constexpr uint32_t kTmDP = 2 * DH + BQ;
+  static constexpr uint32_t kTmDQ = 2 * DH + 2 * BQ;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kTmDQ + BQ <= 512, "tensor-memory budget");
+  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(BQ == 32 || BQ == 64, "query block");
+};
+
+constexpr int kBwdThreads = 320;
+
+template <int D, int DH, int BQ, bool CAUSAL>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                       const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
+  using L = BwdLayout<D, DH, BQ>;
+  constexpr int QS = L::kQStages;
+  constexpr int kHalves = D / DH;  // CTAs per key block
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+  float *vec = reinterpret_cast<float *>(smem + L::kOffVec);
+  auto bar = [&](int i) -> uint32_t { return base + L::kOffBar + 8u * static_cast<uint32_t>(i); };
+  const uint32_t sK = base + L::kOffK, sV = base + L::kOffV;
+  const uint32_t sQ = base + L::kOffQ, sDO = base + L::kOffDO;
+  const uint32_t sDS = base + L::kOffDS, sDQ = base + L::kOffDQ;
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- unit: (b, kv head, key block, d half); heaviest causal key blocks first
+  int u = blockIdx.x;
+  const int half = u % kHalves;
+  u /= kHalves;
+  const int kb = u % p.nkb;
+  u /= p.nkb;
+  const int kvh = u % p.Hkv;
+  const int b = u / p.Hkv;
+  const int g = p.Hq / p.Hkv;
+  const int nqb = (p.N + BQ - 1) / BQ;
+  const int q_first = CAUSAL ? (kb * 128) / BQ : 0;
+  const int nq = nqb - q_first;
+  const int T = g * nq;  // steps: (query head of the group, query block)
+  const int kv0 = kb * 128;
+  const int dcol0 = half * DH;  // first output column owned by this CTA
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i) {
+      uint32_t cnt = 1;
+      if (i == L::kBarP || i == L::kBarDS || i == L::kBarDQEmpty) cnt = 128;
+      mbar_init(bar(i), cnt);
+    }
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), L::kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = misc[0];
+
+  auto step_head = [&](int i) { return kvh * g + i / nq; };
+  auto step_q0 = [&](int i) { return (q_first + i % nq) * BQ; };
+
+  if (warp == 9) {
+    // ================================================================ loader
+    bool ok = true;
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKTile);
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c) {
+        tma_load_3d(sK + c * L::kKChunk, &tm_k, bar(L::kBarKV), c * 64, kv0, b * p.Hkv + kvh);
+        tma_load_3d(sV + c * L::kKChunk, &tm_v, bar(L::kBarKV), c * 64, kv0, b * p.Hkv + kvh);
+      }
+    }
+    int issued = 0;
+    for (int i = 0; ok && i < T; ++i) {
+      const int st = i % QS, use = i / QS;
+      ok = warp_wait_bounded(bar(L::kBarQEmpty + st), (use & 1) ^ 1, abort_flag,
+                             wait_site(3, L::kBarQEmpty + st, i));
+      if (!ok) break;
+      const int h = step_head(i), q0 = step_q0(i);
+      const size_t rowbase = static_cast<size_t>(b * p.Hq + h) * p.N;
+      float *lse2 = vec + (st * 2) * BQ;
+      float *dl = vec + (st * 2 + 1) * BQ;
+      for (int c = lane; c < BQ; c += 32) {
+        const int q = q0 + c;
+        // Query rows past N get LSE = +inf, so their probabilities are exactly 0.
+        lse2[c] = q < p.N ? p.lse[rowbase + q] * 1.4426950408889634f : INFINITY;
+        dl[c] = q < p.N ? p.delta[rowbase + q] : 0.f;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar(L::kBarQFull + st), 2 * L::kQTile);
+#pragma unroll
+        for (int c = 0; c < L::kChunks; ++c) {
+          tma_load_3d(sQ + st * L::kQTile + c * L::kQChunk, &tm_q, bar(L::kBarQFull + st), c * 64, q0,
+                      b * p.Hq + h);
+          tma_load_3d(sDO + st * L::kQTile + c * L::kQChunk, &tm_do, bar(L::kBarQFull + st), c * 64, q0,
+                      b * p.Hq + h);
+        }
+      }
+      ++issued;
+    }
+    if (lane == 0) {
+      for (int i = issued > QS ? issued - QS : 0; i < issued; ++i)
+        wait_drain(bar(L::kBarQFull + i % QS), (i / QS) & 1, 100000000ull);
+      wait_drain(bar(L::kBarKV), 0, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_st = idesc_bf16_f32(128, BQ, 0, 0);   // S^T, dP^T
+      constexpr uint32_t id_kv = idesc_bf16_f32(128, DH, 0, 1);   // dV, dK (B = dO / Q, MN-major)
+      constexpr uint32_t id_dq = idesc_bf16_f32(128, BQ, 1, 1);   // dQ^T = K^T dS^T
+      // S^T (or dP^T) = A B^T over d: A = K (or V) [128 x D], B = Q_i (or dO_i) [BQ x D].
+      auto issue_st = [&](uint32_t dst, uint32_t a0, uint32_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t oa = (kk / 4) * L::kKChunk + (kk % 4) * 32;
+          const uint32_t ob = (kk / 4) * L::kQChunk + (kk % 4) * 32;
+          mma_ss(tmem + dst, sdesc_sw128(a0 + oa, 16, 1024), sdesc_sw128(b0 + ob, 16, 1024), id_st, kk > 0);
+        }
+      };
+      bool ok = wait_bounded(bar(L::kBarKV), 0, abort_flag, wait_site(3, L::kBarKV, 0));
+      if (ok) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
+      if (ok) {
+        tc_fence_after_sync();
+        issue_st(L::kTmS, sK, sQ);
+        tc_commit(bar(L::kBarS));
+        issue_st(L::kTmDP, sV, sDO);
+        tc_commit(bar(L::kBarDP));
+      }
+      for (int i = 0; ok && i < T; ++i) {
+        const int st = i % QS;
+        const uint32_t q_t = sQ + st * L::kQTile, do_t = sDO + st * L::kQTile;
+        // dV += P^T dO_i : M = 128 keys, N = DH, K = BQ queries; P^T (bf16) in TMEM.
+        if (!(ok = wait_bounded(bar(L::kBarP), i & 1, abort_flag, wait_site(3, L::kBarP, i)))) break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ts(tmem + L::kTmDV, tmem + L::kTmS + kk * 8,
+                 sdesc_sw128(do_t + (dcol0 / 64) * L::kQChunk + kk * 2048, L::kQChunk, 1024), id_kv,
+                 (i > 0 || kk > 0));
+        // Next step's S^T can start as soon as P^T has been consumed (issue order).
+        if (i + 1 < T) {
+          const int st1 = (i + 1) % QS;
+          if (!(ok = wait_bounded(bar(L::kBarQFull + st1), ((i + 1) / QS) & 1, abort_flag,
+                                  wait_site(3, L::kBarQFull + st1, i + 1))))
+            break;
+          tc_fence_after_sync();
+          issue_st(L::kTmS, sK, sQ + st1 * L::kQTile);
+          tc_commit(bar(L::kBarS));
+        }
+        // dK += dS^T Q_i : M = 128 keys, N = DH, K = BQ; dS^T K-major in shared memory.
+        if (!(ok = wait_bounded(bar(L::kBarDS), i & 1, abort_flag, wait_site(3, L::kBarDS, i)))) break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < BQ / 16; ++kk)
+          mma_ss(tmem + L::kTmDK, sdesc_sw128(sDS + kk * 32, 16, 1024),
+                 sdesc_sw128(q_t + (dcol0 / 64) * L::kQChunk + kk * 2048, L::kQChunk, 1024), id_kv,
+                 (i > 0 || kk > 0));
+        // dQ_i^T = K^T dS^T : M = 128 d columns, N = BQ, K = 128 keys; both MN-major.
+        if (!(ok = wait_bounded(bar(L::kBarDQEmpty), (i & 1) ^ 1, abort_flag,
+                                wait_site(3, L::kBarDQEmpty, i))))
+          break;
+        tc_fence_after_sync();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ss(tmem + L::kTmDQ, sdesc_sw128(sK + (dcol0 / 64) * L::kKChunk + kk * 2048, L::kKChunk, 1024),
+                 sdesc_sw128(sDS + kk * 2048, 128 * 128, 1024), id_dq, kk > 0);
+        tc_commit(bar(L::kBarDQ));
+        tc_commit(bar(L::kBarDSEmpty));
+        tc_commit(bar(L::kBarQEmpty + st));
+        if (i + 1 < T) {
+          issue_st(L::kTmDP, sV, sDO + ((i + 1) % QS) * L::kQTile);
+          tc_commit(bar(L::kBarDP));
+        }
+      }
+      if (ok) tc_commit(bar(L::kBarFinal));
+      tc_commit(bar(L::kBarDrain));
+      wait_drain(bar(L::kBarDrain), 0, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ================================================================ P^T / dS^T (one key row per thread)
+    const int r = warp * 32 + lane;
+    const int kv = kv0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tS = tmem + L::kTmS + lane_off;
+    const uint32_t tDP = tmem + L::kTmDP + lane_off;
+    const bool row_live = kv < p.N;
+    const float sl2 = p.sl2;
+    bool ok = true;
+    for (int i = 0; ok && i < T; ++i) {
+      const int st = i % QS;
+      const int q0 = step_q0(i);
+      if (!(ok = warp_wait_bounded(bar(L::kBarQFull + st), (i / QS) & 1, abort_flag,
+                                   wait_site(3, L::kBarQFull + st, i))))
+        break;
+      if (!(ok = warp_wait_bounded(bar(L::kBarS), i & 1, abort_flag, wait_site(3, L::kBarS, i)))) break;
+      tc_fence_after_sync();
+      const float *lse2 = vec + (st * 2) * BQ;
+      const float *dl = vec + (st * 2 + 1) * BQ;
+      float pr[BQ];
+#pragma unroll
+      for (int c0 = 0; c0 < BQ; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld_x32(tS + c0, rr);
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          pr[c0 + c] = ex2_approx(fmaf(__uint_as_float(rr[c]), sl2, -lse2[c0 + c]));
+      }
+      // Masks: key rows past N, and (causal) queries before this key.
+      if (!row_live) {
+#pragma unroll
+        for (int c = 0; c < BQ; ++c) pr[c] = 0.f;
+      } else if (CAUSAL && q0 < kv) {
+#pragma unroll
+        for (int c = 0; c < BQ; ++c)
+          if (q0 + c < kv) pr[c] = 0.f;
+      }
+      {
+        uint32_t pk[BQ / 2];
+#pragma unroll
+        for (int c = 0; c < BQ / 2; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+        if constexpr (BQ == 64) {
+          tmem_st_x32(tS, pk);
+        } else {
+          tmem_st_x16(tS, pk);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(bar(L::kBarP));
+
+      if (!(ok = warp_wait_bounded(bar(L::kBarDP), i & 1, abort_flag, wait_site(3, L::kBarDP, i)))) break;
+      tc_fence_after_sync();
+      uint32_t dsk[BQ / 2];
+#pragma unroll
+      for (int c0 = 0; c0 < BQ; c0 += 32) {
+        uint32_t rr[32];
+        tmem_ld_x32(tDP + c0, rr);
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float d0 = pr[c0 + c] * (__uint_as_float(rr[c]) - dl[c0 + c]);
+          const float d1 = pr[c0 + c + 1] * (__uint_as_float(rr[c + 1]) - dl[c0 + c + 1]);
+          dsk[(c0 + c) / 2] = pack_bf16x2(d0, d1);
+        }
+      }
+      // dS^T row r -> shared memory (128-byte swizzled row; BQ * 2 bytes used).
+      if (!(ok = warp_wait_bounded(bar(L::kBarDSEmpty), (i & 1) ^ 1, abort_flag,
+                                   wait_site(3, L::kBarDSEmpty, i))))
+        break;
+      const uint32_t rowp = sDS + r * 128;
+#pragma unroll
+      for (int uu = 0; uu < BQ / 8; ++uu)
+        st_shared_v4(rowp + ((uu ^ (r & 7)) * 16), dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2],
+                     dsk[4 * uu + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(bar(L::kBarDS));
+    }
+
+    // ---- epilogue: dV, then scale * dK -> bf16 -> shared (reusing the V / K tiles) -> TMA
+    bool okw = ok && warp_wait_bounded(bar(L::kBarFinal), 0, abort_flag, wait_site(3, L::kBarFinal, 0));
+    okw = named_bar_and(1, 128, okw && *abort_flag == 0);
+    if (okw) {
+      tc_fence_after_sync();
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tacc = tmem + (which ? L::kTmDK : L::kTmDV) + lane_off;
+        const float mul = which ? p.scale : 1.f;
+        const uint32_t stage = which ? sK : sV;
+#pragma unroll
+        for (int cc = 0; cc < DH / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld_x32(tacc + cc * 32, o);
+          const uint32_t rowbase = stage + (cc / 2) * L::kKChunk + r * 128;
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            const int unit = (cc % 2) * 4 + uu;
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * mul,
+                                 __uint_as_float(o[8 * uu + 2 * e + 1]) * mul);
+            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (r == 0) {
+#pragma unroll
+        for (int c = 0; c < DH / 64; ++c) {
+          tma_store_3d(&tm_dv, sV + c * L::kKChunk, dcol0 + c * 64, kv0, b * p.Hkv + kvh);
+          tma_store_3d(&tm_dk, sK + c * L::kKChunk, dcol0 + c * 64, kv0, b * p.Hkv + kvh);
+        }
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+    }
+  } else {
+    // ================================================================ dQ^T drain (warps 4-7)
+    const int wq = warp - 4;
+    const int dl = wq * 32 + lane;  // d column (TMEM lane) within this CTA's half
+    const uint32_t tDQ = tmem + L::kTmDQ + (static_cast<uint32_t>(wq * 32) << 16);
+    const bool lane_live = dl < DH;  // d = 64 pads M to 128; upper lanes are junk
+    float *stage = reinterpret_cast<float *>(smem + L::kOffDQ);
+    const int tid = threadIdx.x - 128;
+    bool ok = true;
+    for (int i = 0; ok && i < T; ++i) {
+      // The warpgroup leaves the loop together: the named barriers below need all four warps.
+      ok = warp_wait_bounded(bar(L::kBarDQ), i & 1, abort_flag, wait_site(3, L::kBarDQ, i));
+      if (!(ok = named_bar_and(2, 128, ok))) break;
+      tc_fence_after_sync();
+      float acc[BQ];
+      if (wq * 32 < DH) {
+#pragma unroll
+        for (int c0 = 0; c0 < BQ; c0 += 32) {
+          uint32_t rr[32];
+          tmem_ld_x32(tDQ + c0, rr);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) acc[c0 + c] = __uint_as_float(rr[c]);
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(bar(L::kBarDQEmpty));
+      const int h = step_head(i), q0 = step_q0(i);
+#pragma unroll
+      for (int hp = 0; hp < L::kDQHalves; ++hp) {
+        // The previous reduce must have finished reading the staging buffer.
+        if (tid == 0) bulk_wait_group_read0();
+        named_bar_sync(2, 128);
+        const int cl = dl - hp * L::kDQCols;  // column within this pass
+        if (lane_live && cl >= 0 && cl < L::kDQCols) {
+#pragma unroll
+          for (int c = 0; c < BQ; ++c) stage[c * L::kDQCols + cl] = acc[c];
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(2, 128);
+        if (tid == 0) {
+          tma_reduce_add_3d(&tm_dqacc, sDQ, dcol0 + hp * L::kDQCols, q0, b * p.Hq + h);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (tid == 0) bulk_wait_group0();
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ============================================================================ host side
+
+inline size_t pad256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d) {
+  const size_t rows = static_cast<size_t>(B) * Hq * N;
+  return pad256(rows * 4) + pad256(rows * static_cast<size_t>(d) * 4);
+}
+
+template <int D, int DH, int BQ, bool CAUSAL>
+inline bool bwd_set_attr_one() {
+  return cudaFuncSetAttribute(fa_bwd_main_kernel<D, DH, BQ, CAUSAL>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              BwdLayout<D, DH, BQ>::kSmemBytes) == cudaSuccess;
+}
+
+inline bool bwd_set_attributes() {
+  return bwd_set_attr_one<64, 64, 64, false>() && bwd_set_attr_one<64, 64, 64, true>() &&
+         bwd_set_attr_one<128, 128, 64, false>() && bwd_set_attr_one<128, 128, 64, true>() &&
+         bwd_set_attr_one<256, 128, 32, false>() && bwd_set_attr_one<256, 128, 32, true>();
+}
+
+typedef CUresult (*EncodeTiledFnBwd)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                     const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                     const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                     CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline bool bwd_map(EncodeTiledFnBwd enc, CUtensorMap *m, const void *ptr, bool f32, int d, int N,
+                    long long heads, int box_cols, int box_rows) {
+  const cuuint64_t esz = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz,
+                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * esz};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             f32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int DH, int BQ, bool CAUSAL>
+inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                            const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
+                            const CUtensorMap &tdq, const BwdParams &p, unsigned grid, cudaStream_t s) {
+  fa_bwd_main_kernel<D, DH, BQ, CAUSAL><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
+      tq, tk, tv, tdo, tdk, tdv, tdq, p);
+}
+
+template <int D, int DH, int BQ>
+inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                        const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
+                        int Hkv, int N, int causal, float scale, cudaStream_t s, EncodeTiledFnBwd enc) {
+  const long long rows = static_cast<long long>(B) * Hq * N;
+  float *delta = static_cast<float *>(workspace);
+  float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
+  using L = BwdLayout<D, DH, BQ>;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
+  const long long hq = static_cast<long long>(B) * Hq, hkv = static_cast<long long>(B) * Hkv;
+  if (!bwd_map(enc, &tq, q, false, D, N, hq, 64, BQ) || !bwd_map(enc, &tdo, dout, false, D, N, hq, 64, BQ) ||
+      !bwd_map(enc, &tk, k, false, D, N, hkv, 64, 128) || !bwd_map(enc, &tv, v, false, D, N, hkv, 64, 128) ||
+      !bwd_map(enc, &tdk, dk, false, D, N, hkv, 64, 128) || !bwd_map(enc, &tdv, dv, false, D, N, hkv, 64, 128) ||
+      !bwd_map(enc, &tdq, dqacc, true, D, N, hq, L::kDQCols, BQ))
+    return FA_ERR_CUDA;
+
+  fa_bwd_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), delta, dqacc, rows);
+
+  BwdParams p;
+  p.lse = lse;
+  p.delta = delta;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.nkb = (N + 127) / 128;
+  p.scale = scale;
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
+  if (causal)
+    bwd_launch_main<D, DH, BQ, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+  else
+    bwd_launch_main<D, DH, BQ, false>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+
+  const long long n8 = rows * D / 8;
+  fa_bwd_post_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
+      dqacc, static_cast<__nv_bfloat16 *>(dq), scale, n8);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <typename Enc>
+inline int bwd_launch(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                      const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
+                      int Hkv, int N, int d, int causal, float scale, cudaStream_t s, Enc enc) {
+  const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
+  if (d == 64)
+    return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
+                                    scale, s, e);
+  if (d == 128)
+    return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
+                                      scale, s, e);
+  return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
+                                    scale, s, e);
+}
+
+}  // namespace fa

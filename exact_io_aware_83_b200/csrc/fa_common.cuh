@@ -1,0 +1,72 @@
+// fa_common.cuh - device status word and bounded pipeline waits shared by the kernels.
+//
+// Every wait on an mbarrier in the attention kernels is bounded in time.  When a wait
+// gives up, the kernel records FA_ERR_DEVICE_TIMEOUT (plus a site code) in the device
+// status word, raises a per-CTA abort flag in shared memory so that every other role
+// stops waiting too, and all roles drain to the common exit, where tensor memory is
+// released.  The host reads and clears the word with fa_device_status().
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "fa.h"
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+// A single pipeline wait never legitimately takes more than microseconds; two seconds
+// only trips on a broken pipeline.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// Device status word (FA_OK or FA_ERR_DEVICE_TIMEOUT) and the site of the first failure:
+// bits 0..15 iteration, 16..23 barrier id, 24..31 kernel id, 32..63 blockIdx.x.
+__device__ int g_fa_status;
+__device__ unsigned long long g_fa_status_site;
+
+__device__ __forceinline__ uint32_t wait_site(uint32_t kernel, uint32_t barrier, uint32_t iter) {
+  return (kernel << 24) | ((barrier & 0xFFu) << 16) | (iter & 0xFFFFu);
+}
+
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                       uint32_t site) {
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      if (atomicCAS(&g_fa_status, FA_OK, FA_ERR_DEVICE_TIMEOUT) == FA_OK)
+        atomicExch(&g_fa_status_site,
+                   static_cast<unsigned long long>(site) |
+                       (static_cast<unsigned long long>(blockIdx.x) << 32));
+      return false;
+    }
+  }
+}
+
+// Wait for the phase of `bar` with parity `parity`; false if the wait gave up (or another
+// role of this CTA already did).
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile int *abort_flag, uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_slow(bar, parity, abort_flag, site);
+}
+
+// The same for all 32 lanes of a warp: every lane waits, and the warp proceeds only if
+// every lane saw the phase complete, so warp-collective tcgen05 instructions that follow
+// are never reached by part of a warp.
+__device__ __forceinline__ bool warp_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  volatile int *abort_flag, uint32_t site) {
+  const bool ok = wait_bounded(bar, parity, abort_flag, site);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Best-effort wait used while draining after an abort: time-bounded, ignores the flag.
+__device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > limit_ns) return;
+  }
+}
+
+}  // namespace fa

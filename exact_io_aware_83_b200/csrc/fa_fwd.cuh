@@ -1,0 +1,405 @@
+// fa_fwd.cuh - forward attention kernel for head dimensions 64 and 128 on sm_100a.
+//
+// What it computes (per query row i of head h, keys j in J(i)):
+//   O_i = sum_j softmax_j(scale * q_i . k_j) v_j,  LSE_i = ln sum_j exp(scale * q_i . k_j)
+// with the score matrix processed one 128 x 128 tile at a time and the online-softmax
+// recurrence of the "FlashAttention1" Q&A page (question on computing the softmax,
+// items 1-3): a running row maximum m, a running sum l, and a rescale of the partial
+// output by exp(m_old - m_new) when a new key block raises the maximum (the deep-dive
+// page's "Intuition" for merging blocks).  Nothing N x N is written to memory (the
+// "Tiling" bullet of the FlashAttention-2 page).
+//
+// B200 design (not the pages' A100 one):
+//  * One CTA owns two 128-row query tiles that share every K/V block: either two query
+//    blocks of one head, or - for grouped-query attention with an even group - the same
+//    query block of two heads that share a K/V head, so each K/V tile is loaded once for
+//    both.  Work units are ordered so the longest causal units start first.
+//  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and tile 1
+//    (one query row per thread, the row's TMEM lane); warp 8 allocates tensor memory and
+//    issues every tcgen05.mma from one lane; warp 9 issues the TMA loads from one lane.
+//  * Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  S = Q K^T lands in TMEM as
+//    fp32; the softmax warps read it, write P as bf16 over the first half of the same
+//    columns, and the MMA warp computes O += P V with P taken straight from TMEM.
+//  * K and V blocks stream through a ring of shared-memory slots filled by TMA in the
+//    order K_0, V_0, K_1, V_1, ...; 128-byte swizzled tiles feed the tensor core directly.
+//  * The two tiles ping-pong: while the softmax warps of one tile work, the tensor core
+//    runs the other tile's P V and next Q K^T.
+//  * exp is evaluated as exp2 with scale*log2(e) folded into one FMA.  The running max
+//    used as the exponent offset is only moved when a row's max rises by more than 2^8
+//    (the recurrence is exact for any offset; keeping it avoids rescaling O for most
+//    blocks).
+#pragma once
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  float *lse;       // [B, Hq, N] fp32
+  int B, Hq, Hkv, N;
+  int nqb;          // 128-row blocks per sequence, ceil(N / 128)
+  int pair_heads;   // 1: a unit is (2 heads, 1 query block); 0: (1 head, 2 query blocks)
+  float sl2;        // scale * log2(e)
+};
+
+constexpr float kLn2 = 0.693147180559945309f;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kRows = 128;                // query rows per tile = keys per block
+  static constexpr int kChunks = D / 64;           // 128-byte swizzle chunks per row
+  static constexpr int kChunkBytes = kRows * 128;  // one [128 x 64] bf16 TMA box
+  static constexpr int kTileBytes = kChunks * kChunkBytes;
+  static constexpr int kStages = (D == 64) ? 6 : 4;  // K/V ring slots
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kTileBytes;
+  // mbarriers: q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] drain
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKVFull = 2;
+  static constexpr int kBarKVEmpty = kBarKVFull + kStages;
+  static constexpr int kBarS = kBarKVEmpty + kStages;
+  static constexpr int kBarP = kBarS + 2;
+  static constexpr int kBarO = kBarP + 2;
+  static constexpr int kBarDrain = kBarO + 2;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-B alignment
+  static constexpr uint32_t kTmemCols = 512;
+  __host__ __device__ static constexpr uint32_t tm_s(int t) { return static_cast<uint32_t>(t) * 128u; }
+  __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t * D); }
+  static_assert(256 + 2 * D <= 512, "tensor-memory budget");
+  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+};
+
+constexpr int kFwdThreads = 320;
+
+template <int D, bool CAUSAL>
+__global__ void __maxnreg__(200)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                  const FwdParams p) {
+  using L = FwdLayout<D>;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  const uint32_t sQ = base + L::kOffQ;
+  const uint32_t sKV = base + L::kOffKV;
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+  auto bar = [&](int i) -> uint32_t { return base + L::kOffBar + 8u * static_cast<uint32_t>(i); };
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- which two query tiles this CTA owns
+  const int g = p.Hq / p.Hkv;
+  int b, h[2], qb[2];
+  bool valid[2];
+  {
+    int u = blockIdx.x;
+    if (p.pair_heads) {
+      const int hp_count = p.Hq / 2;
+      const int q = p.nqb - 1 - (u % p.nqb);
+      u /= p.nqb;
+      const int hp = u % hp_count;
+      b = u / hp_count;
+      h[0] = 2 * hp;
+      h[1] = 2 * hp + 1;
+      qb[0] = qb[1] = q;
+      valid[0] = valid[1] = true;
+    } else {
+      const int npairs = (p.nqb + 1) / 2;
+      const int pi = npairs - 1 - (u % npairs);
+      u /= npairs;
+      h[0] = h[1] = u % p.Hq;
+      b = u / p.Hq;
+      qb[0] = 2 * pi;
+      qb[1] = 2 * pi + 1;
+      valid[0] = true;
+      valid[1] = qb[1] < p.nqb;
+    }
+  }
+  const int kvh = h[0] / g;
+  int nblk[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) nblk[t] = !valid[t] ? 0 : (CAUSAL ? qb[t] + 1 : p.nqb);
+  const int nmax = nblk[0] > nblk[1] ? nblk[0] : nblk[1];
+
+  // ---- barriers and tensor memory
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i)
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? 128u : 1u);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(misc), L::kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 9) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_o);
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (!valid[t]) continue;
+        mbar_arrive_expect_tx(bar(L::kBarQ + t), L::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tm_q, bar(L::kBarQ + t), c * 64,
+                      qb[t] * 128, b * p.Hq + h[t]);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int j = 0; ok && j < nmax; ++j) {
+#pragma unroll
+        for (int kind = 0; kind < 2; ++kind) {
+          const int seq = 2 * j + kind, slot = seq % S, use = seq / S;
+          if (!wait_bounded(bar(L::kBarKVEmpty + slot), (use & 1) ^ 1, abort_flag,
+                            wait_site(1, L::kBarKVEmpty + slot, j))) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kTileBytes);
+          const CUtensorMap *m = kind ? &tm_v : &tm_k;
+#pragma unroll
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_load_3d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, m, bar(L::kBarKVFull + slot),
+                        c * 64, j * 128, b * p.Hkv + kvh);
+          ++issued;
+        }
+      }
+      // No copy may still be landing in shared memory when the CTA exits.
+      for (int seq = issued > S ? issued - S : 0; seq < issued; ++seq)
+        wait_drain(bar(L::kBarKVFull + seq % S), (seq / S) & 1, 100000000ull);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (valid[t]) wait_drain(bar(L::kBarQ + t), 0, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      auto kslot = [](int j) { return (2 * j) % S; };
+      auto kpar = [](int j) { return static_cast<uint32_t>(((2 * j) / S) & 1); };
+      auto vslot = [](int j) { return (2 * j + 1) % S; };
+      auto vpar = [](int j) { return static_cast<uint32_t>(((2 * j + 1) / S) & 1); };
+      // S_t = Q_t K_j^T : M = 128 query rows, N = 128 keys, K = D (16 per instruction).
+      auto issue_qk = [&](int t, int j) {
+        const uint32_t a0 = sQ + t * L::kTileBytes;
+        const uint32_t b0 = sKV + kslot(j) * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * L::kChunkBytes + (kk % 4) * 32;
+          mma_ss(tmem + L::tm_s(t), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
+                 idesc_qk, kk > 0);
+        }
+      };
+      // O_t += P_t V_j : M = 128 query rows, N = D, K = 128 keys; P (bf16) in TMEM,
+      // V MN-major in shared memory (16 key rows = 2048 bytes per instruction).
+      auto issue_pv = [&](int t, int j) {
+        const uint32_t b0 = sKV + vslot(j) * L::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + L::tm_o(t), tmem + L::tm_s(t) + kk * 8,
+                 sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (j > 0 || kk > 0));
+      };
+
+      bool ok = true;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+        if (ok && valid[t]) ok = wait_bounded(bar(L::kBarQ + t), 0, abort_flag, wait_site(1, L::kBarQ + t, 0));
+      if (ok) ok = wait_bounded(bar(L::kBarKVFull + kslot(0)), kpar(0), abort_flag,
+                                wait_site(1, L::kBarKVFull + kslot(0), 0));
+      if (ok) {
+        tc_fence_after_sync();
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!valid[t]) continue;
+          issue_qk(t, 0);
+          tc_commit(bar(L::kBarS + t));
+        }
+        tc_commit(bar(L::kBarKVEmpty + kslot(0)));
+      }
+      for (int j = 0; ok && j < nmax; ++j) {
+        if (!wait_bounded(bar(L::kBarKVFull + vslot(j)), vpar(j), abort_flag,
+                          wait_site(1, L::kBarKVFull + vslot(j), j))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        bool knext = false;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || j >= nblk[t]) continue;
+          if (!wait_bounded(bar(L::kBarP + t), j & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
+            ok = false;
+            continue;
+          }
+          tc_fence_after_sync();
+          issue_pv(t, j);
+          if (j + 1 < nblk[t]) {
+            if (!knext) {
+              if (!wait_bounded(bar(L::kBarKVFull + kslot(j + 1)), kpar(j + 1), abort_flag,
+                                wait_site(1, L::kBarKVFull + kslot(j + 1), j + 1))) {
+                ok = false;
+                continue;
+              }
+              tc_fence_after_sync();
+              knext = true;
+            }
+            issue_qk(t, j + 1);
+            tc_commit(bar(L::kBarS + t));
+          } else {
+            tc_commit(bar(L::kBarO + t));
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar(L::kBarKVEmpty + vslot(j)));
+        if (knext) tc_commit(bar(L::kBarKVEmpty + kslot(j + 1)));
+      }
+      // Nothing issued by this thread may still run when tensor memory is released.
+      tc_commit(bar(L::kBarDrain));
+      wait_drain(bar(L::kBarDrain), 0, 100000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax warpgroups
+    const int t = warp / 4;
+    const int wq = warp % 4;          // TMEM lane quadrant of this warp
+    const int r = wq * 32 + lane;     // row of the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + L::tm_s(t) + lane_off;
+    const uint32_t tO = tmem + L::tm_o(t) + lane_off;
+    // This warpgroup's tile (selects instead of runtime-indexed arrays keep them in registers).
+    const int my_qb = t ? qb[1] : qb[0];
+    const int my_h = t ? h[1] : h[0];
+    const int my_n = t ? nblk[1] : nblk[0];
+    const bool my_valid = t ? valid[1] : valid[0];
+    const int qrow = my_qb * 128 + r;
+    bool ok = my_valid;
+    float m_run = -INFINITY, l_run = 0.f;
+    const float sl2 = p.sl2;
+    for (int j = 0; ok && j < my_n; ++j) {
+      if (!warp_wait_bounded(bar(L::kBarS + t), j & 1, abort_flag, wait_site(1, L::kBarS + t, j))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      float s[128];
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint32_t rr[32];
+        tmem_ld_x32(tS + c4 * 32, rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c4 * 32 + i] = __uint_as_float(rr[i]);
+      }
+      const int kv0 = j * 128;
+      if ((CAUSAL && j == my_qb) || kv0 + 128 > p.N) {
+        const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;   // keys kv < lim are visible
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kv0 + c >= lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+      const float m_cand = mx * sl2;
+      const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
+      const float alpha = ex2_approx(m_run - m_new);  // 0 on the first block, else <= 1
+      const float neg_m = -m_new;
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * c], sl2, neg_m));
+          const float p1 = ex2_approx(fmaf(s[half * 64 + 2 * c + 1], sl2, neg_m));
+          sum0 += p0;
+          sum1 += p1;
+          pk[c] = pack_bf16x2(p0, p1);
+        }
+        tmem_st_x32(tS + half * 32, pk);
+      }
+      l_run = l_run * alpha + (sum0 + sum1);
+      m_run = m_new;
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O was last written by P V of block j-1, which completed before S_j was ready.
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld_x32(tO + cc * 32, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_x32(tO + cc * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(bar(L::kBarP + t));
+    }
+
+    // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store
+    if (my_valid) {
+      bool okw = ok && warp_wait_bounded(bar(L::kBarO + t), 0, abort_flag, wait_site(1, L::kBarO + t, 0));
+      okw = named_bar_and(1 + t, 128, okw && *abort_flag == 0);
+      if (okw) {
+        tc_fence_after_sync();
+        const float inv_l = 1.f / l_run;
+        const uint32_t stage = sQ + t * L::kTileBytes;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld_x32(tO + cc * 32, o);
+          const uint32_t rowbase = stage + (cc / 2) * L::kChunkBytes + r * 128;
+#pragma unroll
+          for (int uu = 0; uu < 4; ++uu) {
+            const int unit = (cc % 2) * 4 + uu;   // 16-byte unit within the 128-byte row
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * inv_l,
+                                 __uint_as_float(o[8 * uu + 2 * e + 1]) * inv_l);
+            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+          }
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + t, 128);
+        if (r == 0) {
+#pragma unroll
+          for (int c = 0; c < L::kChunks; ++c)
+            tma_store_3d(&tm_o, stage + c * L::kChunkBytes, c * 64, my_qb * 128, b * p.Hq + my_h);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+        if (qrow < p.N)
+          p.lse[static_cast<size_t>(b * p.Hq + my_h) * p.N + qrow] = (m_run + log2f(l_run)) * kLn2;
+      }
+    }
+  }
+
+  // ---- teardown: every role has drained; release tensor memory
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,319 @@
+// fa_fwd_d256.cuh - forward attention kernel for head dimension 256 on sm_100a.
+//
+// Same computation and recurrence as fa_fwd.cuh (online softmax over key blocks with a
+// rescale of the partial output when the running max moves; the "FlashAttention1" Q&A
+// page's softmax question, items 1-3), shaped for d = 256, which the FlashAttention-2
+// page lists as the largest supported head dimension:
+//  * a CTA owns ONE 128-row query tile: two d = 256 fp32 output accumulators would need
+//    512 tensor-memory columns on their own;
+//  * key blocks are 64 rows, so Q (64 KB) plus a 4-slot K/V ring of 32 KB tiles fits in
+//    shared memory;
+//  * tensor memory holds O (256 columns) and TWO score buffers S_a | S_b (64 columns
+//    each): the tensor core computes S_{j+1} while the softmax warps work on S_j, and
+//    P_j (bf16) is written over S_j for the P V product;
+//  * the tensor core consumes K/V in the order K_0, K_1, V_0, K_2, V_1, K_3, ..., which
+//    is also the order the TMA warp loads them;
+//  * a rescale of O for block j must wait until P V of block j-1 has finished (with two
+//    score buffers, S_j being ready does not imply it); the softmax warps wait on a
+//    per-block completion barrier only in the rare blocks that move the max.
+#pragma once
+
+#include "fa_common.cuh"
+#include "fa_fwd.cuh"
+
+namespace fa {
+
+struct FwdD256Layout {
+  static constexpr int D = 256;
+  static constexpr int kQRows = 128;
+  static constexpr int kKRows = 64;
+  static constexpr int kChunks = 4;                       // 64-column swizzle chunks per row
+  static constexpr int kQChunkBytes = kQRows * 128;       // 16 KB
+  static constexpr int kKChunkBytes = kKRows * 128;       // 8 KB
+  static constexpr int kQBytes = kChunks * kQChunkBytes;  // 64 KB
+  static constexpr int kKVBytes = kChunks * kKChunkBytes; // 32 KB
+  static constexpr int kStages = 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kQBytes;
+  static constexpr int kOffBar = kOffKV + kStages * kKVBytes;
+  // mbarriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done, o_full, drain
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKVFull = 1;
+  static constexpr int kBarKVEmpty = kBarKVFull + kStages;
+  static constexpr int kBarS = kBarKVEmpty + kStages;
+  static constexpr int kBarP = kBarS + 2;
+  static constexpr int kBarPV = kBarP + 2;
+  static constexpr int kBarO = kBarPV + 1;
+  static constexpr int kBarDrain = kBarO + 1;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kTmS0 = 0;     // S_a: columns 0..63, S_b: 64..127
+  static constexpr uint32_t kTmO = 128;    // O: columns 128..383
+  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+};
+
+constexpr int kFwdD256Threads = 192;  // warps 0-3 softmax, 4 MMA, 5 TMA
+
+template <bool CAUSAL>
+__global__ void __launch_bounds__(kFwdD256Threads, 1)
+    fa_fwd_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                       const FwdParams p) {
+  using L = FwdD256Layout;
+  constexpr int S = L::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (base - raw);
+  const uint32_t sQ = base + L::kOffQ;
+  const uint32_t sKV = base + L::kOffKV;
+  uint32_t *misc = reinterpret_cast<uint32_t *>(smem + L::kOffMisc);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(misc + 1);
+  auto bar = [&](int i) -> uint32_t { return base + L::kOffBar + 8u * static_cast<uint32_t>(i); };
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+
+  // ---- unit = (b, h, query block), longest causal blocks first
+  int u = blockIdx.x;
+  const int qb = p.nqb - 1 - (u % p.nqb);
+  u /= p.nqb;
+  const int h = u % p.Hq;
+  const int b = u / p.Hq;
+  const int kvh = h / (p.Hq / p.Hkv);
+  const int nkb_all = (p.N + 63) / 64;
+  const int nblk = CAUSAL ? min(2 * qb + 2, nkb_all) : nkb_all;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::kNumBars; ++i)
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? 128u : 1u);
+    misc[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(misc), L::kTmemCols);
+    tmem_relinquish_alloc_permit();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = misc[0];
+
+  // Load/consume order of the K/V ring: K_0, K_1, then V_j followed by K_{j+2}.
+  // Item index -> (is_v, block).  Both the TMA warp and the MMA warp walk this order.
+  if (warp == 5) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_o);
+      mbar_arrive_expect_tx(bar(L::kBarQ), L::kQBytes);
+#pragma unroll
+      for (int c = 0; c < L::kChunks; ++c)
+        tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, bar(L::kBarQ), c * 64, qb * 128, b * p.Hq + h);
+      int seq = 0;
+      bool ok = true;
+      auto produce = [&](bool is_v, int j) {
+        const int slot = seq % S, use = seq / S;
+        if (!wait_bounded(bar(L::kBarKVEmpty + slot), (use & 1) ^ 1, abort_flag,
+                          wait_site(2, L::kBarKVEmpty + slot, j))) {
+          ok = false;
+          return;
+        }
+        mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kKVBytes);
+        const CUtensorMap *m = is_v ? &tm_v : &tm_k;
+#pragma unroll
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sKV + slot * L::kKVBytes + c * L::kKChunkBytes, m, bar(L::kBarKVFull + slot), c * 64,
+                      j * 64, b * p.Hkv + kvh);
+        ++seq;
+      };
+      produce(false, 0);
+      if (ok && nblk > 1) produce(false, 1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        produce(true, j);
+        if (ok && j + 2 < nblk) produce(false, j + 2);
+      }
+      for (int s2 = seq > S ? seq - S : 0; s2 < seq; ++s2)
+        wait_drain(bar(L::kBarKVFull + s2 % S), (s2 / S) & 1, 100000000ull);
+      wait_drain(bar(L::kBarQ), 0, 100000000ull);
+    }
+    __syncwarp();
+  } else if (warp == 4) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
+      int seq = 0;
+      bool ok = wait_bounded(bar(L::kBarQ), 0, abort_flag, wait_site(2, L::kBarQ, 0));
+      // Take the next ring item: wait until it has landed; returns its slot.
+      auto consume = [&](int j) -> int {
+        const int slot = seq % S, use = seq / S;
+        if (!wait_bounded(bar(L::kBarKVFull + slot), use & 1, abort_flag,
+                          wait_site(2, L::kBarKVFull + slot, j)))
+          ok = false;
+        ++seq;
+        return slot;
+      };
+      // S_buf = Q K_j^T : M = 128, N = 64 keys, K = 256.
+      auto issue_qk = [&](int j) {
+        const int slot = consume(j);
+        if (!ok) return;
+        tc_fence_after_sync();
+        const uint32_t buf = L::kTmS0 + (j & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const uint32_t ka = (kk / 4) * L::kQChunkBytes + (kk % 4) * 32;
+          const uint32_t kb = (kk / 4) * L::kKChunkBytes + (kk % 4) * 32;
+          mma_ss(tmem + buf, sdesc_sw128(sQ + ka, 16, 1024),
+                 sdesc_sw128(sKV + slot * L::kKVBytes + kb, 16, 1024), idesc_qk, kk > 0);
+        }
+        tc_commit(bar(L::kBarS + (j & 1)));
+        tc_commit(bar(L::kBarKVEmpty + slot));
+      };
+      if (ok) issue_qk(0);
+      if (ok && nblk > 1) issue_qk(1);
+      for (int j = 0; ok && j < nblk; ++j) {
+        const int vslot = consume(j);
+        if (!ok) break;
+        if (!wait_bounded(bar(L::kBarP + (j & 1)), (j >> 1) & 1, abort_flag,
+                          wait_site(2, L::kBarP + (j & 1), j))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        // O += P_j V_j : M = 128, N = 256, K = 64 keys (4 instructions of 16 keys).
+        const uint32_t pbuf = L::kTmS0 + (j & 1) * 64;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(tmem + L::kTmO, tmem + pbuf + kk * 8,
+                 sdesc_sw128(sKV + vslot * L::kKVBytes + kk * 2048, L::kKChunkBytes, 1024), idesc_pv,
+                 (j > 0 || kk > 0));
+        tc_commit(bar(L::kBarPV));
+        tc_commit(bar(L::kBarKVEmpty + vslot));
+        if (j + 2 < nblk) issue_qk(j + 2);
+      }
+      if (ok) tc_commit(bar(L::kBarO));
+      tc_commit(bar(L::kBarDrain));
+      wait_drain(bar(L::kBarDrain), 0, 100000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ softmax warpgroup
+    const int r = warp * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t tO = tmem + L::kTmO + lane_off;
+    const int qrow = qb * 128 + r;
+    bool ok = true;
+    float m_run = -INFINITY, l_run = 0.f;
+    const float sl2 = p.sl2;
+    for (int j = 0; ok && j < nblk; ++j) {
+      const uint32_t tS = tmem + L::kTmS0 + (j & 1) * 64 + lane_off;
+      if (!warp_wait_bounded(bar(L::kBarS + (j & 1)), (j >> 1) & 1, abort_flag,
+                             wait_site(2, L::kBarS + (j & 1), j))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
+      float s[64];
+#pragma unroll
+      for (int c2 = 0; c2 < 2; ++c2) {
+        uint32_t rr[32];
+        tmem_ld_x32(tS + c2 * 32, rr);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) s[c2 * 32 + i] = __uint_as_float(rr[i]);
+      }
+      const int kv0 = j * 64;
+      if ((CAUSAL && kv0 + 63 > qb * 128) || kv0 + 64 > p.N) {
+        const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (kv0 + c >= lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, s[c]);
+      const float m_cand = mx * sl2;
+      const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
+      const float alpha = ex2_approx(m_run - m_new);
+      const float neg_m = -m_new;
+      float sum0 = 0.f, sum1 = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg_m));
+        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg_m));
+        sum0 += p0;
+        sum1 += p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      tmem_st_x32(tS, pk);
+      l_run = l_run * alpha + (sum0 + sum1);
+      m_run = m_new;
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // P V of block j-1 must have finished before O is rescaled.
+        if (!warp_wait_bounded(bar(L::kBarPV), (j - 1) & 1, abort_flag, wait_site(2, L::kBarPV, j))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          uint32_t o[32];
+          tmem_ld_x32(tO + cc * 32, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_x32(tO + cc * 32, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before_sync();
+      mbar_arrive(bar(L::kBarP + (j & 1)));
+    }
+
+    bool okw = ok && warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0));
+    okw = named_bar_and(1, 128, okw && *abort_flag == 0);
+    if (okw) {
+      tc_fence_after_sync();
+      const float inv_l = 1.f / l_run;
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t o[32];
+        tmem_ld_x32(tO + cc * 32, o);
+        const uint32_t rowbase = sQ + (cc / 2) * L::kQChunkBytes + r * 128;
+#pragma unroll
+        for (int uu = 0; uu < 4; ++uu) {
+          const int unit = (cc % 2) * 4 + uu;
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * inv_l,
+                               __uint_as_float(o[8 * uu + 2 * e + 1]) * inv_l);
+          st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (r == 0) {
+#pragma unroll
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_store_3d(&tm_o, sQ + c * L::kQChunkBytes, c * 64, qb * 128, b * p.Hq + h);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+      }
+      if (qrow < p.N) p.lse[static_cast<size_t>(b * p.Hq + h) * p.N + qrow] = (m_run + log2f(l_run)) * kLn2;
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,114 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact-attention library, libfa_sm100.so.
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ * tile by tile with the online-softmax recurrence, so the N x N score matrix never
+ * reaches device memory, and its gradient by recomputing the score tiles on chip.
+ *
+ * Sources of the operations (web pages on FlashAttention):
+ *  - tiling and on-chip recomputation in the backward pass: "The Future of AI: How
+ *    FlashAttention Revolutionizes Deep Learning", bullets "Tiling" and "Recomputation";
+ *  - the online softmax (running max m, running sum l, rescaling of partial results
+ *    when a block raises the max): "FlashAttention1" interview Q&A, question on how
+ *    FlashAttention computes the softmax function, items 1-3; "Flash attention ... a deep
+ *    dive", section "What is the mathematical aspect of softmax?" ("Intuition");
+ *  - exactness (the blocked result equals standard attention): the same Q&A, question
+ *    on the key algorithmic innovations; the deep-dive page, section "Algorithm behind
+ *    the article";
+ *  - grouped- and multi-query attention and head dimensions up to 256: the
+ *    FlashAttention-2 page, "FlashAttention-2: Enhanced Performance";
+ *  - causal masking: the deep-dive page names masking among the memory-bound steps
+ *    ("Quantitative Evidence"); this library uses the top-left causal mask, key j is
+ *    visible to query i when j <= i.
+ *
+ * Conventions shared by every entry point
+ *  - Layout: Q, dQ, O, dO are [B, Hq, N, d]; K, V, dK, dV are [B, Hkv, N, d]; all
+ *    contiguous bf16 (row of d elements, then N rows, then heads, then batch).  LSE is
+ *    [B, Hq, N] fp32 (natural-log logsumexp of the scaled scores of each query row).
+ *  - Query head h uses K/V head h / (Hq / Hkv) (contiguous groups).
+ *  - Supported head dimensions: d in {64, 128, 256}.  Any N >= 1.
+ *  - Every pointer is a DEVICE pointer owned by the caller and must be 16-byte aligned.
+ *    The library allocates no device memory except its 8-byte status words, which live
+ *    in a file-scope __device__ variable.  Input buffers are read-only.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *    asynchronous with respect to the host; it returns after enqueueing kernels.
+ *  - Argument errors are detected on the host before anything is launched; the outputs
+ *    are then left untouched.  A launch failure returns FA_ERR_CUDA.
+ *  - Device-side failures (a pipeline wait that exceeded its time limit) are recorded in
+ *    the device status word and reported by fa_device_status().
+ *  - The calls may be made from several host threads; the tensor-map encoder they share
+ *    holds no state.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+enum fa_status {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, non-finite/<=0 scale */
+    FA_ERR_UNSUPPORTED = 2,    /* d not in {64, 128, 256}, or sizes beyond int32 index range */
+    FA_ERR_GQA = 3,            /* Hq is not a multiple of Hkv */
+    FA_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned */
+    FA_ERR_WORKSPACE = 5,      /* workspace missing or smaller than fa_bwd_workspace_bytes() */
+    FA_ERR_CUDA = 6,           /* CUDA runtime/driver error (no sm_100 device, launch failure) */
+    FA_ERR_DEVICE_TIMEOUT = 7  /* a kernel's bounded pipeline wait expired (device watchdog) */
+};
+
+/*
+ * Forward pass.
+ *   q   [B, Hq,  N, d] bf16 in      k, v [B, Hkv, N, d] bf16 in
+ *   o   [B, Hq,  N, d] bf16 out     lse  [B, Hq, N] fp32 out (natural log)
+ *   causal: 0 or 1 (top-left mask, key j visible to query i iff j <= i)
+ *   scale: softmax scale (> 0, finite), typically 1/sqrt(d), applied to Q K^T.
+ * O and LSE are each written exactly once; rows are independent.
+ */
+int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
+           int B, int Hq, int Hkv, int N, int d, int causal, float scale, void *stream);
+
+/*
+ * Size in bytes of the fp32 scratch that fa_bwd needs: Delta_i = <dO_i, O_i> per query
+ * row ([B, Hq, N] fp32) plus a dQ accumulator ([B, Hq, N, d] fp32), each padded to
+ * 256 bytes.  Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/*
+ * Backward pass: gradients of <O, dO> with respect to Q, K and V.
+ *   q, k, v, o, lse: as given to / produced by fa_fwd with the same sizes, causal, scale.
+ *   dout [B, Hq, N, d] bf16 in (dL/dO)
+ *   dq   [B, Hq, N, d] bf16 out;  dk, dv [B, Hkv, N, d] bf16 out (summed over the query
+ *        heads that share each K/V head)
+ *   workspace: device scratch of at least fa_bwd_workspace_bytes() bytes, 16-byte
+ *        aligned; its contents on entry do not matter and on return are unspecified.
+ * The score tiles are recomputed from Q, K and LSE (nothing N x N is stored).
+ */
+int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+           const void *dout, void *dq, void *dk, void *dv, void *workspace,
+           size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
+           float scale, void *stream);
+
+/*
+ * Synchronises `stream`, returns the device status word of the current device
+ * (FA_OK or FA_ERR_DEVICE_TIMEOUT) and clears it.  Returns FA_ERR_CUDA if the
+ * synchronisation itself fails.
+ */
+int fa_device_status(void *stream);
+
+/* Static, human-readable text for a status code. */
+const char *fa_status_string(int code);
+
+/* Library ABI version (major * 100 + minor). */
+int fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */

@@ -1,0 +1,121 @@
+"""Host-only checks of the C ABI: the library builds for sm_100a, loads without a GPU,
+exports every entry point that include/fa.h declares, and rejects invalid arguments with
+the documented status codes before touching a device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+from exact_io_aware_83_b200 import fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+FAKE = 0x10000  # never dereferenced: every case below fails validation first
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_device_status",
+                     "fa_status_string", "fa_version"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    fa.load()
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (fa_[a-z0-9_]+)$", out, flags=re.M))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, missing
+
+
+def test_status_strings_and_version():
+    assert fa.load().fa_version() == 100
+    for code in range(8):
+        assert fa.fa_status_string(code) not in ("", "unknown status")
+    assert fa.fa_status_string(99) == "unknown status"
+
+
+def _fwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, N=16, d=128,
+                causal=0, scale=0.125, stream=None)
+    args.update(kw)
+    return fa.load().fa_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"],
+                            args["Hq"], args["Hkv"], args["N"], args["d"], args["causal"],
+                            args["scale"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(lse=None), fa.FA_ERR_INVALID_ARG),
+    (dict(N=0), fa.FA_ERR_INVALID_ARG),
+    (dict(B=-1), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=32), fa.FA_ERR_UNSUPPORTED),
+    (dict(Hq=3, Hkv=2), fa.FA_ERR_GQA),
+    (dict(o=FAKE + 8), fa.FA_ERR_ALIGN),
+    (dict(lse=FAKE + 4), fa.FA_ERR_ALIGN),
+    (dict(B=1 << 16, Hq=1 << 8, Hkv=1, N=1 << 8), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_argument_errors(kw, code):
+    assert _fwd(**kw) == code
+
+
+def _bwd(**kw):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dout=FAKE, dq=FAKE, dk=FAKE, dv=FAKE,
+                ws=FAKE, ws_bytes=1 << 30, B=1, Hq=2, Hkv=1, N=16, d=128, causal=1, scale=0.125,
+                stream=None)
+    args.update(kw)
+    a = args
+    return fa.load().fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["dout"], a["dq"],
+                            a["dk"], a["dv"], a["ws"], a["ws_bytes"], a["B"], a["Hq"], a["Hkv"],
+                            a["N"], a["d"], a["causal"], a["scale"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dout=None), fa.FA_ERR_INVALID_ARG),
+    (dict(dv=None), fa.FA_ERR_INVALID_ARG),
+    (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+    (dict(Hq=4, Hkv=3), fa.FA_ERR_GQA),
+    (dict(ws=None), fa.FA_ERR_WORKSPACE),
+    (dict(ws_bytes=100), fa.FA_ERR_WORKSPACE),
+    (dict(dk=FAKE + 2), fa.FA_ERR_ALIGN),
+])
+def test_bwd_argument_errors(kw, code):
+    assert _bwd(**kw) == code
+
+
+def test_workspace_size():
+    B, Hq, N, d = 2, 4, 100, 128
+    rows = B * Hq * N
+    pad = lambda x: (x + 255) // 256 * 256
+    assert fa.fa_bwd_workspace_bytes(B, Hq, 2, N, d) == pad(rows * 4) + pad(rows * d * 4)
+    assert fa.fa_bwd_workspace_bytes(B, Hq, 3, N, d) == 0
+    assert fa.fa_bwd_workspace_bytes(B, Hq, 2, N, 48) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="valid-argument path needs no GPU")
+def test_valid_arguments_without_a_device_report_cuda_error():
+    # Every argument is valid, so the call reaches the device check and stops there.
+    assert _fwd() == fa.FA_ERR_CUDA
+    assert _bwd() == fa.FA_ERR_CUDA
+
+
+def test_binding_rejects_cpu_tensors():
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.fwd(q, q, q)

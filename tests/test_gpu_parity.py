@@ -1,0 +1,248 @@
+"""GPU parity of the CUDA library (through the C ABI) against the fp64 oracle.
+
+Tolerances, on the same seeded bf16 inputs:
+  max|O - O_ref| <= 1e-2 (after the GPU's bf16 store), max|LSE - LSE_ref| <= 1e-3,
+  ||X - X_ref||_F / ||X_ref||_F <= 2e-2 for X in {dQ, dK, dV};
+no NaN/Inf anywhere, and guard bands of sentinel values around every output buffer left
+untouched (an out-of-bounds write shows up there).
+
+Small cases run the oracle on everything; the five full-size workloads are compared on
+sampled (batch, K/V-head group) slices, which the oracle computes exactly because
+groups never interact, plus invariants that hold at any size.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_83_b200 import fa
+from exact_io_aware_83_b200.inputs import WORKLOADS, draw, draw_workload
+
+pytestmark = pytest.mark.gpu
+
+O_TOL = 1e-2
+LSE_TOL = 1e-3
+GRAD_TOL = 2e-2
+GUARD = 256          # sentinel elements on each side of an output
+SENT_BF16 = 1234.0   # exactly representable in bf16
+SENT_F32 = -7777.0
+
+
+def _guarded(shape, dtype, sentinel):
+    n = int(np.prod(shape))
+    buf = torch.full((GUARD + n + GUARD,), sentinel, dtype=dtype, device="cuda")
+    return buf, buf[GUARD:GUARD + n].view(shape)
+
+
+def _guards_intact(buf, sentinel):
+    lo = buf[:GUARD]
+    hi = buf[-GUARD:]
+    return bool(torch.all(lo == sentinel)) and bool(torch.all(hi == sentinel))
+
+
+def _f64(t):
+    return t.float().double().cpu().numpy()
+
+
+def run_fwd(q, k, v, causal, scale):
+    """Forward through the C ABI with guard bands; returns (o, lse) as CPU tensors."""
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    B, Hq, N, d = q.shape
+    ob, o = _guarded(q.shape, torch.bfloat16, SENT_BF16)
+    lb, lse = _guarded((B, Hq, N), torch.float32, SENT_F32)
+    fa.fwd(qd, kd, vd, causal=causal, scale=scale, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(None) == fa.FA_OK
+    assert _guards_intact(ob, SENT_BF16), "write outside O"
+    assert _guards_intact(lb, SENT_F32), "write outside LSE"
+    return o.cpu(), lse.cpu()
+
+
+def run_bwd(q, k, v, o, lse, do, causal, scale):
+    qd, kd, vd, od, dod = q.cuda(), k.cuda(), v.cuda(), o.cuda(), do.cuda()
+    lsed = lse.cuda()
+    B, Hq, N, d = q.shape
+    Hkv = k.shape[1]
+    dqb, dq = _guarded(q.shape, torch.bfloat16, SENT_BF16)
+    dkb, dk = _guarded(k.shape, torch.bfloat16, SENT_BF16)
+    dvb, dv = _guarded(v.shape, torch.bfloat16, SENT_BF16)
+    ws = torch.full((fa.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d),), 0x7F, dtype=torch.uint8,
+                    device="cuda")  # garbage on entry must not matter
+    fa.bwd(qd, kd, vd, od, lsed, dod, causal=causal, scale=scale, workspace=ws, dq=dq, dk=dk,
+           dv=dv)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status(None) == fa.FA_OK
+    for buf, name in ((dqb, "dQ"), (dkb, "dK"), (dvb, "dV")):
+        assert _guards_intact(buf, SENT_BF16), f"write outside {name}"
+    return dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def _finite(*ts):
+    for t in ts:
+        assert torch.isfinite(t.float()).all(), "non-finite output"
+
+
+def _rel_fro(x, ref):
+    return float(np.linalg.norm(x - ref) / max(np.linalg.norm(ref), 1e-30))
+
+
+def check_fwd(o, lse, q, k, v, causal, scale):
+    o_ref, lse_ref = oracle.attention_fwd(_f64(q), _f64(k), _f64(v), causal, scale)
+    _finite(o, lse)
+    err_o = float(np.max(np.abs(_f64(o) - o_ref)))
+    err_l = float(np.max(np.abs(lse.double().numpy() - lse_ref)))
+    assert err_o <= O_TOL, f"max|O-O_ref| = {err_o}"
+    assert err_l <= LSE_TOL, f"max|LSE-LSE_ref| = {err_l}"
+    return err_o, err_l
+
+
+def check_bwd(dq, dk, dv, q, k, v, do, causal, scale):
+    dq_r, dk_r, dv_r, _, _ = oracle.attention_bwd(_f64(q), _f64(k), _f64(v), _f64(do), causal,
+                                                  scale)
+    _finite(dq, dk, dv)
+    errs = {}
+    for name, x, ref in (("dQ", dq, dq_r), ("dK", dk, dk_r), ("dV", dv, dv_r)):
+        errs[name] = _rel_fro(_f64(x), ref)
+        assert errs[name] <= GRAD_TOL, f"{name} relative Frobenius error {errs[name]}"
+    return errs
+
+
+# ----------------------------------------------------------------------------- small cases
+
+SMALL_N = [1, 2, 17, 128, 129, 255, 256, 384]
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", SMALL_N)
+def test_fwd_small(d, causal, N):
+    q, k, v = draw(1, 2, 1, N, d, seed=1000 + N + d, with_dout=False)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_fwd(q, k, v, causal, scale)
+    check_fwd(o, lse, q, k, v, causal, scale)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (2, 2), (3, 1), (4, 2), (8, 2), (6, 3), (8, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_heads_and_groups(Hq, Hkv, causal):
+    q, k, v = draw(2, Hq, Hkv, 200, 128, seed=Hq * 10 + Hkv, with_dout=False)
+    o, lse = run_fwd(q, k, v, causal, 0.0883883461356163)
+    check_fwd(o, lse, q, k, v, causal, 0.0883883461356163)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 17, 128, 129, 256, 384])
+def test_bwd_small(d, causal, N):
+    q, k, v, do = draw(1, 2, 1, N, d, seed=2000 + N + d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = run_fwd(q, k, v, causal, scale)
+    dq, dk, dv = run_bwd(q, k, v, o, lse, do, causal, scale)
+    check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(1, 1), (4, 4), (4, 2), (8, 2), (3, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_heads_and_groups(Hq, Hkv, causal):
+    q, k, v, do = draw(2, Hq, Hkv, 192, 128, seed=3000 + Hq * 10 + Hkv)
+    scale = 0.0883883461356163
+    o, lse = run_fwd(q, k, v, causal, scale)
+    dq, dk, dv = run_bwd(q, k, v, o, lse, do, causal, scale)
+    check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
+
+
+def test_softmax_stress_large_scores():
+    # Q ~ N(0, 4^2) and a large scale move the row max across key blocks, which
+    # exercises the rescale path of the online recurrence.
+    q, k, v, do = draw(1, 2, 2, 640, 128, seed=77, q_std=4.0)
+    scale = 0.35
+    for causal in (False, True):
+        o, lse = run_fwd(q, k, v, causal, scale)
+        check_fwd(o, lse, q, k, v, causal, scale)
+        dq, dk, dv = run_bwd(q, k, v, o, lse, do, causal, scale)
+        check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
+
+
+def test_toy_example_from_the_article_page():
+    # The 4x4 score matrix of the "Consideration is All You Want" page, embedded as
+    # Q = I, K = S^T, V = I (zero-padded to d = 64), scale 1: then O = P exactly.
+    S = np.array([[1, 2, 3, 4], [2, 1, 3, 4], [3, 2, 1, 4], [4, 2, 3, 1]], dtype=np.float64)
+    d = 64
+    q = torch.zeros(1, 1, 4, d)
+    q[0, 0, :, :4] = torch.eye(4)
+    k = torch.zeros(1, 1, 4, d)
+    k[0, 0, :, :4] = torch.tensor(S.T)
+    v = torch.zeros(1, 1, 4, d)
+    v[0, 0, :, :4] = torch.eye(4)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    e = math.e
+    z = e + e ** 2 + e ** 3 + e ** 4
+    for causal in (False, True):
+        o, lse = run_fwd(q, k, v, causal, 1.0)
+        if not causal:
+            np.testing.assert_allclose(lse[0, 0].numpy(), math.log(z), atol=LSE_TOL)
+            np.testing.assert_allclose(o[0, 0, :, :4].float().numpy(), np.exp(S) / z, atol=O_TOL)
+        else:
+            np.testing.assert_allclose(
+                lse[0, 0].numpy(),
+                [1.0, math.log(e ** 2 + e), math.log(e ** 3 + e ** 2 + e), math.log(z)],
+                atol=LSE_TOL)
+        assert torch.all(o[0, 0, :, 4:] == 0)
+        check_fwd(o, lse, q, k, v, causal, 1.0)
+
+
+def test_repeated_calls_are_stable():
+    q, k, v, do = draw(1, 4, 2, 300, 128, seed=5)
+    o1, l1 = run_fwd(q, k, v, True, 0.1)
+    o2, l2 = run_fwd(q, k, v, True, 0.1)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)  # the forward is deterministic
+    g1 = run_bwd(q, k, v, o1, l1, do, True, 0.1)
+    g2 = run_bwd(q, k, v, o1, l1, do, True, 0.1)
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])  # dK, dV deterministic
+    assert _rel_fro(_f64(g1[0]), _f64(g2[0])) < 1e-3  # dQ: fp32 reduce order may vary
+
+
+# ----------------------------------------------------------------------------- full sizes
+
+def _slice_group(t, b, h0, h1):
+    return t[b:b + 1, h0:h1].contiguous()
+
+
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_full_size_workloads(name):
+    w = WORKLOADS[name]
+    inputs = draw_workload(w)
+    q, k, v = inputs[:3]
+    o, lse = run_fwd(q, k, v, w.causal, w.scale)
+    _finite(o, lse)
+    g = w.Hq // w.Hkv
+    rng = np.random.default_rng(w.seed)
+    # Sampled (b, K/V head) groups: compare every row of the group with the oracle.
+    groups = {(0, 0), (w.B - 1, w.Hkv - 1), (int(rng.integers(w.B)), int(rng.integers(w.Hkv)))}
+    if w.N >= 8192:
+        groups = {(w.B - 1, w.Hkv - 1)}
+    for b, kh in sorted(groups):
+        hs = slice(kh * g, (kh + 1) * g)
+        qs = _slice_group(q, b, hs.start, hs.stop)
+        ks = _slice_group(k, b, kh, kh + 1)
+        vs = _slice_group(v, b, kh, kh + 1)
+        check_fwd(o[b:b + 1, hs], lse[b:b + 1, hs], qs, ks, vs, w.causal, w.scale)
+    if not w.backward:
+        return
+    do = inputs[3]
+    dq, dk, dv = run_bwd(q, k, v, o, lse, do, w.causal, w.scale)
+    _finite(dq, dk, dv)
+    # Invariants at full size: sum_j dK_j = 0 and sum_j dV_j = sum over the group's rows of dO.
+    dk64, dv64 = _f64(dk), _f64(dv)
+    do_sum = _f64(do).reshape(w.B, w.Hkv, g, w.N, w.d).sum(axis=(2, 3))
+    scale_dk = np.abs(dk64).sum(axis=2).max()
+    assert np.abs(dk64.sum(axis=2)).max() <= 2e-2 * scale_dk
+    assert np.abs(dv64.sum(axis=2) - do_sum).max() <= 2e-2 * np.abs(do_sum).max() + 1.0
+    b, kh = sorted(groups)[-1]
+    hs = slice(kh * g, (kh + 1) * g)
+    check_bwd(dq[b:b + 1, hs], dk[b:b + 1, kh:kh + 1], dv[b:b + 1, kh:kh + 1],
+              _slice_group(q, b, hs.start, hs.stop), _slice_group(k, b, kh, kh + 1),
+              _slice_group(v, b, kh, kh + 1), _slice_group(do, b, hs.start, hs.stop),
+              w.causal, w.scale)
