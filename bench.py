@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Throughput of exact attention (forward + backward) on B200 through libfa_sm100.so.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one forward (fa_fwd) and one backward (fa_bwd) pass over one batch of the
+workload (default: GPT-style 2K causal self-attention, B=8, H=16, N=2048, d=128, bf16,
+seeded i.i.d. N(0,1) inputs).  FLOPs follow the metric's convention: 4 B H N^2 d for the
+forward, halved when causal, and 2.5x that for the backward.
+
+Rank 0 prints one JSON line.  Under torchrun each rank (one GPU each) processes its own
+shard of a global batch of N x B sequences with the unchanged kernels (no collective on
+the data path); the timed region is bracketed by barriers and the slowest rank's time is
+used, so `value` is the whole job's TFLOP/s ("scaling": "weak").
+
+`--impl reference` times the fp64 CPU oracle (the parity reference) on a bounded sample of
+the same workload on this host's cores, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime as _dt
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd+bwd TFLOP/s at 1 B200 and % of dense-BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def _profile_traffic():
+    """DRAM bytes per launch of the backward main kernel from the committed ncu summary,
+    scaled to the benchmark workload, or None when no current capture exists."""
+    path = os.path.join(ROOT, "profiles", "bwd_main_traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d
+    except (OSError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples, kept only inside [t0, t1]."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        self.t0 = _dt.datetime.now()
+
+    def stop(self):
+        self.t1 = _dt.datetime.now()
+        time.sleep(0.12)
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.file.flush()
+        self.file.seek(0)
+        rows = [r for r in csv.reader(io.StringIO(self.file.read())) if len(r) >= 9]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, mx, reasons, n = [], [], set(), 0
+        for r in rows:
+            try:
+                ts = _dt.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                continue
+            if self.t0 and self.t1 and not (self.t0 <= ts <= self.t1):
+                continue
+            n += 1
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                pass
+            for name, val in zip(names, r[5:9]):
+                if val.strip() == "Active":
+                    reasons.add(name)
+        os.unlink(self.file.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def _oracle_sample(w, heads: int, seed: int):
+    """fp64 oracle fwd+bwd on the first `heads` query heads (whole K/V groups) of batch
+    row 0 of the workload's inputs; returns (seconds, metric FLOPs of the sample)."""
+    import numpy as np
+    import torch
+    import oracle
+    from exact_io_aware_83_b200.inputs import draw
+    g = w.Hq // w.Hkv
+    groups = max(1, heads // g)
+    q, k, v, do = draw(1, groups * g, groups, w.N, w.d, seed, w.q_std)
+    f64 = lambda t: t.float().double().numpy()
+    q, k, v, do = f64(q), f64(k), f64(v), f64(do)
+    t0 = time.perf_counter()
+    oracle.attention_fwd(q, k, v, w.causal, w.scale)
+    if w.backward:
+        oracle.attention_bwd(q, k, v, do, w.causal, w.scale)
+    dt = time.perf_counter() - t0
+    flops = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) * (groups * g) / (w.B * w.Hq)
+    return dt, flops
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    cores = _cores()
+    oracle.set_threads(cores)
+    # Size the per-step sample so the whole run stays near a two-minute budget: whole
+    # K/V-head groups of batch row 0, at least one.
+    g = w.Hq // w.Hkv
+    t_group, _ = _oracle_sample(w, g, w.seed)
+    budget = 120.0 / (args.steps + args.warmup)
+    heads = g * max(1, min(w.Hkv, int(budget // max(t_group, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_sample(w, heads, w.seed)
+    total_t, total_f = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = _oracle_sample(w, heads, w.seed)
+        total_t += dt
+        total_f += fl
+    value = total_f / total_t / 1e12
+    sample = (f"batch row 0, query heads 0..{heads - 1} of {w.name} (fwd"
+              f"{'+bwd' if w.backward else ''}), fp64 oracle, per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w, world):
+    return {"workload": w.name, "B_per_gpu": w.B, "global_batch": w.B * world, "Hq": w.Hq,
+            "Hkv": w.Hkv, "seq_len": w.N, "head_dim": w.d, "causal": w.causal,
+            "passes": "fwd+bwd" if w.backward else "fwd", "parallelism": f"dp{world}",
+            "l2": "inputs exceed L2 (q, k, v, dO = "
+                  f"{4 * w.B * w.Hq * w.N * w.d * 2 / 1e6:.0f} MB vs 126 MB); no flush"}
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_83_b200 import fa
+    from exact_io_aware_83_b200.inputs import draw
+    from exact_io_aware_83_b200.shard import max_over_ranks, rank_seed
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    fa.load()
+    qh, kh, vh, doh = draw(w.B, w.Hq, w.Hkv, w.N, w.d, rank_seed(w.seed, rank), w.q_std)
+    q, k, v, do = (t.cuda() for t in (qh, kh, vh, doh))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8,
+                     device="cuda")
+
+    def step():
+        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        if w.backward:
+            fa.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws, dq=dq,
+                   dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_device_status(None) != fa.FA_OK:
+        raise SystemExit("device status not clean after warm-up")
+
+    sampler = ClockSampler(local)
+    time.sleep(0.3)  # let nvidia-smi start sampling
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    fa.fa_kernel_timing(True)
+    sampler.start()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    fa.fa_kernel_timing(False)
+    ms_local = e0.elapsed_time(e1)
+    ms = max_over_ranks(ms_local)
+    fwd_ms, nfwd = fa.fa_kernel_time_ms(0)
+    bwd_ms, nbwd = fa.fa_kernel_time_ms(1)
+    status = fa.fa_device_status(None)
+    if status != fa.FA_OK:
+        raise SystemExit(f"device status {status} after the timed region")
+    clocks = sampler.summary()
+
+    step_flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
+    value = step_flops * args.steps * world / (ms / 1e3) / 1e12
+
+    # ---- end to end through the public API: pinned host inputs in, results back to host
+    pin = lambda t: t.pin_memory()
+    qh_p, kh_p, vh_p, doh_p = (pin(t) for t in (qh, kh, vh, doh))
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dqh = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+    dkh = torch.empty(dk.shape, dtype=dk.dtype).pin_memory()
+    dvh = torch.empty(dv.shape, dtype=dv.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(qh_p, non_blocking=True)
+        k.copy_(kh_p, non_blocking=True)
+        v.copy_(vh_p, non_blocking=True)
+        if w.backward:
+            do.copy_(doh_p, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+        if w.backward:
+            dqh.copy_(dq, non_blocking=True)
+            dkh.copy_(dk, non_blocking=True)
+            dvh.copy_(dv, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 10)
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+    h2d = nbytes(q, k, v, do) if w.backward else nbytes(q, k, v)
+    d2h = nbytes(o, lse, dq, dk, dv) if w.backward else nbytes(o, lse)
+    e2e_value = step_flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12
+
+    peaks, peak_src = _peaks()
+    # Dominant kernel: the backward main kernel (or the forward when there is no backward).
+    if w.backward and nbwd:
+        dom_name, dom_ms, dom_n, dom_flops = "fa_bwd_main_kernel", bwd_ms, nbwd, w.bwd_flops()
+    else:
+        dom_name, dom_ms, dom_n, dom_flops = "fa_fwd_kernel", fwd_ms, nfwd, w.fwd_flops()
+    achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = None
+    prof = _profile_traffic()
+    if prof and prof.get("workload") == w.name and prof.get("kernel") == dom_name:
+        traffic = prof.get("dram_bytes_per_launch")
+    kernels = {}
+    if nfwd:
+        kernels["fa_fwd_kernel"] = {"ms_per_launch": fwd_ms / nfwd,
+                                    "tflops": w.fwd_flops() / (fwd_ms / nfwd / 1e3) / 1e12}
+    if nbwd:
+        kernels["fa_bwd_main_kernel"] = {"ms_per_launch": bwd_ms / nbwd,
+                                         "tflops": w.bwd_flops() / (bwd_ms / nbwd / 1e3) / 1e12}
+    for kname, kd in kernels.items():
+        kd["frac_of_burst_peak"] = kd["tflops"] / peak
+        kd["frac_of_sustained_peak"] = kd["tflops"] / float(peaks["bf16_tflops_sustained"])
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config(w, world),
+        "frac_of_peak": value / world / peak,
+        "roofline": {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
+        "kernels": kernels,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": args.steps * (1 + (3 if w.backward else 0)),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        cores = _cores()
+        oracle.set_threads(cores)
+        heads = max(1, min(w.Hq, args.sample_heads))
+        dt, fl = _oracle_sample(w, heads, w.seed)
+        line["cpu_baseline"] = {
+            "value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"batch row 0, query heads 0..{heads - 1} of {w.name}, fp64 oracle "
+                      f"fwd{'+bwd' if w.backward else ''}, one pass, {dt:.1f} s wall"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="gpt_2k_causal")
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--sample-heads", type=int, default=4,
+                    help="query heads in the oracle's bounded CPU sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    from exact_io_aware_83_b200.inputs import WORKLOADS
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -8,6 +8,8 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -23,6 +25,22 @@ using fa::FwdParams;
 
 constexpr int kMaxDevices = 64;
 
+// FA_DEBUG=1 in the environment prints the CUDA call that made an entry point return
+// FA_ERR_CUDA (to stderr).
+bool debug_enabled() {
+  static const bool on = [] {
+    const char *e = std::getenv("FA_DEBUG");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
+bool cuda_ok(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return true;
+  if (debug_enabled()) std::fprintf(stderr, "[fa] %s: %s\n", what, cudaGetErrorString(e));
+  return false;
+}
+
 // cuTensorMapEncodeTiled, fetched once through the runtime so the library does not link
 // the driver library directly.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
@@ -36,7 +54,8 @@ EncodeTiledFn encode_fn() {
   std::call_once(once, [] {
     void *p = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+    if (cuda_ok(cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q),
+                "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)") &&
         q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<EncodeTiledFn>(p);
   });
@@ -52,20 +71,25 @@ DeviceState g_dev[kMaxDevices];
 
 template <typename K>
 bool set_smem(K kernel, int bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-         cudaSuccess;
+  const bool ok = cuda_ok(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
+                          "cudaFuncSetAttribute(max dynamic shared memory)");
+  if (!ok && debug_enabled()) std::fprintf(stderr, "[fa]   requested %d bytes\n", bytes);
+  return ok;
 }
 
 bool device_ready() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice") || dev < 0 || dev >= kMaxDevices) return false;
   DeviceState &st = g_dev[dev];
   std::call_once(st.once, [&] {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return;
-    if (major != 10 || minor != 0) return;  // sm_100a code only
+    if (major != 10 || minor != 0) {  // sm_100a code only
+      if (debug_enabled()) std::fprintf(stderr, "[fa] device is sm_%d%d, not sm_100\n", major, minor);
+      return;
+    }
     bool ok = encode_fn() != nullptr;
     ok = ok && set_smem(fa::fa_fwd_kernel<64, false>, fa::FwdLayout<64>::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_kernel<64, true>, fa::FwdLayout<64>::kSmemBytes);
@@ -73,7 +97,15 @@ bool device_ready() {
     ok = ok && set_smem(fa::fa_fwd_kernel<128, true>, fa::FwdLayout<128>::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<false>, fa::FwdD256Layout::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<true>, fa::FwdD256Layout::kSmemBytes);
-    ok = ok && fa::bwd_set_attributes();
+    using fa::BwdLayout;
+    using fa::fa_bwd_main_kernel;
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, false>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, true>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, false>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, true>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, false>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, true>, BwdLayout<256, 128, 32>::kSmemBytes);
+    if (!ok && debug_enabled()) std::fprintf(stderr, "[fa] device setup failed\n");
     st.ok = ok;
   });
   return st.ok;
@@ -94,6 +126,35 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, int d, int N, long long head
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- optional event pairs around the main kernels (fa_kernel_timing)
+constexpr int kMaxTimed = 4096;
+struct KernelTimer {
+  cudaEvent_t ev[2][kMaxTimed][2] = {};
+  int count[2] = {0, 0};
+  bool enabled = false;
+};
+KernelTimer g_timer;
+
+cudaEvent_t timer_event(int which, int i, int edge) {
+  cudaEvent_t &e = g_timer.ev[which][i][edge];
+  if (!e && cudaEventCreate(&e) != cudaSuccess) e = nullptr;
+  return e;
+}
+
+// Returns the slot index to close with timer_stop, or -1 when not recording.
+int timer_start(int which, cudaStream_t s) {
+  if (!g_timer.enabled || g_timer.count[which] >= kMaxTimed) return -1;
+  const int i = g_timer.count[which];
+  cudaEvent_t a = timer_event(which, i, 0), b = timer_event(which, i, 1);
+  if (!a || !b || cudaEventRecord(a, s) != cudaSuccess) return -1;
+  return i;
+}
+
+void timer_stop(int which, int slot, cudaStream_t s) {
+  if (slot < 0) return;
+  if (cudaEventRecord(g_timer.ev[which][slot][1], s) == cudaSuccess) g_timer.count[which] = slot + 1;
+}
 
 int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale) {
   if (B < 1 || Hq < 1 || Hkv < 1 || N < 1) return FA_ERR_INVALID_ARG;
@@ -143,8 +204,10 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
   if (!make_map_bf16(&tq, q, d, N, static_cast<long long>(B) * Hq, box_rows) ||
       !make_map_bf16(&tk, k, d, N, static_cast<long long>(B) * Hkv, d == 256 ? 64 : box_rows) ||
       !make_map_bf16(&tv, v, d, N, static_cast<long long>(B) * Hkv, d == 256 ? 64 : box_rows) ||
-      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, box_rows))
+      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, box_rows)) {
+    if (debug_enabled()) std::fprintf(stderr, "[fa] cuTensorMapEncodeTiled failed (fa_fwd)\n");
     return FA_ERR_CUDA;
+  }
 
   FwdParams p;
   p.lse = lse;
@@ -157,6 +220,7 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int g = Hq / Hkv;
 
+  const int tslot = timer_start(0, s);
   if (d == 256) {
     p.pair_heads = 0;
     const unsigned units = static_cast<unsigned>(B) * Hq * p.nqb;
@@ -187,7 +251,9 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
             tq, tk, tv, to, p);
     }
   }
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const bool launched = cuda_ok(cudaGetLastError(), "fa_fwd launch");
+  timer_stop(0, tslot, s);
+  return launched ? FA_OK : FA_ERR_CUDA;
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
@@ -208,7 +274,30 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
     if (!aligned16(ptr)) return FA_ERR_ALIGN;
   if (!device_ready()) return FA_ERR_CUDA;
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, causal,
-                        scale, static_cast<cudaStream_t>(stream), encode_fn());
+                        scale, static_cast<cudaStream_t>(stream), encode_fn(), &timer_start,
+                        &timer_stop);
+}
+
+int fa_kernel_timing(int enable) {
+  if (enable != 0 && enable != 1) return FA_ERR_INVALID_ARG;
+  g_timer.enabled = enable != 0;
+  if (enable) g_timer.count[0] = g_timer.count[1] = 0;
+  return FA_OK;
+}
+
+int fa_kernel_time_ms(int which, float *ms, int *launches) {
+  if ((which != 0 && which != 1) || !ms || !launches) return FA_ERR_INVALID_ARG;
+  float total = 0.f;
+  for (int i = 0; i < g_timer.count[which]; ++i) {
+    float t = 0.f;
+    if (cudaEventSynchronize(g_timer.ev[which][i][1]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, g_timer.ev[which][i][0], g_timer.ev[which][i][1]) != cudaSuccess)
+      return FA_ERR_CUDA;
+    total += t;
+  }
+  *ms = total;
+  *launches = g_timer.count[which];
+  return FA_OK;
 }
 
 int fa_device_status(void *stream) {

@@ -524,19 +524,6 @@ inline size_t bwd_workspace_bytes(int B, int Hq, int N, int d) {
   return pad256(rows * 4) + pad256(rows * static_cast<size_t>(d) * 4);
 }
 
-template <int D, int DH, int BQ, bool CAUSAL>
-inline bool bwd_set_attr_one() {
-  return cudaFuncSetAttribute(fa_bwd_main_kernel<D, DH, BQ, CAUSAL>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              BwdLayout<D, DH, BQ>::kSmemBytes) == cudaSuccess;
-}
-
-inline bool bwd_set_attributes() {
-  return bwd_set_attr_one<64, 64, 64, false>() && bwd_set_attr_one<64, 64, 64, true>() &&
-         bwd_set_attr_one<128, 128, 64, false>() && bwd_set_attr_one<128, 128, 64, true>() &&
-         bwd_set_attr_one<256, 128, 32, false>() && bwd_set_attr_one<256, 128, 32, true>();
-}
-
 typedef CUresult (*EncodeTiledFnBwd)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                      const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
                                      const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -565,10 +552,14 @@ inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const 
       tq, tk, tv, tdo, tdk, tdv, tdq, p);
 }
 
+typedef int (*TimerStartFn)(int, cudaStream_t);
+typedef void (*TimerStopFn)(int, int, cudaStream_t);
+
 template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
-                        int Hkv, int N, int causal, float scale, cudaStream_t s, EncodeTiledFnBwd enc) {
+                        int Hkv, int N, int causal, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
+                        TimerStartFn tstart, TimerStopFn tstop) {
   const long long rows = static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
   float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
@@ -595,10 +586,12 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.scale = scale;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
+  const int tslot = tstart(1, s);
   if (causal)
     bwd_launch_main<D, DH, BQ, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
   else
     bwd_launch_main<D, DH, BQ, false>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+  tstop(1, tslot, s);
 
   const long long n8 = rows * D / 8;
   fa_bwd_post_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, s>>>(
@@ -609,16 +602,17 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
 template <typename Enc>
 inline int bwd_launch(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
-                      int Hkv, int N, int d, int causal, float scale, cudaStream_t s, Enc enc) {
+                      int Hkv, int N, int d, int causal, float scale, cudaStream_t s, Enc enc,
+                      TimerStartFn tstart, TimerStopFn tstop) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
     return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
-                                    scale, s, e);
+                                    scale, s, e, tstart, tstop);
   if (d == 128)
     return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
-                                      scale, s, e);
+                                      scale, s, e, tstart, tstop);
   return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
-                                    scale, s, e);
+                                    scale, s, e, tstart, tstop);
 }
 
 }  // namespace fa

@@ -76,7 +76,7 @@ struct FwdLayout {
 constexpr int kFwdThreads = 320;
 
 template <int D, bool CAUSAL>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                   const FwdParams p) {

@@ -66,6 +66,11 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_version.argtypes = []
         lib.fa_version.restype = ci
+        lib.fa_kernel_timing.argtypes = [ci]
+        lib.fa_kernel_timing.restype = ci
+        lib.fa_kernel_time_ms.argtypes = [ci, ctypes.POINTER(ctypes.c_float),
+                                          ctypes.POINTER(ctypes.c_int)]
+        lib.fa_kernel_time_ms.restype = ci
         _lib = lib
         return lib
 
@@ -98,6 +103,19 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq,
 
 def fa_device_status(stream=None) -> int:
     return int(load().fa_device_status(stream))
+
+
+def fa_kernel_timing(enable: bool) -> None:
+    _check(load().fa_kernel_timing(1 if enable else 0), "fa_kernel_timing")
+
+
+def fa_kernel_time_ms(which: int):
+    """(summed device ms, launches) of the forward (0) or backward main (1) kernel."""
+    ms = ctypes.c_float()
+    n = ctypes.c_int()
+    _check(load().fa_kernel_time_ms(int(which), ctypes.byref(ms), ctypes.byref(n)),
+           "fa_kernel_time_ms")
+    return float(ms.value), int(n.value)
 
 
 # ----------------------------------------------------------------------------- tensors

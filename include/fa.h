@@ -101,6 +101,20 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
  */
 int fa_device_status(void *stream);
 
+/*
+ * Kernel timing for benchmarks.  fa_kernel_timing(1) resets the counters and makes every
+ * later fa_fwd / fa_bwd call in this process record a pair of CUDA events (created by the
+ * library, no device memory) around its main attention kernel, on the call's stream;
+ * fa_kernel_timing(0) stops recording.  fa_kernel_time_ms(which, &ms, &launches)
+ * synchronises those events and returns the summed device time in milliseconds and the
+ * number of launches recorded since the reset: which = 0 for the forward kernel, 1 for
+ * the backward main kernel (the Delta and dQ-conversion kernels are not included).  At
+ * most 4096 launches per kind are recorded; later ones are not counted.  Returns FA_OK,
+ * FA_ERR_INVALID_ARG or FA_ERR_CUDA.  Not thread-safe.
+ */
+int fa_kernel_timing(int enable);
+int fa_kernel_time_ms(int which, float *ms, int *launches);
+
 /* Static, human-readable text for a status code. */
 const char *fa_status_string(int code);
 
