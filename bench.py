@@ -50,14 +50,18 @@ def _peaks():
 
 
 def _profile_traffic():
-    """DRAM bytes per launch of the backward main kernel from the committed ncu summary,
-    scaled to the benchmark workload, or None when no current capture exists."""
+    """DRAM bytes per launch of the backward main kernel from the committed ncu capture,
+    or None when there is none or the kernel source has changed since it was taken."""
+    import hashlib
     path = os.path.join(ROOT, "profiles", "bwd_main_traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
+        with open(os.path.join(ROOT, d["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != d["source_sha256"]:
+                return None
         return d
-    except (OSError, ValueError):
+    except (OSError, ValueError, KeyError):
         return None
 
 

@@ -300,6 +300,14 @@ int fa_kernel_time_ms(int which, float *ms, int *launches) {
   return FA_OK;
 }
 
+int fa_watchdog_selftest(int limit_us, void *stream) {
+  if (limit_us < 1 || limit_us > 10000000) return FA_ERR_INVALID_ARG;
+  if (!device_ready()) return FA_ERR_CUDA;
+  fa::fa_watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull);
+  return cuda_ok(cudaGetLastError(), "fa_watchdog_selftest launch") ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_device_status(void *stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
   int status = 0;

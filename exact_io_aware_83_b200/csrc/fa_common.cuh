@@ -28,12 +28,12 @@ __device__ __forceinline__ uint32_t wait_site(uint32_t kernel, uint32_t barrier,
 }
 
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       uint32_t site) {
+                                       uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       if (atomicCAS(&g_fa_status, FA_OK, FA_ERR_DEVICE_TIMEOUT) == FA_OK)
         atomicExch(&g_fa_status_site,
@@ -67,6 +67,20 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > limit_ns) return;
   }
+}
+
+// Self-test of the watchdog path: one thread waits, with a short limit, on an mbarrier
+// that nothing ever arrives at.  The wait must give up, record FA_ERR_DEVICE_TIMEOUT in
+// the status word, and return; no fault, trap or hang is involved.
+__global__ void fa_watchdog_selftest_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  const uint32_t b = smem_u32(&bar);
+  abort_flag = 0;
+  mbar_init(b, 1);
+  fence_mbar_init();
+  wait_slow(b, 0, &abort_flag, wait_site(15, 0, 0), limit_ns);
 }
 
 }  // namespace fa

@@ -66,6 +66,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_status_string.restype = ctypes.c_char_p
         lib.fa_version.argtypes = []
         lib.fa_version.restype = ci
+        lib.fa_watchdog_selftest.argtypes = [ci, vp]
+        lib.fa_watchdog_selftest.restype = ci
         lib.fa_kernel_timing.argtypes = [ci]
         lib.fa_kernel_timing.restype = ci
         lib.fa_kernel_time_ms.argtypes = [ci, ctypes.POINTER(ctypes.c_float),
@@ -103,6 +105,10 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq,
 
 def fa_device_status(stream=None) -> int:
     return int(load().fa_device_status(stream))
+
+
+def fa_watchdog_selftest(limit_us: int, stream=None) -> None:
+    _check(load().fa_watchdog_selftest(int(limit_us), stream), "fa_watchdog_selftest")
 
 
 def fa_kernel_timing(enable: bool) -> None:

@@ -115,6 +115,16 @@ int fa_device_status(void *stream);
 int fa_kernel_timing(int enable);
 int fa_kernel_time_ms(int which, float *ms, int *launches);
 
+/*
+ * Watchdog self-test: launches one thread that waits, with a limit of `limit_us`
+ * microseconds (1 .. 10^7), on a pipeline barrier that nothing ever signals - the same
+ * bounded-wait code every attention kernel uses.  The wait expires, the kernel records
+ * FA_ERR_DEVICE_TIMEOUT in the device status word and returns normally, so a following
+ * fa_device_status() reports the timeout and the CUDA context stays usable.  Returns
+ * FA_OK once enqueued, FA_ERR_INVALID_ARG or FA_ERR_CUDA.
+ */
+int fa_watchdog_selftest(int limit_us, void *stream);
+
 /* Static, human-readable text for a status code. */
 const char *fa_status_string(int code);
 
