@@ -169,6 +169,33 @@ int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale) {
   return FA_OK;
 }
 
+// ---- static scratch for fa_bwd_noalloc (callers that cannot allocate device memory)
+//
+// One buffer per GPU that loads the library, alive until the process exits.  Host code
+// must not use `g_noalloc_scratch` itself as a device address (on the host it names a
+// shadow variable); the address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+struct NoallocState {
+  std::once_flag once;
+  void *ptr = nullptr;
+};
+NoallocState g_noalloc[kMaxDevices];
+
+// Device address of the static scratch on the current device (nullptr on failure).
+// Looked up once per device, on the first fa_bwd_noalloc call made with it current.
+void *noalloc_scratch() {
+  int dev = 0;
+  if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice") || dev < 0 || dev >= kMaxDevices) return nullptr;
+  NoallocState &st = g_noalloc[dev];
+  std::call_once(st.once, [&] {
+    void *p = nullptr;
+    if (cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(no-alloc scratch)"))
+      st.ptr = p;
+  });
+  return st.ptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -185,6 +212,7 @@ const char *fa_status_string(int code) {
     case FA_ERR_WORKSPACE: return "workspace missing or too small";
     case FA_ERR_CUDA: return "CUDA error (no sm_100 device or launch failure)";
     case FA_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case FA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the static no-alloc buffer holds";
     default: return "unknown status";
   }
 }
@@ -298,6 +326,25 @@ int fa_kernel_time_ms(int which, float *ms, int *launches) {
   *ms = total;
   *launches = g_timer.count[which];
   return FA_OK;
+}
+
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                   const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N,
+                   int d, int causal, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  const size_t need = fa::bwd_workspace_bytes(B, Hq, N, d);
+  if (need > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_SCRATCH_LIMIT;
+  const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  void *scratch = noalloc_scratch();
+  if (!scratch) return FA_ERR_CUDA;
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, scratch, B, Hq, Hkv, N, d, causal, scale,
+                        static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop);
 }
 
 int fa_watchdog_selftest(int limit_us, void *stream) {

@@ -29,6 +29,8 @@ FA_ERR_ALIGN = 4
 FA_ERR_WORKSPACE = 5
 FA_ERR_CUDA = 6
 FA_ERR_DEVICE_TIMEOUT = 7
+FA_ERR_SCRATCH_LIMIT = 8
+FA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 _lock = threading.Lock()
@@ -60,6 +62,9 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd.restype = ci
+        lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                       ci, ci, ci, ci, ci, ci, cf, vp]
+        lib.fa_bwd_noalloc.restype = ci
         lib.fa_device_status.argtypes = [vp]
         lib.fa_device_status.restype = ci
         lib.fa_status_string.argtypes = [ci]
@@ -101,6 +106,15 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq,
            causal, scale, stream) -> None:
     _check(load().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
                          B, Hq, Hkv, N, d, int(causal), float(scale), stream), "fa_bwd")
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale,
+                   stream) -> None:
+    """fa_bwd for callers that cannot allocate device memory: the scratch is a static
+    64 MiB device buffer inside the library (see include/fa.h for the size limit and the
+    rule that calls overlapping on the GPU race on that buffer)."""
+    _check(load().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d,
+                                 int(causal), float(scale), stream), "fa_bwd_noalloc")
 
 
 def fa_device_status(stream=None) -> int:

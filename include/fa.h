@@ -58,7 +58,8 @@ enum fa_status {
     FA_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned */
     FA_ERR_WORKSPACE = 5,      /* workspace missing or smaller than fa_bwd_workspace_bytes() */
     FA_ERR_CUDA = 6,           /* CUDA runtime/driver error (no sm_100 device, launch failure) */
-    FA_ERR_DEVICE_TIMEOUT = 7  /* a kernel's bounded pipeline wait expired (device watchdog) */
+    FA_ERR_DEVICE_TIMEOUT = 7, /* a kernel's bounded pipeline wait expired (device watchdog) */
+    FA_ERR_SCRATCH_LIMIT = 8   /* fa_bwd_noalloc: problem needs more than FA_NOALLOC_SCRATCH_BYTES */
 };
 
 /*
@@ -93,6 +94,35 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            const void *dout, void *dq, void *dk, void *dv, void *workspace,
            size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
            float scale, void *stream);
+
+/*
+ * Backward pass for callers that cannot allocate device memory.
+ *
+ * No counterpart on the pages: this is a library convenience.  Some callers are not
+ * allowed to call cudaMalloc or a caching allocator at the point where they run the
+ * backward pass - for example code running under a fixed, pre-reserved memory budget,
+ * a real-time or latency-critical path where an allocation could block or fail, or a
+ * framework hook that must not touch the allocator.  fa_bwd needs caller-provided
+ * scratch; this variant takes none and instead uses one static device buffer of
+ * FA_NOALLOC_SCRATCH_BYTES (64 MiB) compiled into the library.  That buffer exists on
+ * every GPU that loads the library, for as long as the process lives.
+ *
+ * Arguments, layout and results are those of fa_bwd without `workspace` and
+ * `workspace_bytes`.  The problem fits when fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) <=
+ * FA_NOALLOC_SCRATCH_BYTES (for d = 128 about 130 000 query rows B*Hq*N); larger problems
+ * return FA_ERR_SCRATCH_LIMIT before anything is launched.  No call allocates memory.
+ *
+ * The first call on a device (with that device current) looks up the buffer's device
+ * address once; make that first call before any stream capture.  Every call on a device
+ * shares the same buffer, which keeps the previous call's contents (the kernels
+ * re-initialise what they need), so calls whose kernels overlap on the GPU - on different
+ * streams without ordering between them - race on it: order them on one stream or with
+ * events.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                   const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv, int N,
+                   int d, int causal, float scale, void *stream);
 
 /*
  * Synchronises `stream`, returns the device status word of the current device
