@@ -21,9 +21,11 @@
 //        dV  += P^T dO_i       (P^T read from TMEM as the A operand)
 //        dK  += dS^T Q_i       (dS^T from swizzled shared memory, K-major)
 //        dQ_i^T = K^T dS^T     (same dS^T tile read MN-major) -> fp32 TMA reduce-add
-//     Warps 0-3 own one key row each (P^T, dS^T, then the dK/dV epilogue); warps 4-7
-//     drain dQ^T from TMEM into the fp32 accumulator; warp 8 issues the MMAs; warp 9
-//     loads (TMA for K, V, Q_i, dO_i; plain loads for LSE_i and Delta_i).
+//     Warps 0-7 are two elementwise warpgroups: each thread owns one key row (its TMEM
+//     lane) and each warpgroup half of the query columns (P^T, dS^T, then the dV / dK
+//     epilogue); warps 8-11 drain dQ^T from TMEM into the fp32 accumulator; warp 12
+//     issues the MMAs; warp 13 loads (TMA for K, V, Q_i, dO_i; plain loads for LSE_i and
+//     Delta_i).
 //  3. fa_bwd_post: dQ = bf16(scale * dQacc).
 // For d = 256 the two K/V accumulators would need all 512 TMEM columns, so two CTAs
 // share each key block, each owning one 128-column half of dK, dV and dQ (both
@@ -110,7 +112,7 @@ struct BwdLayout {
   static constexpr int kKTile = kChunks * kKChunk;
   static constexpr int kQChunk = BQ * 128;          // [BQ x 64] bf16 box
   static constexpr int kQTile = kChunks * kQChunk;
-  static constexpr int kQStages = 2;
+  static constexpr int kQStages = (D == 256) ? 2 : 3;
   static constexpr int kDSRowBytes = 128;           // dS^T rows padded to one 128-B swizzle row
   static constexpr int kDSBytes = kKRows * kDSRowBytes;
   static constexpr int kDQHalves = (BQ * DH * 4 > 32768) ? 2 : 1;  // dQ staging passes
@@ -148,12 +150,22 @@ struct BwdLayout {
   static constexpr uint32_t kTmDP = 2 * DH + BQ;
   static constexpr uint32_t kTmDQ = 2 * DH + 2 * BQ;
   static constexpr uint32_t kTmemCols = 512;
+  // Elementwise work is split between two warpgroups by query column: each owns HC of
+  // the BQ columns of every key row.  Its bf16 P^T half is packed into the first HC/2
+  // columns of its OWN S^T half, so neither warpgroup overwrites scores the other has
+  // not read yet.  K-step kk (16 queries) of P^T therefore sits at column pcol(kk).
+  static constexpr int kHC = BQ / 2;
+  static constexpr int kKStepsPerHalf = kHC / 16;
+  __host__ __device__ static constexpr uint32_t pcol(int kk) {
+    return static_cast<uint32_t>((kk / kKStepsPerHalf) * kHC + (kk % kKStepsPerHalf) * 8);
+  }
   static_assert(kTmDQ + BQ <= 512, "tensor-memory budget");
   static_assert(kSmemBytes <= 232448, "shared-memory budget");
   static_assert(BQ == 32 || BQ == 64, "query block");
 };
 
-constexpr int kBwdThreads = 320;
+// Warps 0-7: two elementwise warpgroups; 8-11: dQ drain; 12: MMA; 13: loader.
+constexpr int kBwdThreads = 448;
 
 template <int D, int DH, int BQ, bool CAUSAL>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -163,6 +175,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                        const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
   using L = BwdLayout<D, DH, BQ>;
   constexpr int QS = L::kQStages;
+  constexpr int HC = L::kHC;
   constexpr int kHalves = D / DH;  // CTAs per key block
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -198,13 +211,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == L::kBarP || i == L::kBarDS || i == L::kBarDQEmpty) cnt = 128;
+      if (i == L::kBarP || i == L::kBarDS) cnt = 256;
+      if (i == L::kBarDQEmpty) cnt = 128;
+      // Q/dO stages: the TMA expect-tx arrival plus the arrival after the LSE / Delta stores.
+      if (i >= L::kBarQFull && i < L::kBarQFull + QS) cnt = 2;
       mbar_init(bar(i), cnt);
     }
     misc[1] = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(smem_u32(misc), L::kTmemCols);
     tmem_relinquish_alloc_permit();
   }
@@ -216,7 +232,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto step_head = [&](int i) { return kvh * g + i / nq; };
   auto step_q0 = [&](int i) { return (q_first + i % nq) * BQ; };
 
-  if (warp == 9) {
+  if (warp == 13) {
     // ================================================================ loader
     bool ok = true;
     if (lane == 0) {
@@ -238,16 +254,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                              wait_site(3, L::kBarQEmpty + st, i));
       if (!ok) break;
       const int h = step_head(i), q0 = step_q0(i);
-      const size_t rowbase = static_cast<size_t>(b * p.Hq + h) * p.N;
-      float *lse2 = vec + (st * 2) * BQ;
-      float *dl = vec + (st * 2 + 1) * BQ;
-      for (int c = lane; c < BQ; c += 32) {
-        const int q = q0 + c;
-        // Query rows past N get LSE = +inf, so their probabilities are exactly 0.
-        lse2[c] = q < p.N ? p.lse[rowbase + q] * 1.4426950408889634f : INFINITY;
-        dl[c] = q < p.N ? p.delta[rowbase + q] : 0.f;
-      }
-      __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(bar(L::kBarQFull + st), 2 * L::kQTile);
 #pragma unroll
@@ -258,6 +264,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       b * p.Hq + h);
         }
       }
+      const size_t rowbase = static_cast<size_t>(b * p.Hq + h) * p.N;
+      float *lse2 = vec + (st * 2) * BQ;
+      float *dl = vec + (st * 2 + 1) * BQ;
+      for (int c = lane; c < BQ; c += 32) {
+        const int q = q0 + c;
+        // Query rows past N get LSE = +inf, so their probabilities are exactly 0.
+        lse2[c] = q < p.N ? p.lse[rowbase + q] * 1.4426950408889634f : INFINITY;
+        dl[c] = q < p.N ? p.delta[rowbase + q] : 0.f;
+      }
+      // The stores above are ordered before lane 0's arrival by the warp barrier; the
+      // barrier phase completes only when that arrival and the TMA bytes are both in.
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kBarQFull + st));
       ++issued;
     }
     if (lane == 0) {
@@ -266,7 +285,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       wait_drain(bar(L::kBarKV), 0, 100000000ull);
     }
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_st = idesc_bf16_f32(128, BQ, 0, 0);   // S^T, dP^T
@@ -298,7 +317,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after_sync();
 #pragma unroll
         for (int kk = 0; kk < BQ / 16; ++kk)
-          mma_ts(tmem + L::kTmDV, tmem + L::kTmS + kk * 8,
+          mma_ts(tmem + L::kTmDV, tmem + L::kTmS + L::pcol(kk),
                  sdesc_sw128(do_t + (dcol0 / 64) * L::kQChunk + kk * 2048, L::kQChunk, 1024), id_kv,
                  (i > 0 || kk > 0));
         // Next step's S^T can start as soon as P^T has been consumed (issue order).
@@ -341,53 +360,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       wait_drain(bar(L::kBarDrain), 0, 100000000ull);
     }
     __syncwarp();
-  } else if (warp < 4) {
-    // ================================================================ P^T / dS^T (one key row per thread)
-    const int r = warp * 32 + lane;
+  } else if (warp < 8) {
+    // ================================================================ P^T / dS^T
+    // Thread = one key row (TMEM lane); warpgroup wg owns query columns [wg*HC, wg*HC+HC).
+    const int wg = warp / 4;
+    const int wq = warp % 4;
+    const int r = wq * 32 + lane;
     const int kv = kv0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tS = tmem + L::kTmS + lane_off;
-    const uint32_t tDP = tmem + L::kTmDP + lane_off;
+    const int c0 = wg * HC;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + L::kTmS + lane_off + c0;
+    const uint32_t tDP = tmem + L::kTmDP + lane_off + c0;
     const bool row_live = kv < p.N;
     const float sl2 = p.sl2;
     bool ok = true;
     for (int i = 0; ok && i < T; ++i) {
       const int st = i % QS;
-      const int q0 = step_q0(i);
+      const int q0 = step_q0(i) + c0;  // first query column of this warpgroup
       if (!(ok = warp_wait_bounded(bar(L::kBarQFull + st), (i / QS) & 1, abort_flag,
                                    wait_site(3, L::kBarQFull + st, i))))
         break;
       if (!(ok = warp_wait_bounded(bar(L::kBarS), i & 1, abort_flag, wait_site(3, L::kBarS, i)))) break;
       tc_fence_after_sync();
-      const float *lse2 = vec + (st * 2) * BQ;
-      const float *dl = vec + (st * 2 + 1) * BQ;
-      float pr[BQ];
+      const float4 *lse4 = reinterpret_cast<const float4 *>(vec + (st * 2) * BQ + c0);
+      const float4 *dl4 = reinterpret_cast<const float4 *>(vec + (st * 2 + 1) * BQ + c0);
+      float pr[HC];
+      {
+        uint32_t rr[HC];
+        if constexpr (HC == 32) tmem_ld_x32(tS, rr); else tmem_ld_x16(tS, rr);
 #pragma unroll
-      for (int c0 = 0; c0 < BQ; c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld_x32(tS + c0, rr);
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          pr[c0 + c] = ex2_approx(fmaf(__uint_as_float(rr[c]), sl2, -lse2[c0 + c]));
+        for (int c4 = 0; c4 < HC / 4; ++c4) {
+          const float4 l = lse4[c4];
+          pr[4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 0]), sl2, -l.x));
+          pr[4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 1]), sl2, -l.y));
+          pr[4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 2]), sl2, -l.z));
+          pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 3]), sl2, -l.w));
+        }
       }
       // Masks: key rows past N, and (causal) queries before this key.
       if (!row_live) {
 #pragma unroll
-        for (int c = 0; c < BQ; ++c) pr[c] = 0.f;
+        for (int c = 0; c < HC; ++c) pr[c] = 0.f;
       } else if (CAUSAL && q0 < kv) {
 #pragma unroll
-        for (int c = 0; c < BQ; ++c)
+        for (int c = 0; c < HC; ++c)
           if (q0 + c < kv) pr[c] = 0.f;
       }
       {
-        uint32_t pk[BQ / 2];
+        uint32_t pk[HC / 2];
 #pragma unroll
-        for (int c = 0; c < BQ / 2; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
-        if constexpr (BQ == 64) {
-          tmem_st_x32(tS, pk);
-        } else {
-          tmem_st_x16(tS, pk);
-        }
+        for (int c = 0; c < HC / 2; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+        if constexpr (HC == 32) tmem_st_x16(tS, pk); else tmem_st_x8(tS, pk);
       }
       tmem_wait_st();
       tc_fence_before_sync();
@@ -395,61 +418,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
       if (!(ok = warp_wait_bounded(bar(L::kBarDP), i & 1, abort_flag, wait_site(3, L::kBarDP, i)))) break;
       tc_fence_after_sync();
-      uint32_t dsk[BQ / 2];
+      uint32_t dsk[HC / 2];
+      {
+        uint32_t rr[HC];
+        if constexpr (HC == 32) tmem_ld_x32(tDP, rr); else tmem_ld_x16(tDP, rr);
 #pragma unroll
-      for (int c0 = 0; c0 < BQ; c0 += 32) {
-        uint32_t rr[32];
-        tmem_ld_x32(tDP + c0, rr);
-#pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float d0 = pr[c0 + c] * (__uint_as_float(rr[c]) - dl[c0 + c]);
-          const float d1 = pr[c0 + c + 1] * (__uint_as_float(rr[c + 1]) - dl[c0 + c + 1]);
-          dsk[(c0 + c) / 2] = pack_bf16x2(d0, d1);
+        for (int c4 = 0; c4 < HC / 4; ++c4) {
+          const float4 dd = dl4[c4];
+          dsk[2 * c4] = pack_bf16x2(pr[4 * c4 + 0] * (__uint_as_float(rr[4 * c4 + 0]) - dd.x),
+                                    pr[4 * c4 + 1] * (__uint_as_float(rr[4 * c4 + 1]) - dd.y));
+          dsk[2 * c4 + 1] = pack_bf16x2(pr[4 * c4 + 2] * (__uint_as_float(rr[4 * c4 + 2]) - dd.z),
+                                        pr[4 * c4 + 3] * (__uint_as_float(rr[4 * c4 + 3]) - dd.w));
         }
       }
-      // dS^T row r -> shared memory (128-byte swizzled row; BQ * 2 bytes used).
+      // dS^T row r, this warpgroup's 16-byte units -> shared memory (128-byte swizzled row).
       if (!(ok = warp_wait_bounded(bar(L::kBarDSEmpty), (i & 1) ^ 1, abort_flag,
                                    wait_site(3, L::kBarDSEmpty, i))))
         break;
       const uint32_t rowp = sDS + r * 128;
 #pragma unroll
-      for (int uu = 0; uu < BQ / 8; ++uu)
-        st_shared_v4(rowp + ((uu ^ (r & 7)) * 16), dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2],
+      for (int uu = 0; uu < HC / 8; ++uu) {
+        const int unit = c0 / 8 + uu;
+        st_shared_v4(rowp + ((unit ^ (r & 7)) * 16), dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2],
                      dsk[4 * uu + 3]);
+      }
       fence_proxy_async_smem();
       mbar_arrive(bar(L::kBarDS));
     }
 
-    // ---- epilogue: dV, then scale * dK -> bf16 -> shared (reusing the V / K tiles) -> TMA
+    // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK, as bf16 into the
+    // V / K tiles' shared memory (no longer read), then one thread TMA-stores both.
     bool okw = ok && warp_wait_bounded(bar(L::kBarFinal), 0, abort_flag, wait_site(3, L::kBarFinal, 0));
-    okw = named_bar_and(1, 128, okw && *abort_flag == 0);
+    okw = named_bar_and(1, 256, okw && *abort_flag == 0);
     if (okw) {
       tc_fence_after_sync();
+      const uint32_t tacc = tmem + (wg ? L::kTmDK : L::kTmDV) + lane_off;
+      const float mul = wg ? p.scale : 1.f;
+      const uint32_t stage = wg ? sK : sV;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tacc = tmem + (which ? L::kTmDK : L::kTmDV) + lane_off;
-        const float mul = which ? p.scale : 1.f;
-        const uint32_t stage = which ? sK : sV;
+      for (int cc = 0; cc < DH / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld_x32(tacc + cc * 32, o);
+        const uint32_t rowbase = stage + (cc / 2) * L::kKChunk + r * 128;
 #pragma unroll
-        for (int cc = 0; cc < DH / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld_x32(tacc + cc * 32, o);
-          const uint32_t rowbase = stage + (cc / 2) * L::kKChunk + r * 128;
+        for (int uu = 0; uu < 4; ++uu) {
+          const int unit = (cc % 2) * 4 + uu;
+          uint32_t w[4];
 #pragma unroll
-          for (int uu = 0; uu < 4; ++uu) {
-            const int unit = (cc % 2) * 4 + uu;
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * mul,
-                                 __uint_as_float(o[8 * uu + 2 * e + 1]) * mul);
-            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
-          }
+          for (int e = 0; e < 4; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * mul,
+                               __uint_as_float(o[8 * uu + 2 * e + 1]) * mul);
+          st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
         }
       }
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (r == 0) {
+      named_bar_sync(1, 256);
+      if (threadIdx.x == 0) {
 #pragma unroll
         for (int c = 0; c < DH / 64; ++c) {
           tma_store_3d(&tm_dv, sV + c * L::kKChunk, dcol0 + c * 64, kv0, b * p.Hkv + kvh);
@@ -460,13 +484,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
     }
   } else {
-    // ================================================================ dQ^T drain (warps 4-7)
-    const int wq = warp - 4;
+    // ================================================================ dQ^T drain (warps 8-11)
+    const int wq = warp - 8;
     const int dl = wq * 32 + lane;  // d column (TMEM lane) within this CTA's half
     const uint32_t tDQ = tmem + L::kTmDQ + (static_cast<uint32_t>(wq * 32) << 16);
     const bool lane_live = dl < DH;  // d = 64 pads M to 128; upper lanes are junk
     float *stage = reinterpret_cast<float *>(smem + L::kOffDQ);
-    const int tid = threadIdx.x - 128;
+    const int tid = threadIdx.x - 256;
     bool ok = true;
     for (int i = 0; ok && i < T; ++i) {
       // The warpgroup leaves the loop together: the named barriers below need all four warps.
@@ -509,7 +533,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, L::kTmemCols);
   }

@@ -292,7 +292,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const bool my_valid = t ? valid[1] : valid[0];
     const int qrow = my_qb * 128 + r;
     bool ok = my_valid;
-    float m_run = -INFINITY, l_run = 0.f;
+    // l_run: sum of the fp32 probabilities (for the LSE); r_run: sum of the same
+    // probabilities after rounding to bf16, i.e. of the weights the P V product
+    // actually used, so that O / r_run is a properly normalised average.
+    float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float sl2 = p.sl2;
     for (int j = 0; ok && j < my_n; ++j) {
       if (!warp_wait_bounded(bar(L::kBarS + t), j & 1, abort_flag, wait_site(1, L::kBarS + t, j))) {
@@ -322,7 +325,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       const float alpha = ex2_approx(m_run - m_new);  // 0 on the first block, else <= 1
       const float neg_m = -m_new;
-      float sum0 = 0.f, sum1 = 0.f;
+      float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
@@ -333,10 +336,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           sum0 += p0;
           sum1 += p1;
           pk[c] = pack_bf16x2(p0, p1);
+          rsum0 += __uint_as_float(pk[c] << 16);
+          rsum1 += __uint_as_float(pk[c] & 0xFFFF0000u);
         }
         tmem_st_x32(tS + half * 32, pk);
       }
       l_run = l_run * alpha + (sum0 + sum1);
+      r_run = r_run * alpha + (rsum0 + rsum1);
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O was last written by P V of block j-1, which completed before S_j was ready.
@@ -360,7 +366,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       okw = named_bar_and(1 + t, 128, okw && *abort_flag == 0);
       if (okw) {
         tc_fence_after_sync();
-        const float inv_l = 1.f / l_run;
+        const float inv_l = 1.f / r_run;
         const uint32_t stage = sQ + t * L::kTileBytes;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {

@@ -208,7 +208,10 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
     const uint32_t tO = tmem + L::kTmO + lane_off;
     const int qrow = qb * 128 + r;
     bool ok = true;
-    float m_run = -INFINITY, l_run = 0.f;
+    // l_run: sum of the fp32 probabilities (for the LSE); r_run: sum of the same
+    // probabilities after rounding to bf16, i.e. of the weights the P V product
+    // actually used, so that O / r_run is a properly normalised average.
+    float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float sl2 = p.sl2;
     for (int j = 0; ok && j < nblk; ++j) {
       const uint32_t tS = tmem + L::kTmS0 + (j & 1) * 64 + lane_off;
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       const float alpha = ex2_approx(m_run - m_new);
       const float neg_m = -m_new;
-      float sum0 = 0.f, sum1 = 0.f;
+      float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -249,9 +252,12 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
         sum0 += p0;
         sum1 += p1;
         pk[c] = pack_bf16x2(p0, p1);
+        rsum0 += __uint_as_float(pk[c] << 16);
+        rsum1 += __uint_as_float(pk[c] & 0xFFFF0000u);
       }
       tmem_st_x32(tS, pk);
       l_run = l_run * alpha + (sum0 + sum1);
+      r_run = r_run * alpha + (rsum0 + rsum1);
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // P V of block j-1 must have finished before O is rescaled.
@@ -278,7 +284,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
     okw = named_bar_and(1, 128, okw && *abort_flag == 0);
     if (okw) {
       tc_fence_after_sync();
-      const float inv_l = 1.f / l_run;
+      const float inv_l = 1.f / r_run;
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         uint32_t o[32];
