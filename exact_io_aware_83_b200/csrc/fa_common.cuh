@@ -27,7 +27,7 @@ __device__ __forceinline__ uint32_t wait_site(uint32_t kernel, uint32_t barrier,
   return (kernel << 24) | ((barrier & 0xFFu) << 16) | (iter & 0xFFFFu);
 }
 
-__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, volatile int *abort_flag,
                                        uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
   const uint64_t t0 = globaltimer_ns();
   while (true) {

@@ -16,7 +16,8 @@
 //    both.  Work units are ordered so the longest causal units start first.
 //  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and tile 1
 //    (one query row per thread, the row's TMEM lane); warp 8 allocates tensor memory and
-//    issues every tcgen05.mma from one lane; warp 9 issues the TMA loads from one lane.
+//    issues every tcgen05.mma from one lane; warp 9 issues the TMA loads from one lane;
+//    registers are moved from the producer warpgroup to the softmax warpgroups.
 //  * Tensor memory (512 columns): S_0 | S_1 | O_0 | O_1.  S = Q K^T lands in TMEM as
 //    fp32; the softmax warps read it, write P as bf16 over the first half of the same
 //    columns, and the MMA warp computes O += P V with P taken straight from TMEM.
@@ -73,7 +74,79 @@ struct FwdLayout {
   static_assert(kSmemBytes <= 232448, "shared-memory budget");
 };
 
-constexpr int kFwdThreads = 320;
+// Warps 0-7: softmax warpgroups of the two tiles; warp 8: MMA; warp 9: TMA; warps 10-11
+// idle.  The kernel launches with 168 registers per thread (65536 / 384, rounded down to
+// a multiple of 8); the producer warpgroup (warps 8-11) then gives registers back and the
+// softmax warpgroups take them: 2 * 128 * 216 + 128 * 72 = 64512 <= 384 * 168 = 64512,
+// and per SM sub-partition (one warp of each warpgroup) 216 + 216 + 72 <= 3 * 168.
+constexpr int kFwdThreads = 384;
+constexpr uint32_t kFwdRegsSoftmax = 216;
+constexpr uint32_t kFwdRegsProducer = 72;
+static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsProducer <= kFwdThreads * 168, "register split");
+
+// Row maximum of N raw scores (fp32 bits): four independent chains of 3-input max.
+template <int N>
+__device__ __forceinline__ float row_max(const uint32_t (&s)[N]) {
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < N; c += 8) {
+    m0 = fmax3(m0, __uint_as_float(s[c + 0]), __uint_as_float(s[c + 1]));
+    m1 = fmax3(m1, __uint_as_float(s[c + 2]), __uint_as_float(s[c + 3]));
+    m2 = fmax3(m2, __uint_as_float(s[c + 4]), __uint_as_float(s[c + 5]));
+    m3 = fmax3(m3, __uint_as_float(s[c + 6]), __uint_as_float(s[c + 7]));
+  }
+  return fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+}
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) { return row_max<128>(s); }
+
+// P = 2^(s * sl2 - m) for N scores, packed to bf16 pairs and stored to TMEM at tP (32
+// packed columns at a time, so few packed words are live at once), with the fp32 sum
+// (lsum, for the LSE) and the sum of the bf16-rounded values (rsum, the weights the
+// P V product uses).  With POLY, every fourth pair is evaluated on the FMA pipe
+// (f2_exp2_poly) instead of the MUFU unit, which is the forward's scarcest resource;
+// blocks containing masked keys use the MUFU path only so masked keys give exact zeros.
+// The caller waits for the stores (tcgen05.wait::st) before signalling the MMA warp.
+template <int N, bool POLY>
+__device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, float m, uint32_t tP, float &lsum,
+                                          float &rsum) {
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+  const uint64_t negm2 = f2_pack(-m, -m);
+  uint64_t l0 = 0, l1 = 0, r0 = 0, r1 = 0;  // packed (0.f, 0.f)
+#pragma unroll
+  for (int h = 0; h < N / 64; ++h) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int pp = h * 32 + q;
+      const uint64_t x =
+          f2_fma(f2_pack(__uint_as_float(s[2 * pp]), __uint_as_float(s[2 * pp + 1])), sl2x2, negm2);
+      uint64_t pr;
+      if (POLY && (pp & 3) == 3) {
+        pr = f2_exp2_poly(x);
+      } else {
+        float x0, x1;
+        f2_unpack(x, x0, x1);
+        pr = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      }
+      float p0, p1;
+      f2_unpack(pr, p0, p1);
+      pk[q] = pack_bf16x2(p0, p1);
+      if (pp & 1) {
+        l1 = f2_add(l1, pr);
+        r1 = f2_add(r1, bf16x2_widen(pk[q]));
+      } else {
+        l0 = f2_add(l0, pr);
+        r0 = f2_add(r0, bf16x2_widen(pk[q]));
+      }
+    }
+    tmem_st_x32(tP + h * 32, pk);
+  }
+  float a, b;
+  f2_unpack(f2_add(l0, l1), a, b);
+  lsum = a + b;
+  f2_unpack(f2_add(r0, r1), a, b);
+  rsum = a + b;
+}
 
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -145,7 +218,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = misc[0];
 
-  if (warp == 9) {
+  if (warp >= 8) {
+  // ================================================================ producer warpgroup
+  setmaxnreg_dec<kFwdRegsProducer>();
+  if (warp >= 10) {
+    // idle warps of the producer warpgroup
+  } else if (warp == 9) {
     // ================================================================ TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
@@ -277,8 +355,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       wait_drain(bar(L::kBarDrain), 0, 100000000ull);
     }
     __syncwarp();
+  }
   } else {
     // ================================================================ softmax warpgroups
+    setmaxnreg_inc<kFwdRegsSoftmax>();
     const int t = warp / 4;
     const int wq = warp % 4;          // TMEM lane quadrant of this warp
     const int r = wq * 32 + lane;     // row of the tile = TMEM lane
@@ -303,55 +383,48 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         break;
       }
       tc_fence_after_sync();
-      float s[128];
-#pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
-        uint32_t rr[32];
-        tmem_ld_x32(tS + c4 * 32, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c4 * 32 + i] = __uint_as_float(rr[i]);
+      uint32_t s[128];
+      {
+        // Two 64-column loads (a single 128-register load cannot be allocated once the
+        // warpgroup's register budget is set with setmaxnreg).
+        uint32_t (&s0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&s[0]);
+        uint32_t (&s1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&s[64]);
+        tmem_ld_x64(tS, s0);
+        tmem_ld_x64(tS + 64, s1);
       }
       const int kv0 = j * 128;
-      if ((CAUSAL && j == my_qb) || kv0 + 128 > p.N) {
+      const bool masked = (CAUSAL && j == my_qb) || kv0 + 128 > p.N;
+      if (masked) {
         const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;   // keys kv < lim are visible
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          if (kv0 + c >= lim) s[c] = -INFINITY;
+          if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
-      const float m_cand = mx * sl2;
+      const float m_cand = row_max128(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       const float alpha = ex2_approx(m_run - m_new);  // 0 on the first block, else <= 1
-      const float neg_m = -m_new;
-      float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float p0 = ex2_approx(fmaf(s[half * 64 + 2 * c], sl2, neg_m));
-          const float p1 = ex2_approx(fmaf(s[half * 64 + 2 * c + 1], sl2, neg_m));
-          sum0 += p0;
-          sum1 += p1;
-          pk[c] = pack_bf16x2(p0, p1);
-          rsum0 += __uint_as_float(pk[c] << 16);
-          rsum1 += __uint_as_float(pk[c] & 0xFFFF0000u);
-        }
-        tmem_st_x32(tS + half * 32, pk);
-      }
-      l_run = l_run * alpha + (sum0 + sum1);
-      r_run = r_run * alpha + (rsum0 + rsum1);
+      float lsum, rsum;
+      if (masked)
+        exp_block<128, false>(s, sl2, m_new, tS, lsum, rsum);   // exact zeros for masked keys
+      else
+        exp_block<128, true>(s, sl2, m_new, tS, lsum, rsum);
+      l_run = l_run * alpha + lsum;
+      r_run = r_run * alpha + rsum;
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O was last written by P V of block j-1, which completed before S_j was ready.
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld_x32(tO + cc * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), x0, x1);
+            o[i] = __float_as_uint(x0);
+            o[i + 1] = __float_as_uint(x1);
+          }
           tmem_st_x32(tO + cc * 32, o);
         }
       }

@@ -221,43 +221,26 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
         break;
       }
       tc_fence_after_sync();
-      float s[64];
-#pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        uint32_t rr[32];
-        tmem_ld_x32(tS + c2 * 32, rr);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) s[c2 * 32 + i] = __uint_as_float(rr[i]);
-      }
+      uint32_t s[64];
+      tmem_ld_x64(tS, s);
       const int kv0 = j * 64;
-      if ((CAUSAL && kv0 + 63 > qb * 128) || kv0 + 64 > p.N) {
+      const bool masked = (CAUSAL && kv0 + 63 > qb * 128) || kv0 + 64 > p.N;
+      if (masked) {
         const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (kv0 + c >= lim) s[c] = -INFINITY;
+          if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
       }
-      float mx = s[0];
-#pragma unroll
-      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, s[c]);
-      const float m_cand = mx * sl2;
+      const float m_cand = row_max<64>(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       const float alpha = ex2_approx(m_run - m_new);
-      const float neg_m = -m_new;
-      float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(fmaf(s[2 * c], sl2, neg_m));
-        const float p1 = ex2_approx(fmaf(s[2 * c + 1], sl2, neg_m));
-        sum0 += p0;
-        sum1 += p1;
-        pk[c] = pack_bf16x2(p0, p1);
-        rsum0 += __uint_as_float(pk[c] << 16);
-        rsum1 += __uint_as_float(pk[c] & 0xFFFF0000u);
-      }
-      tmem_st_x32(tS, pk);
-      l_run = l_run * alpha + (sum0 + sum1);
-      r_run = r_run * alpha + (rsum0 + rsum1);
+      float lsum, rsum;
+      if (masked)
+        exp_block<64, false>(s, sl2, m_new, tS, lsum, rsum);
+      else
+        exp_block<64, true>(s, sl2, m_new, tS, lsum, rsum);
+      l_run = l_run * alpha + lsum;
+      r_run = r_run * alpha + rsum;
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // P V of block j-1 must have finished before O is rescaled.
@@ -266,12 +249,18 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
           break;
         }
         tc_fence_after_sync();
+        const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc) {
           uint32_t o[32];
           tmem_ld_x32(tO + cc * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; i += 2) {
+            float x0, x1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), x0, x1);
+            o[i] = __float_as_uint(x0);
+            o[i + 1] = __float_as_uint(x1);
+          }
           tmem_st_x32(tO + cc * 32, o);
         }
       }
