@@ -211,8 +211,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
       uint32_t cnt = 1;
-      if (i == L::kBarP || i == L::kBarDS) cnt = 256;
-      if (i == L::kBarDQEmpty) cnt = 128;
+      if (i == L::kBarP || i == L::kBarDS) cnt = 8;   // one arrival per elementwise warp
+      if (i == L::kBarDQEmpty) cnt = 4;               // one per dQ-drain warp
       // Q/dO stages: the TMA expect-tx arrival plus the arrival after the LSE / Delta stores.
       if (i >= L::kBarQFull && i < L::kBarQFull + QS) cnt = 2;
       mbar_init(bar(i), cnt);
@@ -414,7 +414,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(bar(L::kBarP));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kBarP));
 
       if (!(ok = warp_wait_bounded(bar(L::kBarDP), i & 1, abort_flag, wait_site(3, L::kBarDP, i)))) break;
       tc_fence_after_sync();
@@ -443,7 +444,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                      dsk[4 * uu + 3]);
       }
       fence_proxy_async_smem();
-      mbar_arrive(bar(L::kBarDS));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kBarDS));
     }
 
     // ---- epilogue: warpgroup 0 writes dV, warpgroup 1 writes scale * dK, as bf16 into the
@@ -508,7 +510,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(bar(L::kBarDQEmpty));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kBarDQEmpty));
       const int h = step_head(i), q0 = step_q0(i);
 #pragma unroll
       for (int hp = 0; hp < L::kDQHalves; ++hp) {

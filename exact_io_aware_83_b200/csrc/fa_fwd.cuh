@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // ---- barriers and tensor memory
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
-      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? 4u : 1u);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -430,7 +430,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(bar(L::kBarP + t));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kBarP + t));  // one arrival per warp
     }
 
     // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store

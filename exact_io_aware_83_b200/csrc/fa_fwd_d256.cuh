@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
-      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? 128u : 1u);
+      mbar_init(bar(i), (i == L::kBarP || i == L::kBarP + 1) ? 4u : 1u);
     misc[1] = 0;
     fence_mbar_init();
   }
@@ -266,7 +266,8 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       }
       tmem_wait_st();
       tc_fence_before_sync();
-      mbar_arrive(bar(L::kBarP + (j & 1)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(L::kBarP + (j & 1)));  // one arrival per warp
     }
 
     bool okw = ok && warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0));
