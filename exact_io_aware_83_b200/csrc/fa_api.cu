@@ -69,6 +69,19 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
+// A kernel that rebalances registers with setmaxnreg must have been compiled for the
+// launch register count its split assumes; otherwise setmaxnreg.inc could never be
+// satisfied.  Refuse to use such a kernel rather than launch it.
+template <typename K>
+bool regs_at_least(K kernel, int regs) {
+  cudaFuncAttributes attr;
+  if (!cuda_ok(cudaFuncGetAttributes(&attr, kernel), "cudaFuncGetAttributes")) return false;
+  if (attr.numRegs >= regs) return true;
+  if (debug_enabled())
+    std::fprintf(stderr, "[fa] kernel compiled for %d registers per thread, split needs %d\n", attr.numRegs, regs);
+  return false;
+}
+
 template <typename K>
 bool set_smem(K kernel, int bytes) {
   const bool ok = cuda_ok(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes),
@@ -95,6 +108,10 @@ bool device_ready() {
     ok = ok && set_smem(fa::fa_fwd_kernel<64, true>, fa::FwdLayout<64>::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_kernel<128, false>, fa::FwdLayout<128>::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_kernel<128, true>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, false>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, false>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, true>, fa::kFwdRegsLaunch);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<false>, fa::FwdD256Layout::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<true>, fa::FwdD256Layout::kSmemBytes);
     using fa::BwdLayout;
@@ -227,12 +244,13 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
     return FA_ERR_ALIGN;
   if (!device_ready()) return FA_ERR_CUDA;
 
-  const int box_rows = 128;
+  // Q and O move in 128-row tiles; K and V in 128-row blocks (64-row for d = 256).
+  const int kv_rows = d == 256 ? 64 : 128;
   CUtensorMap tq, tk, tv, to;
-  if (!make_map_bf16(&tq, q, d, N, static_cast<long long>(B) * Hq, box_rows) ||
-      !make_map_bf16(&tk, k, d, N, static_cast<long long>(B) * Hkv, d == 256 ? 64 : box_rows) ||
-      !make_map_bf16(&tv, v, d, N, static_cast<long long>(B) * Hkv, d == 256 ? 64 : box_rows) ||
-      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, box_rows)) {
+  if (!make_map_bf16(&tq, q, d, N, static_cast<long long>(B) * Hq, 128) ||
+      !make_map_bf16(&tk, k, d, N, static_cast<long long>(B) * Hkv, kv_rows) ||
+      !make_map_bf16(&tv, v, d, N, static_cast<long long>(B) * Hkv, kv_rows) ||
+      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, 128)) {
     if (debug_enabled()) std::fprintf(stderr, "[fa] cuTensorMapEncodeTiled failed (fa_fwd)\n");
     return FA_ERR_CUDA;
   }

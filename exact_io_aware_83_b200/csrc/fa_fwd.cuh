@@ -78,11 +78,14 @@ struct FwdLayout {
 // idle.  The kernel launches with 168 registers per thread (65536 / 384, rounded down to
 // a multiple of 8); the producer warpgroup (warps 8-11) then gives registers back and the
 // softmax warpgroups take them: 2 * 128 * 216 + 128 * 72 = 64512 <= 384 * 168 = 64512,
-// and per SM sub-partition (one warp of each warpgroup) 216 + 216 + 72 <= 3 * 168.
+// and per SM sub-partition (one warp of each warpgroup) 216 + 216 + 72 <= 3 * 168.  The
+// host checks the launch register count before launching.
 constexpr int kFwdThreads = 384;
+constexpr uint32_t kFwdRegsLaunch = 168;
 constexpr uint32_t kFwdRegsSoftmax = 216;
 constexpr uint32_t kFwdRegsProducer = 72;
-static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsProducer <= kFwdThreads * 168, "register split");
+static_assert(2 * 128 * kFwdRegsSoftmax + 128 * kFwdRegsProducer <= kFwdThreads * kFwdRegsLaunch,
+              "register split");
 
 // Row maximum of N raw scores (fp32 bits): four independent chains of 3-input max.
 template <int N>
@@ -385,12 +388,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_after_sync();
       uint32_t s[128];
       {
-        // Two 64-column loads (a single 128-register load cannot be allocated once the
-        // warpgroup's register budget is set with setmaxnreg).
+        // Two 64-column loads and one wait (a single 128-register load cannot be
+        // allocated once the warpgroup's register budget is set with setmaxnreg).
         uint32_t (&s0)[64] = *reinterpret_cast<uint32_t(*)[64]>(&s[0]);
         uint32_t (&s1)[64] = *reinterpret_cast<uint32_t(*)[64]>(&s[64]);
-        tmem_ld_x64(tS, s0);
-        tmem_ld_x64(tS + 64, s1);
+        tmem_ld_x64_nowait(tS, s0);
+        tmem_ld_x64_nowait(tS + 64, s1);
+        tmem_wait_ld_2x64(s0, s1);
       }
       const int kv0 = j * 128;
       const bool masked = (CAUSAL && j == my_qb) || kv0 + 128 > p.N;
