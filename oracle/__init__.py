@@ -8,8 +8,8 @@ Every function takes and returns numpy float64 arrays in the ``[B, H, N, d]`` la
 
 Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy example
 of the "Consideration"/FlashAttention article page, finite differences and invariants):
-``oracle_fwd``, ``oracle_bwd`` and ``online_softmax_stats`` all have pins; none is
-"parity unpinned".
+``oracle_fwd``, ``oracle_bwd``, their key-window forms and ``online_softmax_stats`` all
+have pins; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -35,6 +35,12 @@ def _lib():
         lib.oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp,
                                    ci, ci, ci, ci, ci, ci, ctypes.c_double]
         lib.oracle_bwd.restype = ci
+        lib.oracle_fwd_window.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, ci, ci,
+                                          ctypes.c_double]
+        lib.oracle_fwd_window.restype = ci
+        lib.oracle_bwd_window.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                          ci, ci, ci, ci, ci, ci, ci, ctypes.c_double]
+        lib.oracle_bwd_window.restype = ci
         lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
         lib.oracle_online_softmax_stats.restype = ci
         _LIB = lib
@@ -95,6 +101,37 @@ def attention_bwd(q, k, v, dout, causal: bool, scale: float):
                            int(bool(causal)), float(scale))
     if rc != 0:
         raise RuntimeError(f"oracle_bwd failed with {rc}")
+    return dq, dk, dv, lse, delta
+
+
+def attention_fwd_window(q, k, v, left: int, right: int, scale: float):
+    """Local attention: key j is visible to query i iff i - left <= j <= i + right
+    (a negative bound is unlimited; causal is right = 0)."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    rc = _lib().oracle_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                  B, Hq, Hkv, N, d, int(left), int(right), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_fwd_window failed with {rc}")
+    return o, lse
+
+
+def attention_bwd_window(q, k, v, dout, left: int, right: int, scale: float):
+    """Gradient of <O, dO> for local attention: returns dq, dk, dv, lse, delta."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    delta = np.empty((B, Hq, N), dtype=np.float64)
+    rc = _lib().oracle_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _ptr(lse), _ptr(delta), B, Hq, Hkv, N, d,
+                                  int(left), int(right), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bwd_window failed with {rc}")
     return dq, dk, dv, lse, delta
 
 

@@ -15,7 +15,8 @@
  *   output = softmax(S) V), evaluated one query row at a time in fp64:
  *
  *     g      = Hq / Hkv, kv(h) = floor(h / g)          (grouped-query heads share K/V)
- *     J(i)   = {0..N-1}, or {0..i} when causal          (top-left causal mask)
+ *     J(i)   = {0..N-1}, or {0..i} when causal          (top-left causal mask), or, for
+ *              local attention with a key window, {j : i - left <= j <= i + right}
  *     s_ij   = scale * <q_i, k_j>,  j in J(i)
  *     m_i    = max_j s_ij,  l_i = sum_j exp(s_ij - m_i)
  *     LSE_i  = m_i + ln l_i                              (natural log)
@@ -58,30 +59,36 @@ static double dotd(const double *a, const double *b, int d)
     return acc;
 }
 
-/* Number of keys row i may attend to: |J(i)|. */
-static int row_extent(int i, int N, int causal)
+/*
+ * Keys visible to query row i: J(i) = {j : lo <= j < hi} with
+ *   lo = max(0, i - left)      (left  < 0: no lower limit)
+ *   hi = min(N, i + right + 1) (right < 0: no upper limit)
+ * Causal attention is right = 0; full attention is left = right = -1.
+ */
+static void row_range(int i, int N, int left, int right, int *lo, int *hi)
 {
-    return causal ? i + 1 : N;
+    *lo = (left < 0 || i - left < 0) ? 0 : i - left;
+    *hi = (right < 0 || i + right + 1 > N) ? N : i + right + 1;
 }
 
-/* s_ij for j in J(i) into s[], and the natural-log logsumexp of that row. */
-static double scores_and_lse(const double *qi, const double *kh, int i, int N, int d,
-                             int causal, double scale, double *s)
+/* s_ij for j in J(i) into s[j - lo], and the natural-log logsumexp of that row. */
+static double scores_and_lse(const double *qi, const double *kh, int lo, int hi, int d,
+                             double scale, double *s)
 {
-    const int J = row_extent(i, N, causal);
     double m = -INFINITY;
-    for (int j = 0; j < J; ++j) {
-        s[j] = scale * dotd(qi, kh + (size_t)j * d, d);
-        if (s[j] > m) m = s[j];
+    for (int j = lo; j < hi; ++j) {
+        s[j - lo] = scale * dotd(qi, kh + (size_t)j * d, d);
+        if (s[j - lo] > m) m = s[j - lo];
     }
     double l = 0.0;
-    for (int j = 0; j < J; ++j) l += exp(s[j] - m);
+    for (int j = lo; j < hi; ++j) l += exp(s[j - lo] - m);
     return m + log(l);
 }
 
-/* Forward: O [B,Hq,N,d] and LSE [B,Hq,N]. */
-int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
-               int B, int Hq, int Hkv, int N, int d, int causal, double scale)
+/* Forward with a key window: O [B,Hq,N,d] and LSE [B,Hq,N].  Every row must see at least
+ * one key (always true when left >= 0 or right >= 0 admits j = i, or for full rows). */
+int oracle_fwd_window(const double *q, const double *k, const double *v, double *o, double *lse,
+                      int B, int Hq, int Hkv, int N, int d, int left, int right, double scale)
 {
     if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !o || !lse) return -1;
     const int g = Hq / Hkv;
@@ -102,12 +109,13 @@ int oracle_fwd(const double *q, const double *k, const double *v, double *o, dou
                 const double *qi = q + (size_t)r * d;
                 const double *kh = k + ((size_t)b * Hkv + kvh) * (size_t)N * d;
                 const double *vh = v + ((size_t)b * Hkv + kvh) * (size_t)N * d;
-                const double L = scores_and_lse(qi, kh, i, N, d, causal, scale, s);
+                int lo, hi;
+                row_range(i, N, left, right, &lo, &hi);
+                const double L = scores_and_lse(qi, kh, lo, hi, d, scale, s);
                 double *oi = o + (size_t)r * d;
                 for (int c = 0; c < d; ++c) oi[c] = 0.0;
-                const int J = row_extent(i, N, causal);
-                for (int j = 0; j < J; ++j) {
-                    const double p = exp(s[j] - L);
+                for (int j = lo; j < hi; ++j) {
+                    const double p = exp(s[j - lo] - L);
                     const double *vj = vh + (size_t)j * d;
                     for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
                 }
@@ -119,6 +127,13 @@ int oracle_fwd(const double *q, const double *k, const double *v, double *o, dou
     return fail ? -2 : 0;
 }
 
+/* Forward: O [B,Hq,N,d] and LSE [B,Hq,N]; causal keeps keys j <= i. */
+int oracle_fwd(const double *q, const double *k, const double *v, double *o, double *lse,
+               int B, int Hq, int Hkv, int N, int d, int causal, double scale)
+{
+    return oracle_fwd_window(q, k, v, o, lse, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale);
+}
+
 /*
  * Backward: dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d].  lse_out and delta_out ([B,Hq,N])
  * may be NULL; when given they receive LSE_i and Delta_i.
@@ -126,9 +141,9 @@ int oracle_fwd(const double *q, const double *k, const double *v, double *o, dou
  * Pass 1 runs over query rows (LSE_i, Delta_i, dQ_i); pass 2 runs over key rows and
  * recomputes s_ij, P_ij and dP_ij for every query row that attends to that key.
  */
-int oracle_bwd(const double *q, const double *k, const double *v, const double *dout,
-               double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
-               int B, int Hq, int Hkv, int N, int d, int causal, double scale)
+int oracle_bwd_window(const double *q, const double *k, const double *v, const double *dout,
+                      double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
+                      int B, int Hq, int Hkv, int N, int d, int left, int right, double scale)
 {
     if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !dout || !dq || !dk || !dv)
         return -1;
@@ -157,17 +172,18 @@ int oracle_bwd(const double *q, const double *k, const double *v, const double *
                 const double *doi = dout + (size_t)r * d;
                 const double *kh = k + ((size_t)b * Hkv + kvh) * (size_t)N * d;
                 const double *vh = v + ((size_t)b * Hkv + kvh) * (size_t)N * d;
-                const double Li = scores_and_lse(qi, kh, i, N, d, causal, scale, s);
-                const int J = row_extent(i, N, causal);
+                int lo, hi;
+                row_range(i, N, left, right, &lo, &hi);
+                const double Li = scores_and_lse(qi, kh, lo, hi, d, scale, s);
                 double Di = 0.0;
-                for (int j = 0; j < J; ++j) {
-                    dp[j] = dotd(doi, vh + (size_t)j * d, d);
-                    Di += exp(s[j] - Li) * dp[j];
+                for (int j = lo; j < hi; ++j) {
+                    dp[j - lo] = dotd(doi, vh + (size_t)j * d, d);
+                    Di += exp(s[j - lo] - Li) * dp[j - lo];
                 }
                 double *dqi = dq + (size_t)r * d;
                 for (int c = 0; c < d; ++c) dqi[c] = 0.0;
-                for (int j = 0; j < J; ++j) {
-                    const double dS = exp(s[j] - Li) * (dp[j] - Di);
+                for (int j = lo; j < hi; ++j) {
+                    const double dS = exp(s[j - lo] - Li) * (dp[j - lo] - Di);
                     const double *kj = kh + (size_t)j * d;
                     for (int c = 0; c < d; ++c) dqi[c] += dS * kj[c];
                 }
@@ -195,8 +211,10 @@ int oracle_bwd(const double *q, const double *k, const double *v, const double *
         for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
         for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
             const size_t head = ((size_t)b * Hq + h) * (size_t)N;
-            const int i0 = causal ? j : 0;
-            for (int i = i0; i < N; ++i) {
+            /* queries that see key j: j - right <= i <= j + left */
+            const int i0 = (right < 0 || j - right < 0) ? 0 : j - right;
+            const int i1 = (left < 0 || j + left + 1 > N) ? N : j + left + 1;
+            for (int i = i0; i < i1; ++i) {
                 const double *qi = q + (head + i) * d;
                 const double *doi = dout + (head + i) * d;
                 const double s = scale * dotd(qi, kj, d);
@@ -219,6 +237,14 @@ int oracle_bwd(const double *q, const double *k, const double *v, const double *
     free(L);
     free(D);
     return 0;
+}
+
+int oracle_bwd(const double *q, const double *k, const double *v, const double *dout,
+               double *dq, double *dk, double *dv, double *lse_out, double *delta_out,
+               int B, int Hq, int Hkv, int N, int d, int causal, double scale)
+{
+    return oracle_bwd_window(q, k, v, dout, dq, dk, dv, lse_out, delta_out, B, Hq, Hkv, N, d,
+                             -1, causal ? 0 : -1, scale);
 }
 
 /*

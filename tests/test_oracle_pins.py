@@ -319,3 +319,85 @@ def test_invalid_arguments_are_rejected():
         oracle.attention_fwd(q, k, k, False, 1.0)  # Hq % Hkv != 0
     with pytest.raises(ValueError):
         oracle.attention_fwd(q, np.zeros((1, 1, 5, 2)), np.zeros((1, 1, 5, 2)), False, 1.0)
+
+
+# ---------------------------------------------------------------------------- key windows
+# Local attention keeps key j for query i iff i - left <= j <= i + right (a negative bound
+# is unlimited; causal attention is right = 0).
+
+
+def _brute_window(q, k, v, left, right, scale):
+    """Masked two-pass softmax over a full score matrix (small sizes only)."""
+    N = q.shape[0]
+    s = scale * (q @ k.T)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    vis = np.ones((N, N), dtype=bool)
+    if left >= 0:
+        vis &= j >= i - left
+    if right >= 0:
+        vis &= j <= i + right
+    s = np.where(vis, s, -np.inf)
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p / l) @ v, (m + np.log(l))[:, 0]
+
+
+@pytest.mark.parametrize("left,right", [(-1, -1), (-1, 0), (3, 0), (0, 0), (5, 2), (2, -1),
+                                        (0, 4), (100, 100)])
+def test_window_forward_equals_masked_softmax(left, right):
+    r = _rng(20 + left + 3 * right)
+    N, d, scale = 29, 8, 0.4
+    q = 3 * r.standard_normal((N, d))
+    k = r.standard_normal((N, d))
+    v = r.standard_normal((N, d))
+    o, lse = oracle.attention_fwd_window(q[None, None], k[None, None], v[None, None], left,
+                                         right, scale)
+    o_b, lse_b = _brute_window(q, k, v, left, right, scale)
+    np.testing.assert_allclose(o[0, 0], o_b, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse[0, 0], lse_b, rtol=1e-13, atol=1e-13)
+
+
+def test_window_special_cases():
+    r = _rng(31)
+    q, k, v = (r.standard_normal((2, 2, 17, 4)) for _ in range(3))
+    # Unlimited window = full attention; right = 0 with no left limit = causal.
+    for causal, (left, right) in ((False, (-1, -1)), (True, (-1, 0))):
+        o1, l1 = oracle.attention_fwd(q, k, v, causal, 0.5)
+        o2, l2 = oracle.attention_fwd_window(q, k, v, left, right, 0.5)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+    # A zero-width window keeps only the diagonal: O_i = v_i, LSE_i = s_ii.
+    o, lse = oracle.attention_fwd_window(q, k, v, 0, 0, 0.5)
+    np.testing.assert_array_equal(o, v)
+    np.testing.assert_allclose(lse, 0.5 * np.einsum("bhnd,bhnd->bhn", q, k), atol=1e-15)
+
+
+@pytest.mark.parametrize("left,right", [(2, 0), (1, 2), (-1, 1)])
+def test_window_gradients_match_central_differences(left, right):
+    r = _rng(40 + left + right)
+    N, d, scale = 6, 3, 0.6
+    q = r.standard_normal((1, 2, N, d))
+    k = r.standard_normal((1, 1, N, d))
+    v = r.standard_normal((1, 1, N, d))
+    do = r.standard_normal((1, 2, N, d))
+    dq, dk, dv, _, _ = oracle.attention_bwd_window(q, k, v, do, left, right, scale)
+
+    def loss(q_, k_, v_):
+        o, _ = oracle.attention_fwd_window(q_, k_, v_, left, right, scale)
+        return float(np.sum(o * do))
+
+    h = 1e-6
+    for name, x, grad in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v, name: xp}
+            args_m = {"q": q, "k": k, "v": v, name: xm}
+            num[idx] = (loss(args_p["q"], args_p["k"], args_p["v"])
+                        - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
+        err = np.linalg.norm(grad - num) / max(np.linalg.norm(num), 1e-30)
+        assert err < 1e-6, (name, err)
