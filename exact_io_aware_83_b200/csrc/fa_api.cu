@@ -180,10 +180,20 @@ int check_sizes(int B, int Hq, int Hkv, int N, int d, float scale) {
   if (Hq % Hkv != 0) return FA_ERR_GQA;
   // Row indices (b*H + h)*N + i must fit in int32 for the kernels' index arithmetic, and
   // the grid size in int32.
+  // N <= 2^30 keeps window arithmetic (row +- window, both below N) inside int32.
   const long long rows = static_cast<long long>(B) * Hq * N;
-  if (rows >= (1ll << 31) || static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
+  if (N > (1 << 30) || rows >= (1ll << 31) ||
+      static_cast<long long>(B) * Hq * ((N + 127) / 128) >= (1ll << 31))
     return FA_ERR_UNSUPPORTED;
   return FA_OK;
+}
+
+// Window bound as the kernels take it: -1 (unlimited) or a value below N - 1.  A bound
+// of N - 1 or more hides nothing and is unlimited too.  Bounds below -1 are rejected.
+bool normalise_window(int w, int N, int *out) {
+  if (w < -1) return false;
+  *out = (w < 0 || w >= N - 1) ? -1 : w;
+  return true;
 }
 
 // ---- static scratch for fa_bwd_noalloc (callers that cannot allocate device memory)
@@ -217,7 +227,7 @@ void *noalloc_scratch() {
 
 extern "C" {
 
-int fa_version(void) { return 100; }
+int fa_version(void) { return 101; }
 
 const char *fa_status_string(int code) {
   switch (code) {
@@ -236,10 +246,19 @@ const char *fa_status_string(int code) {
 
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
            int N, int d, int causal, float scale, void *stream) {
-  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  return fa_fwd_window(q, k, v, o, lse, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale, stream);
+}
+
+int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                  int Hkv, int N, int d, int window_left, int window_right, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
   int rc = check_sizes(B, Hq, Hkv, N, d, scale);
   if (rc != FA_OK) return rc;
+  int left = -1, right = -1;
+  if (!normalise_window(window_left, N, &left) || !normalise_window(window_right, N, &right))
+    return FA_ERR_INVALID_ARG;
+  const bool window = left >= 0 || right >= 0;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_ALIGN;
   if (!device_ready()) return FA_ERR_CUDA;
@@ -262,6 +281,8 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
   p.Hkv = Hkv;
   p.N = N;
   p.nqb = (N + 127) / 128;
+  p.left = left;
+  p.right = right;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int g = Hq / Hkv;
@@ -270,7 +291,7 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
   if (d == 256) {
     p.pair_heads = 0;
     const unsigned units = static_cast<unsigned>(B) * Hq * p.nqb;
-    if (causal)
+    if (window)
       fa::fa_fwd_d256_kernel<true><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
           tq, tk, tv, to, p);
     else
@@ -282,14 +303,14 @@ int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int
                                ? static_cast<unsigned>(B) * (Hq / 2) * p.nqb
                                : static_cast<unsigned>(B) * Hq * ((p.nqb + 1) / 2);
     if (d == 64) {
-      if (causal)
+      if (window)
         fa::fa_fwd_kernel<64, true><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(
             tq, tk, tv, to, p);
       else
         fa::fa_fwd_kernel<64, false><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(
             tq, tk, tv, to, p);
     } else {
-      if (causal)
+      if (window)
         fa::fa_fwd_kernel<128, true><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(
             tq, tk, tv, to, p);
       else
@@ -310,16 +331,27 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
            const void *dout, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
            int B, int Hq, int Hkv, int N, int d, int causal, float scale, void *stream) {
-  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  return fa_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d,
+                       -1, causal ? 0 : -1, scale, stream);
+}
+
+int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dout, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                  int B, int Hq, int Hkv, int N, int d, int window_left, int window_right, float scale,
+                  void *stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
   int rc = check_sizes(B, Hq, Hkv, N, d, scale);
   if (rc != FA_OK) return rc;
+  int left = -1, right = -1;
+  if (!normalise_window(window_left, N, &left) || !normalise_window(window_right, N, &right))
+    return FA_ERR_INVALID_ARG;
   if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(B, Hq, N, d)) return FA_ERR_WORKSPACE;
   const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
   for (const void *ptr : ptrs)
     if (!aligned16(ptr)) return FA_ERR_ALIGN;
   if (!device_ready()) return FA_ERR_CUDA;
-  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, causal,
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, left, right,
                         scale, static_cast<cudaStream_t>(stream), encode_fn(), &timer_start,
                         &timer_stop);
 }
@@ -361,7 +393,7 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, c
   if (!device_ready()) return FA_ERR_CUDA;
   void *scratch = noalloc_scratch();
   if (!scratch) return FA_ERR_CUDA;
-  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, scratch, B, Hq, Hkv, N, d, causal, scale,
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, scratch, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
                         static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop);
 }
 

@@ -9,13 +9,14 @@
 //   Delta_i = sum_j P_ij dP_ij = do_i . o_i
 //   dS_ij  = P_ij (dP_ij - Delta_i)
 //   dV_j   = sum_i P_ij do_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
-// (dK, dV summed over the query heads that share a K/V head).
+// (dK, dV summed over the query heads that share a K/V head), with P_ij = 0 for keys
+// outside query i's window i - left <= j <= i + right (causal: left unlimited, right 0).
 //
 // Three kernels on one stream:
 //  1. fa_bwd_pre:  Delta_i = <dO_i, O_i> (fp32) and a zeroed fp32 dQ accumulator.
 //  2. fa_bwd_main: one CTA per (b, K/V head, 128-key block).  It keeps K_j and V_j in
 //     shared memory and dK_j, dV_j in tensor memory, and walks every (query head of the
-//     group, 64-row query block) that can see the key block:
+//     group, 64-row query block) that can see the key block (a window skips the others):
 //        S^T  = K Q_i^T        (tcgen05, TMEM)      P^T = exp2(S^T scale log2e - LSE2_i)
 //        dP^T = V dO_i^T       (tcgen05, TMEM)      dS^T = P^T (dP^T - Delta_i)
 //        dV  += P^T dO_i       (P^T read from TMEM as the A operand)
@@ -98,6 +99,7 @@ struct BwdParams {
   const float *delta;  // [B, Hq, N]
   int B, Hq, Hkv, N;
   int nkb;             // key blocks of 128
+  int left, right;     // key window: key j seen by query i iff i - left <= j <= i + right; -1 = unlimited
   float sl2;           // scale * log2(e)
   float scale;
 };
@@ -167,7 +169,7 @@ struct BwdLayout {
 // Warps 0-7: two elementwise warpgroups; 8-11: dQ drain; 12: MMA; 13: loader.
 constexpr int kBwdThreads = 448;
 
-template <int D, int DH, int BQ, bool CAUSAL>
+template <int D, int DH, int BQ, bool WINDOW>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -192,7 +194,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- unit: (b, kv head, key block, d half); heaviest causal key blocks first
+  // ---- unit: (b, kv head, key block, d half); first key blocks (heaviest under a causal
+  // mask) first
   int u = blockIdx.x;
   const int half = u % kHalves;
   u /= kHalves;
@@ -201,11 +204,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int kvh = u % p.Hkv;
   const int b = u / p.Hkv;
   const int g = p.Hq / p.Hkv;
-  const int nqb = (p.N + BQ - 1) / BQ;
-  const int q_first = CAUSAL ? (kb * 128) / BQ : 0;
-  const int nq = nqb - q_first;
-  const int T = g * nq;  // steps: (query head of the group, query block)
   const int kv0 = kb * 128;
+  // Query blocks that can see some key of this block: queries i with
+  // j - right <= i <= j + left for a key j in [kv0, kv0 + 127].
+  const int kv1 = min(kv0 + 127, p.N - 1);
+  const int q_first = (p.right < 0 || kv0 <= p.right) ? 0 : (kv0 - p.right) / BQ;
+  const int q_last = (p.left < 0 || p.left >= p.N - 1 - kv1) ? (p.N - 1) / BQ : (kv1 + p.left) / BQ;
+  const int nq = q_last - q_first + 1;
+  const int T = g * nq;  // steps: (query head of the group, query block)
   const int dcol0 = half * DH;  // first output column owned by this CTA
 
   if (threadIdx.x == 0) {
@@ -397,14 +403,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pr[4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 3]), sl2, -l.w));
         }
       }
-      // Masks: key rows past N, and (causal) queries before this key.
+      // Masks: key rows past N, and queries q0 + c whose window misses this key
+      // (visible iff c_lo <= c <= c_hi).  Query rows past N already have P = 0.
       if (!row_live) {
 #pragma unroll
         for (int c = 0; c < HC; ++c) pr[c] = 0.f;
-      } else if (CAUSAL && q0 < kv) {
+      } else if (WINDOW) {
+        const int c_lo = p.right < 0 ? INT_MIN : kv - p.right - q0;
+        const int c_hi = p.left < 0 ? INT_MAX : kv + p.left - q0;
+        if (c_lo > 0 || c_hi < HC - 1) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c)
-          if (q0 + c < kv) pr[c] = 0.f;
+          for (int c = 0; c < HC; ++c)
+            if (c < c_lo || c > c_hi) pr[c] = 0.f;
+        }
       }
       {
         uint32_t pk[HC / 2];
@@ -571,11 +582,11 @@ inline bool bwd_map(EncodeTiledFnBwd enc, CUtensorMap *m, const void *ptr, bool 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int DH, int BQ, bool CAUSAL>
+template <int D, int DH, int BQ, bool WINDOW>
 inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
                             const CUtensorMap &tdq, const BwdParams &p, unsigned grid, cudaStream_t s) {
-  fa_bwd_main_kernel<D, DH, BQ, CAUSAL><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
+  fa_bwd_main_kernel<D, DH, BQ, WINDOW><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
       tq, tk, tv, tdo, tdk, tdv, tdq, p);
 }
 
@@ -585,7 +596,7 @@ typedef void (*TimerStopFn)(int, int, cudaStream_t);
 template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
-                        int Hkv, int N, int causal, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
+                        int Hkv, int N, int left, int right, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
                         TimerStartFn tstart, TimerStopFn tstop) {
   const long long rows = static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
@@ -610,11 +621,13 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.Hkv = Hkv;
   p.N = N;
   p.nkb = (N + 127) / 128;
+  p.left = left;
+  p.right = right;
   p.scale = scale;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
-  if (causal)
+  if (left >= 0 || right >= 0)
     bwd_launch_main<D, DH, BQ, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
   else
     bwd_launch_main<D, DH, BQ, false>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
@@ -629,16 +642,16 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
 template <typename Enc>
 inline int bwd_launch(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
-                      int Hkv, int N, int d, int causal, float scale, cudaStream_t s, Enc enc,
+                      int Hkv, int N, int d, int left, int right, float scale, cudaStream_t s, Enc enc,
                       TimerStartFn tstart, TimerStopFn tstop) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
-    return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
+    return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
                                     scale, s, e, tstart, tstop);
   if (d == 128)
-    return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
+    return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
                                       scale, s, e, tstart, tstop);
-  return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, causal,
+  return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
                                     scale, s, e, tstart, tstop);
 }
 

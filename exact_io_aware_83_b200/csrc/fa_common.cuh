@@ -7,6 +7,7 @@
 // released.  The host reads and clears the word with fa_device_status().
 #pragma once
 
+#include <climits>
 #include <cuda_bf16.h>
 
 #include "fa.h"

@@ -2,6 +2,10 @@
 //
 // What it computes (per query row i of head h, keys j in J(i)):
 //   O_i = sum_j softmax_j(scale * q_i . k_j) v_j,  LSE_i = ln sum_j exp(scale * q_i . k_j)
+// where J(i) is every key, or the local window i - left <= j <= i + right (causal
+// attention is left unlimited, right = 0; the "FlashAttention1" Q&A's scaling question,
+// item 4, pairs the method with local attention).  Key blocks no row of a tile can see
+// are skipped, not masked.
 // with the score matrix processed one 128 x 128 tile at a time and the online-softmax
 // recurrence of the "FlashAttention1" Q&A page (question on computing the softmax,
 // items 1-3): a running row maximum m, a running sum l, and a rescale of the partial
@@ -40,8 +44,38 @@ struct FwdParams {
   int B, Hq, Hkv, N;
   int nqb;          // 128-row blocks per sequence, ceil(N / 128)
   int pair_heads;   // 1: a unit is (2 heads, 1 query block); 0: (1 head, 2 query blocks)
+  int left, right;  // key window: j in [i - left, i + right]; -1 = unlimited (both < N)
   float sl2;        // scale * log2(e)
 };
+
+// First and last block of KB keys that some row of the 128-row query block qb can see.
+// Every row sees its own key, so the range is never empty and contains the diagonal.
+template <int KB>
+__device__ __forceinline__ void key_block_range(const FwdParams &p, int qb, int &lo, int &hi) {
+  const int q0 = qb * 128, q1 = min(q0 + 127, p.N - 1);
+  lo = (p.left < 0 || q0 <= p.left) ? 0 : (q0 - p.left) / KB;
+  hi = (p.right < 0 || p.right >= p.N - 1 - q1) ? (p.N - 1) / KB : (q1 + p.right) / KB;
+}
+
+// True when some key of the block [kv0, kv0 + KB) is hidden from some row of the
+// 128-row query tile starting at q0 (window edge or the end of the sequence).
+template <int KB>
+__device__ __forceinline__ bool block_needs_mask(const FwdParams &p, int q0, int kv0) {
+  return kv0 + KB > p.N || (p.left >= 0 && q0 + 127 - kv0 > p.left) ||
+         (p.right >= 0 && kv0 + KB - 1 - q0 > p.right);
+}
+
+// Hides the scores of keys kv0 + c outside row qrow's window (or past N) with -inf.
+template <int NC>
+__device__ __forceinline__ void mask_scores(uint32_t (&s)[NC], const FwdParams &p, int qrow, int kv0) {
+  // key kv0 + c is visible iff c_lo <= c < c_hi
+  const int rel = qrow - kv0;
+  const int c_lo = p.left < 0 ? INT_MIN : rel - p.left;
+  const int c_hi = min(p.N - kv0, p.right < 0 ? INT_MAX : rel + p.right + 1);
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+    if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
+}
 
 constexpr float kLn2 = 0.693147180559945309f;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
@@ -151,7 +185,7 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
   rsum = a + b;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool WINDOW>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -200,10 +234,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   }
   const int kvh = h[0] / g;
-  int nblk[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) nblk[t] = !valid[t] ? 0 : (CAUSAL ? qb[t] + 1 : p.nqb);
-  const int nmax = nblk[0] > nblk[1] ? nblk[0] : nblk[1];
+  // Key blocks: the CTA walks the union [ulo, ulo + nu) of its tiles' ranges (contiguous,
+  // since both ranges contain their tile's diagonal block and the tiles are adjacent or
+  // equal); tile t takes part in the local blocks [a[t], a[t] + nblk[t]).
+  int a[2], nblk[2], ulo, nu;
+  {
+    int lo0, hi0, lo1, hi1;
+    key_block_range<128>(p, qb[0], lo0, hi0);
+    key_block_range<128>(p, valid[1] ? qb[1] : qb[0], lo1, hi1);
+    ulo = lo0 < lo1 ? lo0 : lo1;
+    nu = (hi0 > hi1 ? hi0 : hi1) - ulo + 1;
+    a[0] = lo0 - ulo;
+    nblk[0] = hi0 - lo0 + 1;
+    a[1] = lo1 - ulo;
+    nblk[1] = valid[1] ? hi1 - lo1 + 1 : 0;
+  }
 
   // ---- barriers and tensor memory
   if (threadIdx.x == 0) {
@@ -244,7 +289,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       int issued = 0;
       bool ok = true;
-      for (int j = 0; ok && j < nmax; ++j) {
+      for (int j = 0; ok && j < nu; ++j) {
 #pragma unroll
         for (int kind = 0; kind < 2; ++kind) {
           const int seq = 2 * j + kind, slot = seq % S, use = seq / S;
@@ -258,7 +303,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_3d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, m, bar(L::kBarKVFull + slot),
-                        c * 64, j * 128, b * p.Hkv + kvh);
+                        c * 64, (ulo + j) * 128, b * p.Hkv + kvh);
           ++issued;
         }
       }
@@ -292,12 +337,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       // O_t += P_t V_j : M = 128 query rows, N = D, K = 128 keys; P (bf16) in TMEM,
       // V MN-major in shared memory (16 key rows = 2048 bytes per instruction).
-      auto issue_pv = [&](int t, int j) {
+      auto issue_pv = [&](int t, int j, bool first) {
         const uint32_t b0 = sKV + vslot(j) * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(tmem + L::tm_o(t), tmem + L::tm_s(t) + kk * 8,
-                 sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (j > 0 || kk > 0));
+                 sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (!first || kk > 0));
       };
 
       bool ok = true;
@@ -310,13 +355,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after_sync();
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!valid[t]) continue;
+          if (!valid[t] || a[t] != 0) continue;
           issue_qk(t, 0);
           tc_commit(bar(L::kBarS + t));
         }
         tc_commit(bar(L::kBarKVEmpty + kslot(0)));
       }
-      for (int j = 0; ok && j < nmax; ++j) {
+      for (int j = 0; ok && j < nu; ++j) {
         if (!wait_bounded(bar(L::kBarKVFull + vslot(j)), vpar(j), abort_flag,
                           wait_site(1, L::kBarKVFull + vslot(j), j))) {
           ok = false;
@@ -326,14 +371,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bool knext = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!ok || j >= nblk[t]) continue;
-          if (!wait_bounded(bar(L::kBarP + t), j & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
-            ok = false;
-            continue;
+          // jt: block j counted from this tile's first block; -1 means only its first
+          // S = Q K^T is due (K_{j+1} is the tile's first block).
+          const int jt = j - a[t];
+          if (!ok || !valid[t] || jt + 1 < 0 || jt >= nblk[t]) continue;
+          if (jt >= 0) {
+            if (!wait_bounded(bar(L::kBarP + t), jt & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
+              ok = false;
+              continue;
+            }
+            tc_fence_after_sync();
+            issue_pv(t, j, jt == 0);
           }
-          tc_fence_after_sync();
-          issue_pv(t, j);
-          if (j + 1 < nblk[t]) {
+          if (jt + 1 < nblk[t]) {
             if (!knext) {
               if (!wait_bounded(bar(L::kBarKVFull + kslot(j + 1)), kpar(j + 1), abort_flag,
                                 wait_site(1, L::kBarKVFull + kslot(j + 1), j + 1))) {
@@ -346,7 +396,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             issue_qk(t, j + 1);
             tc_commit(bar(L::kBarS + t));
           } else {
-            tc_commit(bar(L::kBarO + t));
+            tc_commit(bar(L::kBarO + t));  // jt is this tile's last block
           }
         }
         if (!ok) break;
@@ -372,6 +422,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int my_qb = t ? qb[1] : qb[0];
     const int my_h = t ? h[1] : h[0];
     const int my_n = t ? nblk[1] : nblk[0];
+    const int my_j0 = ulo + (t ? a[1] : a[0]);  // first key block of this tile
     const bool my_valid = t ? valid[1] : valid[0];
     const int qrow = my_qb * 128 + r;
     bool ok = my_valid;
@@ -396,20 +447,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_ld_x64_nowait(tS + 64, s1);
         tmem_wait_ld_2x64(s0, s1);
       }
-      const int kv0 = j * 128;
-      const bool masked = (CAUSAL && j == my_qb) || kv0 + 128 > p.N;
-      if (masked) {
-        const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;   // keys kv < lim are visible
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
-      }
+      const int kv0 = (my_j0 + j) * 128;
+      const bool masked = WINDOW ? block_needs_mask<128>(p, my_qb * 128, kv0) : kv0 + 128 > p.N;
+      if (masked) mask_scores<128>(s, p, qrow, kv0);
       const float m_cand = row_max128(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
-      const float alpha = ex2_approx(m_run - m_new);  // 0 on the first block, else <= 1
+      // 0 on a row's first visible block, else <= 1.  A window can hide a whole block from
+      // a row; while its max is still -inf the offset stays 0 and alpha 1 (no inf - inf).
+      const float alpha = (WINDOW && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
       float lsum, rsum;
       if (masked)
-        exp_block<128, false>(s, sl2, m_new, tS, lsum, rsum);   // exact zeros for masked keys
+        exp_block<128, false>(s, sl2, (WINDOW && m_new == -INFINITY) ? 0.f : m_new, tS, lsum,
+                              rsum);   // exact zeros for masked keys
       else
         exp_block<128, true>(s, sl2, m_new, tS, lsum, rsum);
       l_run = l_run * alpha + lsum;

@@ -56,7 +56,7 @@ struct FwdD256Layout {
 
 constexpr int kFwdD256Threads = 192;  // warps 0-3 softmax, 4 MMA, 5 TMA
 
-template <bool CAUSAL>
+template <bool WINDOW>
 __global__ void __launch_bounds__(kFwdD256Threads, 1)
     fa_fwd_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -76,15 +76,18 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- unit = (b, h, query block), longest causal blocks first
+  // ---- unit = (b, h, query block), last query blocks (longest under a causal mask) first
   int u = blockIdx.x;
   const int qb = p.nqb - 1 - (u % p.nqb);
   u /= p.nqb;
   const int h = u % p.Hq;
   const int b = u / p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
-  const int nkb_all = (p.N + 63) / 64;
-  const int nblk = CAUSAL ? min(2 * qb + 2, nkb_all) : nkb_all;
+  // 64-key blocks [jlo, jlo + nblk) that some row of the query block can see; the loop
+  // index j below counts from jlo.
+  int jlo, jhi;
+  key_block_range<64>(p, qb, jlo, jhi);
+  const int nblk = jhi - jlo + 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
@@ -128,7 +131,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(sKV + slot * L::kKVBytes + c * L::kKChunkBytes, m, bar(L::kBarKVFull + slot), c * 64,
-                      j * 64, b * p.Hkv + kvh);
+                      (jlo + j) * 64, b * p.Hkv + kvh);
         ++seq;
       };
       produce(false, 0);
@@ -223,20 +226,17 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       tc_fence_after_sync();
       uint32_t s[64];
       tmem_ld_x64(tS, s);
-      const int kv0 = j * 64;
-      const bool masked = (CAUSAL && kv0 + 63 > qb * 128) || kv0 + 64 > p.N;
-      if (masked) {
-        const int lim = CAUSAL ? min(qrow + 1, p.N) : p.N;
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
-      }
+      const int kv0 = (jlo + j) * 64;
+      const bool masked = WINDOW ? block_needs_mask<64>(p, qb * 128, kv0) : kv0 + 64 > p.N;
+      if (masked) mask_scores<64>(s, p, qrow, kv0);
       const float m_cand = row_max<64>(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
-      const float alpha = ex2_approx(m_run - m_new);
+      // A window can hide a whole block from a row: while its max is still -inf the
+      // offset stays 0 and alpha 1.
+      const float alpha = (WINDOW && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
       float lsum, rsum;
       if (masked)
-        exp_block<64, false>(s, sl2, m_new, tS, lsum, rsum);
+        exp_block<64, false>(s, sl2, (WINDOW && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum);
       else
         exp_block<64, true>(s, sl2, m_new, tS, lsum, rsum);
       l_run = l_run * alpha + lsum;

@@ -8,7 +8,10 @@ is no fallback: if the library cannot be loaded, or a call returns an error stat
 Entry points mirror the C ABI names:
 
 * :func:`fa_fwd` / :func:`fa_bwd` - pointer-level calls (device pointers as ints);
-* :func:`fwd` / :func:`bwd` - tensor conveniences that allocate outputs with torch;
+* :func:`fa_fwd_window` / :func:`fa_bwd_window` - the same for local attention (key j
+  visible to query i iff i - left <= j <= i + right, -1 = unlimited);
+* :func:`fwd` / :func:`bwd` - tensor conveniences that allocate outputs with torch
+  (``window=(left, right)`` selects local attention);
 * :func:`fa_bwd_workspace_bytes`, :func:`fa_device_status`, :func:`fa_status_string`.
 """
 from __future__ import annotations
@@ -62,6 +65,11 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd.restype = ci
+        lib.fa_fwd_window.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, vp]
+        lib.fa_fwd_window.restype = ci
+        lib.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                      ci, ci, ci, ci, ci, ci, ci, cf, vp]
+        lib.fa_bwd_window.restype = ci
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd_noalloc.restype = ci
@@ -98,6 +106,12 @@ def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream) -> None:
            "fa_fwd")
 
 
+def fa_fwd_window(q, k, v, o, lse, B, Hq, Hkv, N, d, window_left, window_right, scale,
+                  stream) -> None:
+    _check(load().fa_fwd_window(q, k, v, o, lse, B, Hq, Hkv, N, d, int(window_left),
+                                int(window_right), float(scale), stream), "fa_fwd_window")
+
+
 def fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) -> int:
     return int(load().fa_bwd_workspace_bytes(B, Hq, Hkv, N, d))
 
@@ -106,6 +120,13 @@ def fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq,
            causal, scale, stream) -> None:
     _check(load().fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
                          B, Hq, Hkv, N, d, int(causal), float(scale), stream), "fa_bwd")
+
+
+def fa_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N,
+                  d, window_left, window_right, scale, stream) -> None:
+    _check(load().fa_bwd_window(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                                B, Hq, Hkv, N, d, int(window_left), int(window_right),
+                                float(scale), stream), "fa_bwd_window")
 
 
 def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale,
@@ -165,9 +186,22 @@ def default_scale(d: int) -> float:
     return 1.0 / math.sqrt(d)
 
 
-def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
-    """O, LSE = attention(q, k, v); q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 on one GPU."""
+def _window(causal, window):
+    if window is None:
+        return None
+    if causal:
+        raise ValueError("give either causal=True or window=(left, right), not both")
+    left, right = (int(w) for w in window)
+    return left, right
+
+
+def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+        window=None):
+    """O, LSE = attention(q, k, v); q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 on one GPU.
+    ``window=(left, right)``: local attention, key j visible to query i iff
+    i - left <= j <= i + right (-1 = unlimited on that side)."""
     import torch
+    win = _window(causal, window)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n)
     B, Hq, Hkv, N, d = _dims(q, k)
@@ -176,15 +210,20 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     scale = default_scale(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
-           B, Hq, Hkv, N, d, causal, scale, _stream_handle(q))
+    if win is None:
+        fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+               B, Hq, Hkv, N, d, causal, scale, _stream_handle(q))
+    else:
+        fa_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                      B, Hq, Hkv, N, d, win[0], win[1], scale, _stream_handle(q))
     return o, l
 
 
 def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
-        workspace=None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV of <O, dO> given the forward's O and LSE."""
+        workspace=None, dq=None, dk=None, dv=None, window=None):
+    """dQ, dK, dV of <O, dO> given the forward's O and LSE (same causal / window)."""
     import torch
+    win = _window(causal, window)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _need(t, n)
     B, Hq, Hkv, N, d = _dims(q, k)
@@ -195,8 +234,11 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-           dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-           workspace.numel() * workspace.element_size(), B, Hq, Hkv, N, d, causal, scale,
-           _stream_handle(q))
+    ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+            dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+            workspace.numel() * workspace.element_size(), B, Hq, Hkv, N, d)
+    if win is None:
+        fa_bwd(*ptrs, causal, scale, _stream_handle(q))
+    else:
+        fa_bwd_window(*ptrs, win[0], win[1], scale, _stream_handle(q))
     return dq, dk, dv

@@ -20,14 +20,20 @@
  *    FlashAttention-2 page, "FlashAttention-2: Enhanced Performance";
  *  - causal masking: the deep-dive page names masking among the memory-bound steps
  *    ("Quantitative Evidence"); this library uses the top-left causal mask, key j is
- *    visible to query i when j <= i.
+ *    visible to query i when j <= i;
+ *  - local (sliding-window) attention: the "FlashAttention1" Q&A, question on scaling to
+ *    very long sequences, item 4, proposes combining the method with local attention;
+ *    the deep-dive page's closing paragraph names block-sparse FlashAttention.  Neither
+ *    defines the window; this library's reading is the band i - left <= j <= i + right,
+ *    and key blocks outside every row's band are skipped rather than masked.
  *
  * Conventions shared by every entry point
  *  - Layout: Q, dQ, O, dO are [B, Hq, N, d]; K, V, dK, dV are [B, Hkv, N, d]; all
  *    contiguous bf16 (row of d elements, then N rows, then heads, then batch).  LSE is
  *    [B, Hq, N] fp32 (natural-log logsumexp of the scaled scores of each query row).
  *  - Query head h uses K/V head h / (Hq / Hkv) (contiguous groups).
- *  - Supported head dimensions: d in {64, 128, 256}.  Any N >= 1.
+ *  - Supported head dimensions: d in {64, 128, 256}.  Any 1 <= N <= 2^30 with
+ *    B * Hq * N < 2^31.
  *  - Every pointer is a DEVICE pointer owned by the caller and must be 16-byte aligned.
  *    The library allocates no device memory except its 8-byte status words, which live
  *    in a file-scope __device__ variable.  Input buffers are read-only.
@@ -52,7 +58,8 @@ extern "C" {
 /* Status codes. */
 enum fa_status {
     FA_OK = 0,
-    FA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, non-finite/<=0 scale */
+    FA_ERR_INVALID_ARG = 1,    /* null pointer, non-positive size, non-finite/<=0 scale,
+                                  causal not 0/1, window bound below -1 */
     FA_ERR_UNSUPPORTED = 2,    /* d not in {64, 128, 256}, or sizes beyond int32 index range */
     FA_ERR_GQA = 3,            /* Hq is not a multiple of Hkv */
     FA_ERR_ALIGN = 4,          /* a pointer is not 16-byte aligned */
@@ -72,6 +79,20 @@ enum fa_status {
  */
 int fa_fwd(const void *q, const void *k, const void *v, void *o, float *lse,
            int B, int Hq, int Hkv, int N, int d, int causal, float scale, void *stream);
+
+/*
+ * Forward pass of local (sliding-window) attention.  Arguments as fa_fwd, with the mask
+ * given by two bounds instead of `causal`: key j is visible to query i iff
+ *     i - window_left <= j <= i + window_right,
+ * where a bound of -1 is unlimited on that side (values below -1 are FA_ERR_INVALID_ARG;
+ * a bound >= N - 1 hides nothing and is treated as unlimited).  Every row sees at least
+ * its own key, so every row's softmax is defined.  (-1, -1) is fa_fwd with causal = 0 and
+ * (-1, 0) is fa_fwd with causal = 1, bit for bit.  Work is proportional to the number of
+ * 128-key blocks that intersect each query tile's band.
+ */
+int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *lse,
+                  int B, int Hq, int Hkv, int N, int d, int window_left, int window_right,
+                  float scale, void *stream);
 
 /*
  * Size in bytes of the fp32 scratch that fa_bwd needs: Delta_i = <dO_i, O_i> per query
@@ -94,6 +115,16 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            const void *dout, void *dq, void *dk, void *dv, void *workspace,
            size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
            float scale, void *stream);
+
+/*
+ * Backward pass of local attention: arguments as fa_bwd, with the window bounds of
+ * fa_fwd_window in place of `causal`; q, k, v, o, lse must come from fa_fwd_window with
+ * the same bounds.  Key blocks are visited only by the query blocks whose band meets them.
+ */
+int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                  size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int window_left,
+                  int window_right, float scale, void *stream);
 
 /*
  * Backward pass for callers that cannot allocate device memory.

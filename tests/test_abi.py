@@ -25,8 +25,9 @@ def _declared_functions():
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for required in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_device_status",
-                     "fa_status_string", "fa_version"):
+    for required in ("fa_fwd", "fa_bwd", "fa_fwd_window", "fa_bwd_window",
+                     "fa_bwd_workspace_bytes", "fa_device_status", "fa_status_string",
+                     "fa_version"):
         assert required in names
 
 
@@ -40,7 +41,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert fa.load().fa_version() == 100
+    assert fa.load().fa_version() == 101
     for code in range(8):
         assert fa.fa_status_string(code) not in ("", "unknown status")
     assert fa.fa_status_string(99) == "unknown status"
@@ -99,6 +100,52 @@ def test_bwd_argument_errors(kw, code):
     assert _bwd(**kw) == code
 
 
+def _fwd_w(left, right, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, B=1, Hq=2, Hkv=1, N=16, d=128,
+             scale=0.125)
+    a.update(kw)
+    return fa.load().fa_fwd_window(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"],
+                                   a["Hkv"], a["N"], a["d"], left, right, a["scale"], None)
+
+
+def _bwd_w(left, right, **kw):
+    a = dict(B=1, Hq=2, Hkv=1, N=16, d=128, ws_bytes=1 << 30)
+    a.update(kw)
+    return fa.load().fa_bwd_window(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                   a["ws_bytes"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], left,
+                                   right, 0.125, None)
+
+
+@pytest.mark.parametrize("left,right,kw,code", [
+    (-2, 0, {}, fa.FA_ERR_INVALID_ARG),
+    (0, -2, {}, fa.FA_ERR_INVALID_ARG),
+    (-(1 << 31), -1, {}, fa.FA_ERR_INVALID_ARG),
+    (4, 4, dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (4, 4, dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (4, 4, dict(Hq=3, Hkv=2), fa.FA_ERR_GQA),
+    (4, 4, dict(o=FAKE + 8), fa.FA_ERR_ALIGN),
+    (4, 4, dict(B=1, Hq=1, Hkv=1, N=(1 << 30) + 1), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_window_argument_errors(left, right, kw, code):
+    assert _fwd_w(left, right, **kw) == code
+
+
+@pytest.mark.parametrize("left,right,kw,code", [
+    (-5, 3, {}, fa.FA_ERR_INVALID_ARG),
+    (3, -3, {}, fa.FA_ERR_INVALID_ARG),
+    (3, 3, dict(d=80), fa.FA_ERR_UNSUPPORTED),
+    (3, 3, dict(ws_bytes=100), fa.FA_ERR_WORKSPACE),
+])
+def test_bwd_window_argument_errors(left, right, kw, code):
+    assert _bwd_w(left, right, **kw) == code
+
+
+def test_binding_rejects_causal_together_with_a_window():
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.fwd(q, q, q, causal=True, window=(4, 0))
+
+
 def test_workspace_size():
     B, Hq, N, d = 2, 4, 100, 128
     rows = B * Hq * N
@@ -113,6 +160,8 @@ def test_valid_arguments_without_a_device_report_cuda_error():
     # Every argument is valid, so the call reaches the device check and stops there.
     assert _fwd() == fa.FA_ERR_CUDA
     assert _bwd() == fa.FA_ERR_CUDA
+    assert _fwd_w(3, 0) == fa.FA_ERR_CUDA
+    assert _bwd_w(-1, 7) == fa.FA_ERR_CUDA
 
 
 def test_binding_rejects_cpu_tensors():
