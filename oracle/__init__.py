@@ -8,8 +8,8 @@ Every function takes and returns numpy float64 arrays in the ``[B, H, N, d]`` la
 
 Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy example
 of the "Consideration"/FlashAttention article page, finite differences and invariants):
-``oracle_fwd``, ``oracle_bwd``, their key-window forms and ``online_softmax_stats`` all
-have pins; none is "parity unpinned".
+``oracle_fwd``, ``oracle_bwd``, their key-window forms, ``oracle_decode``,
+``oracle_merge`` and ``online_softmax_stats`` all have pins; none is "parity unpinned".
 """
 from __future__ import annotations
 
@@ -41,6 +41,12 @@ def _lib():
         lib.oracle_bwd_window.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp,
                                           ci, ci, ci, ci, ci, ci, ci, ctypes.c_double]
         lib.oracle_bwd_window.restype = ci
+        ip = ctypes.POINTER(ctypes.c_int)
+        lib.oracle_decode.argtypes = [dp, dp, dp, ip, dp, dp, ci, ci, ci, ci, ci, ci, ci,
+                                      ctypes.c_double]
+        lib.oracle_decode.restype = ci
+        lib.oracle_merge.argtypes = [dp, dp, ci, ctypes.c_longlong, ci, dp, dp]
+        lib.oracle_merge.restype = ci
         lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
         lib.oracle_online_softmax_stats.restype = ci
         _LIB = lib
@@ -133,6 +139,46 @@ def attention_bwd_window(q, k, v, dout, left: int, right: int, scale: float):
     if rc != 0:
         raise RuntimeError(f"oracle_bwd_window failed with {rc}")
     return dq, dk, dv, lse, delta
+
+
+def attention_decode(q, k, v, lens, causal: bool, scale: float):
+    """Nq queries [B,Hq,Nq,d] against the first lens[b] of Nk cached keys [B,Hkv,Nk,d]
+    (lens None: all).  Causal: the queries are the last Nq positions (bottom-right).
+    Rows that see no key get O = 0, LSE = -inf."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, dk) != (B, d) or v.shape != k.shape:
+        raise ValueError(f"shape mismatch q{q.shape} k{k.shape} v{v.shape}")
+    lens_arr = None
+    if lens is not None:
+        lens_arr = np.ascontiguousarray(np.asarray(lens, dtype=np.int32).reshape(B))
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, Nq), dtype=np.float64)
+    lp = None if lens_arr is None else lens_arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+    rc = _lib().oracle_decode(_ptr(q), _ptr(k), _ptr(v), lp, _ptr(o), _ptr(lse), B, Hq, Hkv,
+                              Nq, Nk, d, int(bool(causal)), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_decode failed with {rc}")
+    return o, lse
+
+
+def merge(o_parts, lse_parts):
+    """Combine S partial results over disjoint key sets: o_parts [S, ..., d] (each part
+    normalised), lse_parts [S, ...] -> (o [..., d], lse [...])."""
+    op = _as_f64(o_parts)
+    lp = _as_f64(lse_parts)
+    S = op.shape[0]
+    d = op.shape[-1]
+    if lp.shape != op.shape[:-1]:
+        raise ValueError("lse_parts must be o_parts without its last axis")
+    rows = int(np.prod(op.shape[1:-1])) if op.ndim > 2 else 1
+    o = np.empty(op.shape[1:], dtype=np.float64)
+    lse = np.empty(lp.shape[1:], dtype=np.float64)
+    rc = _lib().oracle_merge(_ptr(op), _ptr(lp), S, rows, d, _ptr(o), _ptr(lse))
+    if rc != 0:
+        raise RuntimeError(f"oracle_merge failed with {rc}")
+    return o, lse
 
 
 def online_softmax_stats(scores, block: int):

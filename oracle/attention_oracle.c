@@ -277,3 +277,98 @@ int oracle_online_softmax_stats(const double *s, int n, int block, double *m_out
     *l_out = l;
     return 0;
 }
+
+/*
+ * Attention of Nq query rows against a cache of Nk key rows, of which the first lens[b]
+ * are valid in batch b (lens == NULL: all Nk).  This is the incremental case of the
+ * "FlashAttention1" Q&A page (question on scaling to long sequences, item 8: incremental
+ * attention updates for streaming inference): the newest Nq tokens attend to everything
+ * cached so far.  With `causal` the queries are the LAST Nq positions of the sequence
+ * (bottom-right alignment): query t sits at position lens[b] - Nq + t and sees keys
+ * j <= lens[b] - Nq + t.  A query that sees no key gets O = 0 and LSE = -inf.
+ * q, o: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d]; lse: [B, Hq, Nq].
+ */
+int oracle_decode(const double *q, const double *k, const double *v, const int *lens,
+                  double *o, double *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                  int causal, double scale)
+{
+    if (check_args(B, Hq, Hkv, Nq, d) || Nk < 1 || !q || !k || !v || !o || !lse) return -1;
+    if (lens)
+        for (int b = 0; b < B; ++b)
+            if (lens[b] < 0 || lens[b] > Nk) return -1;
+    const int g = Hq / Hkv;
+    const long long rows = (long long)B * Hq * Nq;
+    int fail = 0;
+#pragma omp parallel reduction(|: fail)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)Nk);
+        if (!s) {
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4)
+            for (long long r = 0; r < rows; ++r) {
+                const int t = (int)(r % Nq);
+                const long long bh = r / Nq;
+                const int h = (int)(bh % Hq), b = (int)(bh / Hq);
+                const int len = lens ? lens[b] : Nk;
+                int hi = len;
+                if (causal && len - Nq + t + 1 < hi) hi = len - Nq + t + 1;
+                double *oi = o + (size_t)r * d;
+                for (int c = 0; c < d; ++c) oi[c] = 0.0;
+                if (hi <= 0) {
+                    lse[r] = -INFINITY;
+                    continue;
+                }
+                const double *kh = k + ((size_t)b * Hkv + h / g) * (size_t)Nk * d;
+                const double *vh = v + ((size_t)b * Hkv + h / g) * (size_t)Nk * d;
+                const double L = scores_and_lse(q + (size_t)r * d, kh, 0, hi, d, scale, s);
+                for (int j = 0; j < hi; ++j) {
+                    const double p = exp(s[j] - L);
+                    const double *vj = vh + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
+                }
+                lse[r] = L;
+            }
+            free(s);
+        }
+    }
+    return fail ? -2 : 0;
+}
+
+/*
+ * Merge of S partial attention results over disjoint key sets: the "efficient reduction"
+ * that combines partial results of different blocks ("FlashAttention1" Q&A, question on
+ * the key algorithmic innovations, item 3), in the log-sum-exp form of the softmax
+ * recurrence on the same page (question on computing the softmax):
+ *     LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s
+ * where O_s is part s's normalised output.  Parts with LSE_s = -inf (no visible key)
+ * contribute nothing; when every part is -inf, O = 0 and LSE = -inf.
+ * o_parts: [S, rows, d]; lse_parts: [S, rows]; o: [rows, d]; lse: [rows].
+ */
+int oracle_merge(const double *o_parts, const double *lse_parts, int S, long long rows, int d,
+                 double *o, double *lse)
+{
+    if (!o_parts || !lse_parts || !o || !lse || S < 1 || rows < 1 || d < 1) return -1;
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < rows; ++r) {
+        double m = -INFINITY;
+        for (int s = 0; s < S; ++s)
+            if (lse_parts[(size_t)s * rows + r] > m) m = lse_parts[(size_t)s * rows + r];
+        double *orow = o + (size_t)r * d;
+        for (int c = 0; c < d; ++c) orow[c] = 0.0;
+        if (m == -INFINITY) {
+            lse[r] = -INFINITY;
+            continue;
+        }
+        double l = 0.0;
+        for (int s = 0; s < S; ++s) l += exp(lse_parts[(size_t)s * rows + r] - m);
+        const double L = m + log(l);
+        for (int s = 0; s < S; ++s) {
+            const double w = exp(lse_parts[(size_t)s * rows + r] - L);
+            const double *op = o_parts + ((size_t)s * rows + r) * d;
+            for (int c = 0; c < d; ++c) orow[c] += w * op[c];
+        }
+        lse[r] = L;
+    }
+    return 0;
+}

@@ -14,7 +14,12 @@ the causal mask on the wrong side, a missing scale) fails at least one test:
 * scipy's logsumexp for the LSE;
 * central finite differences of L = <O, dO> for the gradient;
 * Delta_i = <dO_i, O_i>, sum_j dK_j = 0, sum_j dV_j = sum_i dO_i;
-* grouped-query attention equals multi-head attention with repeated K/V.
+* grouped-query attention equals multi-head attention with repeated K/V;
+* local attention against a brute-force masked softmax and its full/causal special cases;
+* decode (queries at the end of a longer cache) against a bottom-right-masked softmax on
+  the full score matrix, the square forward, and single-key / no-key closed forms;
+* the merge of partial results against attention over the union of the key ranges, and
+  closed forms (one part, equal weights, weights 1/4 and 3/4, all parts empty).
 """
 import math
 import os
@@ -401,3 +406,128 @@ def test_window_gradients_match_central_differences(left, right):
                         - loss(args_m["q"], args_m["k"], args_m["v"])) / (2 * h)
         err = np.linalg.norm(grad - num) / max(np.linalg.norm(num), 1e-30)
         assert err < 1e-6, (name, err)
+
+
+# ---------------------------------------------------------------------------- decode / merge
+
+def _brute_decode(q, k, v, lens, causal, scale):
+    """Bottom-right-aligned masked softmax on the full score matrix, with numpy."""
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    o = np.zeros_like(q)
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        n = Nk if lens is None else lens[b]
+        for h in range(Hq):
+            s = scale * q[b, h] @ k[b, h // g, :n].T               # [Nq, n]
+            if causal:
+                pos = n - Nq + np.arange(Nq)                        # absolute query positions
+                s = np.where(np.arange(n)[None, :] <= pos[:, None], s, -np.inf)
+            for t in range(Nq):
+                if not np.isfinite(s[t]).any():
+                    continue
+                lse[b, h, t] = scipy.special.logsumexp(s[t])
+                o[b, h, t] = np.exp(s[t] - lse[b, h, t]) @ v[b, h // g, :n]
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk,lens", [(1, 9, None), (3, 9, [9, 4]), (4, 6, [2, 6]),
+                                         (5, 5, [0, 5]), (2, 7, [1, 7])])
+def test_decode_equals_bottom_right_masked_softmax(causal, Nq, Nk, lens):
+    r = _rng(31 + Nq * 7 + Nk)
+    q = r.normal(size=(2, 4, Nq, 8))
+    k = r.normal(size=(2, 2, Nk, 8))
+    v = r.normal(size=(2, 2, Nk, 8))
+    o, lse = oracle.attention_decode(q, k, v, lens, causal, 0.4)
+    o_ref, lse_ref = _brute_decode(q, k, v, lens, causal, 0.4)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(lse_ref))
+    fin = np.isfinite(lse_ref)
+    np.testing.assert_allclose(lse[fin], lse_ref[fin], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_decode_with_nq_equal_nk_is_the_square_forward(causal):
+    # When the queries are the whole sequence, bottom-right and top-left alignment agree.
+    r = _rng(41)
+    q, k, v = r.normal(size=(2, 4, 11, 6)), r.normal(size=(2, 2, 11, 6)), r.normal(size=(2, 2, 11, 6))
+    o1, l1 = oracle.attention_decode(q, k, v, None, causal, 0.3)
+    o2, l2 = oracle.attention_fwd(q, k, v, causal, 0.3)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+
+
+def test_decode_special_cases():
+    r = _rng(43)
+    q, k, v = r.normal(size=(2, 2, 1, 5)), r.normal(size=(2, 1, 8, 5)), r.normal(size=(2, 1, 8, 5))
+    # One query: the causal mask hides nothing.
+    o1, l1 = oracle.attention_decode(q, k, v, [8, 3], True, 0.5)
+    o2, l2 = oracle.attention_decode(q, k, v, [8, 3], False, 0.5)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    # lens[b] valid keys equal a cache that holds only those keys.
+    o3, l3 = oracle.attention_decode(q[1:], k[1:, :, :3], v[1:, :, :3], None, False, 0.5)
+    np.testing.assert_allclose(o2[1:], o3, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(l2[1:], l3, rtol=0, atol=1e-14)
+    # A single visible key: O is that key's value row, LSE its scaled score.
+    o4, l4 = oracle.attention_decode(q, k, v, [1, 1], False, 0.5)
+    np.testing.assert_allclose(o4[:, :, 0], np.broadcast_to(v[:, :, 0], (2, 2, 5)), atol=1e-15)
+    np.testing.assert_allclose(l4[:, :, 0], 0.5 * np.einsum("bhd,bd->bh", q[:, :, 0], k[:, 0, 0]),
+                               atol=1e-14)
+    # No visible key: O = 0, LSE = -inf.
+    o5, l5 = oracle.attention_decode(q, k, v, [0, 2], False, 0.5)
+    assert np.all(o5[0] == 0) and np.all(np.isneginf(l5[0]))
+    with pytest.raises(RuntimeError):
+        oracle.attention_decode(q, k, v, [9, 1], False, 0.5)   # more keys than the cache
+
+
+@pytest.mark.parametrize("bounds", [[0, 4, 9, 16], [0, 1, 2, 16], [0, 16], [0, 5, 5, 12, 16]])
+def test_merge_of_disjoint_key_ranges_is_full_attention(bounds):
+    # Attention over each key range separately, merged, equals attention over all keys; an
+    # empty range (LSE = -inf) contributes nothing.
+    r = _rng(47)
+    q, k, v = r.normal(size=(1, 3, 4, 7)), r.normal(size=(1, 3, 16, 7)), r.normal(size=(1, 3, 16, 7))
+    parts_o, parts_l = [], []
+    for a, b in zip(bounds[:-1], bounds[1:]):
+        if b == a:
+            parts_o.append(np.full_like(q, 123.0))   # must be ignored: its weight is zero
+            parts_l.append(np.full(q.shape[:-1], -np.inf))
+        else:
+            o_s, l_s = oracle.attention_decode(q, k[:, :, a:b], v[:, :, a:b], None, False, 0.35)
+            parts_o.append(o_s)
+            parts_l.append(l_s)
+    o, lse = oracle.merge(np.stack(parts_o), np.stack(parts_l))
+    o_ref, lse_ref = oracle.attention_decode(q, k, v, None, False, 0.35)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_ref, rtol=0, atol=1e-13)
+
+
+def test_merge_closed_forms():
+    r = _rng(53)
+    o1 = r.normal(size=(1, 3, 4))
+    l1 = r.normal(size=(1, 3))
+    # One part: identity.
+    o, lse = oracle.merge(o1, l1)
+    np.testing.assert_array_equal(o, o1[0])
+    np.testing.assert_array_equal(lse, l1[0])
+    # Two parts with equal LSE: the mean, and LSE + ln 2.
+    o2 = r.normal(size=(1, 3, 4))
+    o, lse = oracle.merge(np.concatenate([o1, o2]), np.concatenate([l1, l1]))
+    np.testing.assert_allclose(o, 0.5 * (o1[0] + o2[0]), atol=1e-15)
+    np.testing.assert_allclose(lse, l1[0] + math.log(2.0), atol=1e-15)
+    # LSEs 0 and ln 3: weights 1/4 and 3/4.
+    l2 = np.zeros((1, 3))
+    l3 = np.full((1, 3), math.log(3.0))
+    o, lse = oracle.merge(np.concatenate([o1, o2]), np.concatenate([l2, l3]))
+    np.testing.assert_allclose(o, 0.25 * o1[0] + 0.75 * o2[0], atol=1e-15)
+    np.testing.assert_allclose(lse, math.log(4.0), atol=1e-15)
+    # All parts empty.
+    o, lse = oracle.merge(np.concatenate([o1, o2]), np.full((2, 3), -np.inf))
+    assert np.all(o == 0) and np.all(np.isneginf(lse))
+    # Order of the parts does not matter.
+    oa, la = oracle.merge(np.concatenate([o1, o2]), np.concatenate([l1, l3]))
+    ob, lb = oracle.merge(np.concatenate([o2, o1]), np.concatenate([l3, l1]))
+    np.testing.assert_allclose(oa, ob, atol=1e-15)
+    np.testing.assert_allclose(la, lb, atol=1e-15)
