@@ -18,6 +18,7 @@
 #include "fa_fwd.cuh"
 #include "fa_fwd_d256.cuh"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 
 namespace {
 
@@ -122,6 +123,17 @@ bool device_ready() {
     ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, true>, BwdLayout<128, 128, 64>::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, false>, BwdLayout<256, 128, 32>::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, true>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<64, 16>, fa::DecodeLayout<64, 16>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<64, 32>, fa::DecodeLayout<64, 32>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<64, 64>, fa::DecodeLayout<64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<64, 128>, fa::DecodeLayout<64, 128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<128, 16>, fa::DecodeLayout<128, 16>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<128, 32>, fa::DecodeLayout<128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<128, 64>, fa::DecodeLayout<128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<128, 128>, fa::DecodeLayout<128, 128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<256, 16>, fa::DecodeLayout<256, 16>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<256, 32>, fa::DecodeLayout<256, 32>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_decode_kernel<256, 64>, fa::DecodeLayout<256, 64>::kSmemBytes);
     if (!ok && debug_enabled()) std::fprintf(stderr, "[fa] device setup failed\n");
     st.ok = ok;
   });
@@ -147,8 +159,8 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // ---- optional event pairs around the main kernels (fa_kernel_timing)
 constexpr int kMaxTimed = 4096;
 struct KernelTimer {
-  cudaEvent_t ev[2][kMaxTimed][2] = {};
-  int count[2] = {0, 0};
+  cudaEvent_t ev[3][kMaxTimed][2] = {};
+  int count[3] = {0, 0, 0};
   bool enabled = false;
 };
 KernelTimer g_timer;
@@ -221,6 +233,56 @@ void *noalloc_scratch() {
       st.ptr = p;
   });
   return st.ptr;
+}
+
+// ---- decode (a few new query rows against a long cache) and the merge of partials
+
+constexpr int kMaxDecodeSplits = 1024;
+
+// Query rows handled by one decode CTA, padded to the MMA width the kernel is built for.
+int decode_rows_padded(int R) { return R <= 16 ? 16 : R <= 32 ? 32 : R <= 64 ? 64 : 128; }
+
+int check_decode_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return FA_ERR_GQA;
+  const long long R = static_cast<long long>(Hq / Hkv) * Nq;
+  if (R > (d == 256 ? 64 : 128)) return FA_ERR_UNSUPPORTED;
+  if (Nk > (1 << 30) || static_cast<long long>(B) * Hq * Nq >= (1ll << 31) ||
+      static_cast<long long>(B) * Hkv * Nk >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t decode_workspace(int B, int Hq, int Nq, int d, int splits) {
+  if (splits <= 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+  return fa::pad256(static_cast<size_t>(splits) * rows * d * 4) + fa::pad256(static_cast<size_t>(splits) * rows * 4);
+}
+
+template <int D, int RP>
+void launch_decode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                   const fa::DecodeParams &p, unsigned grid, cudaStream_t s) {
+  fa::fa_decode_kernel<D, RP><<<grid, fa::kDecodeThreads, fa::DecodeLayout<D, RP>::kSmemBytes, s>>>(tq, tk, tv, p);
+}
+
+template <int D>
+void launch_decode_d(int RP, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
+                     const fa::DecodeParams &p, unsigned grid, cudaStream_t s) {
+  if (RP == 16) launch_decode<D, 16>(tq, tk, tv, p, grid, s);
+  else if (RP == 32) launch_decode<D, 32>(tq, tk, tv, p, grid, s);
+  else if (RP == 64) launch_decode<D, 64>(tq, tk, tv, p, grid, s);
+  else if constexpr (D != 256) launch_decode<D, 128>(tq, tk, tv, p, grid, s);
+}
+
+void launch_merge(const float *o_part, const float *lse_part, void *o, float *lse, int S, long long rows,
+                  int d, cudaStream_t s) {
+  const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+  __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(o);
+  if (d == 64) fa::fa_merge_kernel<64><<<grid, 256, 0, s>>>(o_part, lse_part, ob, lse, S, rows);
+  else if (d == 128) fa::fa_merge_kernel<128><<<grid, 256, 0, s>>>(o_part, lse_part, ob, lse, S, rows);
+  else fa::fa_merge_kernel<256><<<grid, 256, 0, s>>>(o_part, lse_part, ob, lse, S, rows);
 }
 
 }  // namespace
@@ -359,12 +421,12 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, co
 int fa_kernel_timing(int enable) {
   if (enable != 0 && enable != 1) return FA_ERR_INVALID_ARG;
   g_timer.enabled = enable != 0;
-  if (enable) g_timer.count[0] = g_timer.count[1] = 0;
+  if (enable) g_timer.count[0] = g_timer.count[1] = g_timer.count[2] = 0;
   return FA_OK;
 }
 
 int fa_kernel_time_ms(int which, float *ms, int *launches) {
-  if ((which != 0 && which != 1) || !ms || !launches) return FA_ERR_INVALID_ARG;
+  if (which < 0 || which > 2 || !ms || !launches) return FA_ERR_INVALID_ARG;
   float total = 0.f;
   for (int i = 0; i < g_timer.count[which]; ++i) {
     float t = 0.f;
@@ -403,6 +465,99 @@ int fa_watchdog_selftest(int limit_us, void *stream) {
   fa::fa_watchdog_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint64_t>(limit_us) * 1000ull);
   return cuda_ok(cudaGetLastError(), "fa_watchdog_selftest launch") ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_decode_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  if (check_decode_sizes(B, Hq, Hkv, Nq, Nk, d, 1.0f) != FA_OK) return 0;
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    (void)cudaGetLastError();
+    sms = 148;
+  }
+  // One CTA per SM: as many splits as fit into one wave of (b, K/V head) units, but at
+  // least two 128-key blocks per split so each CTA streams a few blocks.
+  const long long units = static_cast<long long>(B) * Hkv;
+  long long s = units >= sms ? 1 : sms / units;
+  const long long blocks = (Nk + 127) / 128;
+  const long long max_by_len = blocks / 2 > 1 ? blocks / 2 : 1;
+  if (s > max_by_len) s = max_by_len;
+  if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;
+  return static_cast<int>(s < 1 ? 1 : s);
+}
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits) {
+  if (check_decode_sizes(B, Hq, Hkv, Nq, Nk, d, 1.0f) != FA_OK) return 0;
+  if (num_splits < 1 || num_splits > kMaxDecodeSplits) return 0;
+  return decode_workspace(B, Hq, Nq, d, num_splits);
+}
+
+int fa_decode(const void *q, const void *k, const void *v, void *o, float *lse, const int *seqlens_k,
+              void *workspace, size_t workspace_bytes, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+              int causal, int num_splits, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (num_splits < 1 || num_splits > kMaxDecodeSplits) return FA_ERR_INVALID_ARG;
+  int rc = check_decode_sizes(B, Hq, Hkv, Nq, Nk, d, scale);
+  if (rc != FA_OK) return rc;
+  if (static_cast<long long>(B) * Hkv * num_splits >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  const size_t need = decode_workspace(B, Hq, Nq, d, num_splits);
+  if (need > 0 && (!workspace || workspace_bytes < need)) return FA_ERR_WORKSPACE;
+  const void *ptrs[] = {q, k, v, o, lse};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if ((need > 0 && !aligned16(workspace)) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+
+  const int g = Hq / Hkv, R = g * Nq, RP = decode_rows_padded(R);
+  CUtensorMap tq, tk, tv;
+  // Q viewed as [B * Hkv][R][d]: the rows of the query heads that share a K/V head.
+  if (!make_map_bf16(&tq, q, d, R, static_cast<long long>(B) * Hkv, RP) ||
+      !make_map_bf16(&tk, k, d, Nk, static_cast<long long>(B) * Hkv, 128) ||
+      !make_map_bf16(&tv, v, d, Nk, static_cast<long long>(B) * Hkv, 128)) {
+    if (debug_enabled()) std::fprintf(stderr, "[fa] cuTensorMapEncodeTiled failed (fa_decode)\n");
+    return FA_ERR_CUDA;
+  }
+  const size_t rows = static_cast<size_t>(B) * Hq * Nq;
+  fa::DecodeParams p;
+  p.lens = seqlens_k;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.lse = lse;
+  p.o_part = num_splits > 1 ? static_cast<float *>(workspace) : nullptr;
+  p.lse_part = num_splits > 1
+                   ? reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                               fa::pad256(static_cast<size_t>(num_splits) * rows * d * 4))
+                   : nullptr;
+  p.B = B;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.R = R;
+  p.splits = num_splits;
+  const int per = (Nk + num_splits - 1) / num_splits;
+  p.chunk = (per + 127) / 128 * 128;
+  p.causal = causal;
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const unsigned grid = static_cast<unsigned>(B) * Hkv * num_splits;
+  const int tslot = timer_start(2, s);
+  if (d == 64) launch_decode_d<64>(RP, tq, tk, tv, p, grid, s);
+  else if (d == 128) launch_decode_d<128>(RP, tq, tk, tv, p, grid, s);
+  else launch_decode_d<256>(RP, tq, tk, tv, p, grid, s);
+  timer_stop(2, tslot, s);
+  if (num_splits > 1) launch_merge(p.o_part, p.lse_part, o, lse, num_splits, static_cast<long long>(rows), d, s);
+  return cuda_ok(cudaGetLastError(), "fa_decode launch") ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_merge(const float *o_parts, const float *lse_parts, void *o, float *lse, int num_parts, int rows,
+             int d, void *stream) {
+  if (!o_parts || !lse_parts || !o || !lse || num_parts < 1 || rows < 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(num_parts) * rows * d >= (1ll << 40)) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(lse_parts) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  launch_merge(o_parts, lse_parts, o, lse, num_parts, rows, d, static_cast<cudaStream_t>(stream));
+  return cuda_ok(cudaGetLastError(), "fa_merge launch") ? FA_OK : FA_ERR_CUDA;
 }
 
 int fa_device_status(void *stream) {

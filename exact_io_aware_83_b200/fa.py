@@ -10,8 +10,10 @@ Entry points mirror the C ABI names:
 * :func:`fa_fwd` / :func:`fa_bwd` - pointer-level calls (device pointers as ints);
 * :func:`fa_fwd_window` / :func:`fa_bwd_window` - the same for local attention (key j
   visible to query i iff i - left <= j <= i + right, -1 = unlimited);
-* :func:`fwd` / :func:`bwd` - tensor conveniences that allocate outputs with torch
-  (``window=(left, right)`` selects local attention);
+* :func:`fa_decode` / :func:`fa_merge` - a few new query rows against a long key/value
+  cache, split over the cache, and the merge of partial results;
+* :func:`fwd` / :func:`bwd` / :func:`decode` / :func:`merge` - tensor conveniences that
+  allocate outputs with torch (``window=(left, right)`` selects local attention);
 * :func:`fa_bwd_workspace_bytes`, :func:`fa_device_status`, :func:`fa_status_string`.
 """
 from __future__ import annotations
@@ -70,6 +72,15 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                       ci, ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd_window.restype = ci
+        lib.fa_decode_num_splits.argtypes = [ci, ci, ci, ci, ci, ci]
+        lib.fa_decode_num_splits.restype = ci
+        lib.fa_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci, ci]
+        lib.fa_decode_workspace_bytes.restype = sz
+        lib.fa_decode.argtypes = [vp, vp, vp, vp, vp, vp, vp, sz, ci, ci, ci, ci, ci, ci, ci, ci,
+                                  cf, vp]
+        lib.fa_decode.restype = ci
+        lib.fa_merge.argtypes = [vp, vp, vp, vp, ci, ci, ci, vp]
+        lib.fa_merge.restype = ci
         lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                        ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd_noalloc.restype = ci
@@ -136,6 +147,26 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, 
     rule that calls overlapping on the GPU race on that buffer)."""
     _check(load().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d,
                                  int(causal), float(scale), stream), "fa_bwd_noalloc")
+
+
+def fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d) -> int:
+    return int(load().fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d))
+
+
+def fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits) -> int:
+    return int(load().fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits))
+
+
+def fa_decode(q, k, v, o, lse, seqlens_k, workspace, workspace_bytes, B, Hq, Hkv, Nq, Nk, d,
+              causal, num_splits, scale, stream) -> None:
+    _check(load().fa_decode(q, k, v, o, lse, seqlens_k, workspace, workspace_bytes, B, Hq, Hkv,
+                            Nq, Nk, d, int(causal), int(num_splits), float(scale), stream),
+           "fa_decode")
+
+
+def fa_merge(o_parts, lse_parts, o, lse, num_parts, rows, d, stream) -> None:
+    _check(load().fa_merge(o_parts, lse_parts, o, lse, int(num_parts), int(rows), int(d),
+                           stream), "fa_merge")
 
 
 def fa_device_status(stream=None) -> int:
@@ -242,3 +273,59 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
     else:
         fa_bwd_window(*ptrs, win[0], win[1], scale, _stream_handle(q))
     return dq, dk, dv
+
+
+def decode(q, k, v, seqlens_k=None, causal: bool = False, scale: float | None = None,
+           num_splits: int | None = None, out=None, lse=None, workspace=None):
+    """Attention of q [B, Hq, Nq, d] against a cache k, v [B, Hkv, Nk, d] (bf16, one GPU),
+    of which the first seqlens_k[b] keys are valid (int32 [B] on the GPU, or None: all).
+    Causal: the Nq queries are the last Nq positions.  Returns (O, LSE); rows that see
+    no key get O = 0 and LSE = -inf."""
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    if q.dim() != 4 or k.dim() != 4 or v.shape != k.shape:
+        raise ValueError("expected q [B,Hq,Nq,d] and k, v [B,Hkv,Nk,d]")
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if (Bk, dk) != (B, d):
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)}")
+    lens_ptr = None
+    if seqlens_k is not None:
+        if (not seqlens_k.is_cuda or seqlens_k.dtype != torch.int32 or seqlens_k.numel() != B
+                or not seqlens_k.is_contiguous()):
+            raise ValueError("seqlens_k must be a contiguous int32 CUDA tensor of B entries")
+        lens_ptr = seqlens_k.data_ptr()
+    scale = default_scale(d) if scale is None else scale
+    if num_splits is None:
+        num_splits = fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d)
+        if num_splits < 1:
+            raise FAError(FA_ERR_UNSUPPORTED, "fa_decode_num_splits")
+    nbytes = fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, num_splits)
+    if workspace is None and nbytes > 0:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    ws_ptr = None if workspace is None else workspace.data_ptr()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), lens_ptr,
+              ws_ptr, ws_bytes, B, Hq, Hkv, Nq, Nk, d, causal, num_splits, scale,
+              _stream_handle(q))
+    return o, l
+
+
+def merge(o_parts, lse_parts, out=None, lse=None):
+    """Combine partial results over disjoint key sets: o_parts [S, ..., d] fp32 (each part
+    normalised), lse_parts [S, ...] fp32 -> (O bf16 [..., d], LSE fp32 [...])."""
+    import torch
+    if (not o_parts.is_cuda or o_parts.dtype != torch.float32 or not o_parts.is_contiguous()
+            or not lse_parts.is_cuda or lse_parts.dtype != torch.float32
+            or not lse_parts.is_contiguous() or tuple(lse_parts.shape) != tuple(o_parts.shape[:-1])):
+        raise ValueError("o_parts [S, ..., d] and lse_parts [S, ...] must be contiguous fp32 CUDA tensors")
+    S, d = o_parts.shape[0], o_parts.shape[-1]
+    rows = lse_parts[0].numel()
+    o = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device) if out is None else out
+    l = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device) if lse is None else lse
+    fa_merge(o_parts.data_ptr(), lse_parts.data_ptr(), o.data_ptr(), l.data_ptr(), S, rows, d,
+             _stream_handle(o_parts))
+    return o, l

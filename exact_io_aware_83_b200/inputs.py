@@ -89,3 +89,18 @@ def draw_workload(w: Workload, with_dout: bool | None = None):
     if with_dout is None:
         with_dout = w.backward
     return draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, w.q_std, with_dout)
+
+
+def draw_decode(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, seed: int,
+                q_std: float = 1.0):
+    """Return bf16 CPU tensors (q [B, Hq, Nq, d], k_cache, v_cache [B, Hkv, Nk, d]):
+    a few new query rows against a longer key/value cache, all N(0, 1) (q scaled by
+    q_std)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((B, Hq, Nq, d), generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q = q * q_std
+    k = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
+    return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)

@@ -156,6 +156,58 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, c
                    int d, int causal, float scale, void *stream);
 
 /*
+ * Decode: attention of Nq new query rows against a key/value cache of Nk rows.
+ *
+ * Source: the "FlashAttention1" Q&A page names incremental attention updates for
+ * streaming inference (question on scaling to long sequences, item 8) and the combination
+ * of partial results from different blocks by a reduction (question on the key
+ * algorithmic innovations, item 3).  The pages give no decode algorithm; this is the
+ * library's reading: the keys are split into `num_splits` ranges processed in parallel,
+ * and the partial results (O_s normalised, LSE_s) are merged as
+ *     LSE = ln sum_s exp(LSE_s),   O = sum_s exp(LSE_s - LSE) O_s.
+ *
+ *   q    [B, Hq, Nq, d] bf16 in        k, v [B, Hkv, Nk, d] bf16 in (the cache)
+ *   o    [B, Hq, Nq, d] bf16 out       lse  [B, Hq, Nq] fp32 out (natural log)
+ *   seqlens_k: DEVICE int32 [B] (4-byte aligned), valid keys per batch (the first
+ *        seqlens_k[b] rows of the cache; values are clamped to [0, Nk]), or NULL for Nk.
+ *   causal: 0 or 1; with 1 the Nq queries are the LAST Nq positions of the sequence
+ *        (bottom-right alignment): query t sees keys j <= seqlens_k[b] - Nq + t.
+ *   num_splits: 1 .. 1024 key ranges (fa_decode_num_splits gives the library's choice).
+ *   workspace: device scratch of fa_decode_workspace_bytes() bytes, 16-byte aligned (may be
+ *        NULL when that is 0, i.e. num_splits == 1).
+ * Rows that see no key (seqlens_k[b] == 0, or causal with seqlens_k[b] < Nq) get O = 0 and
+ * LSE = -inf.  Limits: (Hq / Hkv) * Nq <= 128 (<= 64 for d = 256) query rows per K/V head
+ * (longer query blocks belong to fa_fwd), Nk <= 2^30, B * Hq * Nq < 2^31,
+ * B * Hkv * Nk < 2^31; other sizes return FA_ERR_UNSUPPORTED.
+ */
+int fa_decode(const void *q, const void *k, const void *v, void *o, float *lse,
+              const int *seqlens_k, void *workspace, size_t workspace_bytes, int B, int Hq,
+              int Hkv, int Nq, int Nk, int d, int causal, int num_splits, float scale,
+              void *stream);
+
+/*
+ * The library's split count for fa_decode: enough (b, K/V head, key range) units to fill
+ * the current device's SMs once, with at least two 128-key blocks per range.  Returns 0
+ * for sizes fa_decode rejects.
+ */
+int fa_decode_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/* Scratch bytes fa_decode needs for `num_splits` (0 when num_splits == 1 or invalid). */
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d, int num_splits);
+
+/*
+ * Merge of `num_parts` partial attention results over disjoint key sets (the reduction
+ * that fa_decode uses, exposed for callers that compute the parts themselves, e.g. over
+ * key ranges held by different devices):
+ *   o_parts   [num_parts, rows, d] fp32 in (each part normalised by its own sum)
+ *   lse_parts [num_parts, rows]    fp32 in (natural log; -inf for a part with no key)
+ *   o [rows, d] bf16 out,  lse [rows] fp32 out
+ * A row whose parts are all -inf gets O = 0 and LSE = -inf.  d in {64, 128, 256}.
+ */
+int fa_merge(const float *o_parts, const float *lse_parts, void *o, float *lse, int num_parts,
+             int rows, int d, void *stream);
+
+/*
  * Synchronises `stream`, returns the device status word of the current device
  * (FA_OK or FA_ERR_DEVICE_TIMEOUT) and clears it.  Returns FA_ERR_CUDA if the
  * synchronisation itself fails.
@@ -164,12 +216,14 @@ int fa_device_status(void *stream);
 
 /*
  * Kernel timing for benchmarks.  fa_kernel_timing(1) resets the counters and makes every
- * later fa_fwd / fa_bwd call in this process record a pair of CUDA events (created by the
+ * later fa_fwd / fa_bwd / fa_decode call (and their window forms) in this process record
+ * a pair of CUDA events (created by the
  * library, no device memory) around its main attention kernel, on the call's stream;
  * fa_kernel_timing(0) stops recording.  fa_kernel_time_ms(which, &ms, &launches)
  * synchronises those events and returns the summed device time in milliseconds and the
  * number of launches recorded since the reset: which = 0 for the forward kernel, 1 for
- * the backward main kernel (the Delta and dQ-conversion kernels are not included).  At
+ * the backward main kernel (the Delta and dQ-conversion kernels are not included), 2 for
+ * the decode kernel (the merge kernel is not included).  At
  * most 4096 launches per kind are recorded; later ones are not counted.  Returns FA_OK,
  * FA_ERR_INVALID_ARG or FA_ERR_CUDA.  Not thread-safe.
  */

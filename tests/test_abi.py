@@ -25,7 +25,8 @@ def _declared_functions():
 
 def test_header_declares_the_boundary():
     names = _declared_functions()
-    for required in ("fa_fwd", "fa_bwd", "fa_fwd_window", "fa_bwd_window",
+    for required in ("fa_fwd", "fa_bwd", "fa_fwd_window", "fa_bwd_window", "fa_decode",
+                     "fa_decode_num_splits", "fa_decode_workspace_bytes", "fa_merge",
                      "fa_bwd_workspace_bytes", "fa_device_status", "fa_status_string",
                      "fa_version"):
         assert required in names
@@ -146,6 +147,66 @@ def test_binding_rejects_causal_together_with_a_window():
         fa.fwd(q, q, q, causal=True, window=(4, 0))
 
 
+def _dec(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, lens=None, ws=FAKE, ws_bytes=1 << 30,
+             B=2, Hq=8, Hkv=2, Nq=1, Nk=1000, d=128, causal=0, splits=4, scale=0.125)
+    a.update(kw)
+    return fa.load().fa_decode(a["q"], a["k"], a["v"], a["o"], a["lse"], a["lens"], a["ws"],
+                               a["ws_bytes"], a["B"], a["Hq"], a["Hkv"], a["Nq"], a["Nk"],
+                               a["d"], a["causal"], a["splits"], a["scale"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), fa.FA_ERR_INVALID_ARG),
+    (dict(Nq=0), fa.FA_ERR_INVALID_ARG),
+    (dict(Nk=0), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=3), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=0), fa.FA_ERR_INVALID_ARG),
+    (dict(splits=1025), fa.FA_ERR_INVALID_ARG),
+    (dict(scale=-1.0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=80), fa.FA_ERR_UNSUPPORTED),
+    (dict(Hq=8, Hkv=3), fa.FA_ERR_GQA),
+    (dict(Hq=8, Hkv=1, Nq=17), fa.FA_ERR_UNSUPPORTED),          # 136 query rows per K/V head
+    (dict(Hq=8, Hkv=1, Nq=9, d=256), fa.FA_ERR_UNSUPPORTED),    # 72 > 64 for d = 256
+    (dict(ws=None), fa.FA_ERR_WORKSPACE),
+    (dict(ws_bytes=64), fa.FA_ERR_WORKSPACE),
+    (dict(o=FAKE + 8), fa.FA_ERR_ALIGN),
+    (dict(lens=FAKE + 2), fa.FA_ERR_ALIGN),
+])
+def test_decode_argument_errors(kw, code):
+    assert _dec(**kw) == code
+
+
+def test_decode_workspace_and_splits():
+    B, Hq, Hkv, Nq, Nk, d = 2, 8, 2, 3, 1000, 128
+    rows = B * Hq * Nq
+    pad = lambda x: (x + 255) // 256 * 256
+    assert fa.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, 1) == 0
+    assert fa.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, 5) == pad(5 * rows * d * 4) + pad(5 * rows * 4)
+    assert fa.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, 0) == 0
+    assert fa.fa_decode_workspace_bytes(B, Hq, 3, Nq, Nk, d, 2) == 0
+    # Without a device the split choice assumes 148 SMs: 4 units -> 37 splits, capped by
+    # the 8 key blocks (at least two per split) -> 4.
+    assert fa.fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d) == 4
+    assert fa.fa_decode_num_splits(B, Hq, Hkv, Nq, 1 << 20, d) == 37
+    assert fa.fa_decode_num_splits(64, Hq, Hkv, Nq, 1 << 20, d) == 1
+    assert fa.fa_decode_num_splits(B, Hq, 3, Nq, Nk, d) == 0
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(o=None), fa.FA_ERR_INVALID_ARG),
+    (dict(parts=0), fa.FA_ERR_INVALID_ARG),
+    (dict(rows=0), fa.FA_ERR_INVALID_ARG),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(lse=FAKE + 4), fa.FA_ERR_ALIGN),
+])
+def test_merge_argument_errors(kw, code):
+    a = dict(op=FAKE, lp=FAKE, o=FAKE, lse=FAKE, parts=3, rows=10, d=128)
+    a.update(kw)
+    assert fa.load().fa_merge(a["op"], a["lp"], a["o"], a["lse"], a["parts"], a["rows"], a["d"],
+                              None) == code
+
+
 def test_workspace_size():
     B, Hq, N, d = 2, 4, 100, 128
     rows = B * Hq * N
@@ -162,6 +223,8 @@ def test_valid_arguments_without_a_device_report_cuda_error():
     assert _bwd() == fa.FA_ERR_CUDA
     assert _fwd_w(3, 0) == fa.FA_ERR_CUDA
     assert _bwd_w(-1, 7) == fa.FA_ERR_CUDA
+    assert _dec() == fa.FA_ERR_CUDA
+    assert fa.load().fa_merge(FAKE, FAKE, FAKE, FAKE, 2, 4, 64, None) == fa.FA_ERR_CUDA
 
 
 def test_binding_rejects_cpu_tensors():
