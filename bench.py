@@ -6,7 +6,12 @@
 A step is one forward (fa_fwd) and one backward (fa_bwd) pass over one batch of the
 workload (default: GPT-style 2K causal self-attention, B=8, H=16, N=2048, d=128, bf16,
 seeded i.i.d. N(0,1) inputs).  FLOPs follow the metric's convention: 4 B H N^2 d for the
-forward, halved when causal, and 2.5x that for the backward.
+forward, halved when causal, and 2.5x that for the backward; a local-attention workload
+counts 4 d flop per visible (query, key) pair.
+
+Decode workloads (--workload decode_*) time one fa_decode call per step (new query rows
+against a resident key/value cache, split over the cache and merged); their metric is
+the cache-read bandwidth in GB/s against the measured HBM copy peak.
 
 Rank 0 prints one JSON line.  Under torchrun each rank (one GPU each) processes its own
 shard of a global batch of N x B sequences with the unchanged kernels (no collective on
@@ -49,20 +54,25 @@ def _peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def _profile_traffic():
-    """DRAM bytes per launch of the backward main kernel from the committed ncu capture,
-    or None when there is none or the kernel source has changed since it was taken."""
+def _profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture
+    (profiles/dram_traffic.json), or None when there is none or a source file of the
+    kernel has changed since it was taken."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", "bwd_main_traffic.json")
     try:
-        with open(path) as f:
-            d = json.load(f)
-        with open(os.path.join(ROOT, d["source"]), "rb") as f:
-            if hashlib.sha256(f.read()).hexdigest() != d["source_sha256"]:
-                return None
-        return d
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            entries = json.load(f)["entries"]
+        for e in entries:
+            if e["kernel"] != kernel or e["workload"] != workload:
+                continue
+            for src, digest in zip(e["sources"], e["sources_sha256"]):
+                with open(os.path.join(ROOT, src), "rb") as f:
+                    if hashlib.sha256(f.read()).hexdigest() != digest:
+                        return None
+            return int(e["dram_bytes_per_launch"])
     except (OSError, ValueError, KeyError):
         return None
+    return None
 
 
 class ClockSampler:
@@ -139,9 +149,14 @@ def _oracle_sample(w, heads: int, seed: int):
     f64 = lambda t: t.float().double().numpy()
     q, k, v, do = f64(q), f64(k), f64(v), f64(do)
     t0 = time.perf_counter()
-    oracle.attention_fwd(q, k, v, w.causal, w.scale)
-    if w.backward:
-        oracle.attention_bwd(q, k, v, do, w.causal, w.scale)
+    if w.window is not None:
+        oracle.attention_fwd_window(q, k, v, w.window[0], w.window[1], w.scale)
+        if w.backward:
+            oracle.attention_bwd_window(q, k, v, do, w.window[0], w.window[1], w.scale)
+    else:
+        oracle.attention_fwd(q, k, v, w.causal, w.scale)
+        if w.backward:
+            oracle.attention_bwd(q, k, v, do, w.causal, w.scale)
     dt = time.perf_counter() - t0
     flops = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) * (groups * g) / (w.B * w.Hq)
     return dt, flops
@@ -192,11 +207,19 @@ def run_reference(args, w):
 
 
 def _config(w, world):
-    return {"workload": w.name, "B_per_gpu": w.B, "global_batch": w.B * world, "Hq": w.Hq,
-            "Hkv": w.Hkv, "seq_len": w.N, "head_dim": w.d, "causal": w.causal,
-            "passes": "fwd+bwd" if w.backward else "fwd", "parallelism": f"dp{world}",
-            "l2": "inputs exceed L2 (q, k, v, dO = "
-                  f"{4 * w.B * w.Hq * w.N * w.d * 2 / 1e6:.0f} MB vs 126 MB); no flush"}
+    if hasattr(w, "Nk"):
+        return {"workload": w.name, "B_per_gpu": w.B, "global_batch": w.B * world, "Hq": w.Hq,
+                "Hkv": w.Hkv, "new_tokens": w.Nq, "cache_len": w.Nk, "head_dim": w.d,
+                "causal": w.causal, "passes": "decode", "parallelism": f"dp{world}",
+                "l2": f"cache exceeds L2 ({w.cache_bytes() / 1e6:.0f} MB vs 126 MB); no flush"}
+    c = {"workload": w.name, "B_per_gpu": w.B, "global_batch": w.B * world, "Hq": w.Hq,
+         "Hkv": w.Hkv, "seq_len": w.N, "head_dim": w.d, "causal": w.causal,
+         "passes": "fwd+bwd" if w.backward else "fwd", "parallelism": f"dp{world}",
+         "l2": "inputs exceed L2 (q, k, v, dO = "
+               f"{4 * w.B * w.Hq * w.N * w.d * 2 / 1e6:.0f} MB vs 126 MB); no flush"}
+    if w.window is not None:
+        c["window"] = list(w.window)
+    return c
 
 
 def run_ours(args, w):
@@ -230,10 +253,10 @@ def run_ours(args, w):
                      device="cuda")
 
     def step():
-        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, window=w.window)
         if w.backward:
             fa.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws, dq=dq,
-                   dk=dk, dv=dv)
+                   dk=dk, dv=dv, window=w.window)
 
     for _ in range(args.warmup):
         step()
@@ -317,10 +340,7 @@ def run_ours(args, w):
         dom_name, dom_ms, dom_n, dom_flops = "fa_fwd_kernel", fwd_ms, nfwd, w.fwd_flops()
     achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = None
-    prof = _profile_traffic()
-    if prof and prof.get("workload") == w.name and prof.get("kernel") == dom_name:
-        traffic = prof.get("dram_bytes_per_launch")
+    traffic = _profile_traffic(dom_name, w.name)
     kernels = {}
     if nfwd:
         kernels["fa_fwd_kernel"] = {"ms_per_launch": fwd_ms / nfwd,
@@ -364,6 +384,176 @@ def run_ours(args, w):
     return 0
 
 
+DECODE_METRIC = "decode KV-cache read bandwidth GB/s at 1 B200 and % of measured HBM copy peak"
+
+
+def _oracle_decode_sample(w, groups: int):
+    """fp64 oracle decode of the first `groups` K/V-head groups of batch row 0; returns
+    (seconds, algorithmic bytes of the sample)."""
+    import oracle
+    from exact_io_aware_83_b200.inputs import draw_decode
+    g = w.Hq // w.Hkv
+    q, k, v = draw_decode(1, groups * g, groups, w.Nq, w.Nk, w.d, w.seed)
+    f64 = lambda t: t.float().double().numpy()
+    q, k, v = f64(q), f64(k), f64(v)
+    t0 = time.perf_counter()
+    oracle.attention_decode(q, k, v, None, w.causal, w.scale)
+    dt = time.perf_counter() - t0
+    return dt, w.io_bytes() * groups / (w.B * w.Hkv)
+
+
+def run_reference_decode(args, w):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    cores = _cores()
+    oracle.set_threads(cores)
+    t1, _ = _oracle_decode_sample(w, 1)
+    budget = 120.0 / (args.steps + args.warmup)
+    groups = max(1, min(w.B * w.Hkv if w.B == 1 else w.Hkv, int(budget // max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        _oracle_decode_sample(w, groups)
+    tt, tb = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, nb = _oracle_decode_sample(w, groups)
+        tt += dt
+        tb += nb
+    value = tb / tt / 1e9
+    line = {
+        "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": f"batch row 0, K/V heads 0..{groups - 1} of {w.name}, fp64 oracle, per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours_decode(args, w):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_83_b200 import fa
+    from exact_io_aware_83_b200.inputs import draw_decode
+    from exact_io_aware_83_b200.shard import max_over_ranks, rank_seed
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    fa.load()
+    qh, kh, vh = draw_decode(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, rank_seed(w.seed, rank))
+    q, k, v = qh.cuda(), kh.cuda(), vh.cuda()
+    del kh, vh
+    S = fa.fa_decode_num_splits(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)
+    ws = torch.empty(max(16, fa.fa_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, S)),
+                     dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device="cuda")
+
+    def step():
+        fa.decode(q, k, v, causal=w.causal, scale=w.scale, num_splits=S, out=o, lse=lse,
+                  workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_device_status(None) != fa.FA_OK:
+        raise SystemExit("device status not clean after warm-up")
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    fa.fa_kernel_timing(True)
+    sampler.start()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    fa.fa_kernel_timing(False)
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    dec_ms, ndec = fa.fa_kernel_time_ms(2)
+    if fa.fa_device_status(None) != fa.FA_OK:
+        raise SystemExit("device status not clean after the timed region")
+    clocks = sampler.summary()
+    value = w.io_bytes() * args.steps * world / (ms / 1e3) / 1e9
+
+    # End to end: the new query rows come from pinned host memory and O, LSE go back; the
+    # cache stays resident on the device, as it does between decode steps.
+    qh_p = qh.pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def e2e_step():
+        q.copy_(qh_p, non_blocking=True)
+        step()
+        oh.copy_(o, non_blocking=True)
+        lseh.copy_(lse, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 10)
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+
+    peaks, peak_src = _peaks()
+    peak = float(peaks["hbm_gbs"])
+    achieved = w.io_bytes() / (dec_ms / ndec / 1e3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": dict(_config(w, world), num_splits=S),
+        "frac_of_peak": value / world / peak,
+        "roofline": {"bound": "hbm", "kernel": "fa_decode_kernel", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": _profile_traffic("fa_decode_kernel", w.name),
+                     "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"},
+        "e2e": {"value": w.io_bytes() * e2e_steps * world / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": nb(q), "d2h_bytes_per_step": nb(o, lse), "steps": e2e_steps},
+        "gpu_launches": args.steps * (2 if S > 1 else 1),
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        cores = _cores()
+        oracle.set_threads(cores)
+        dt, nbytes = _oracle_decode_sample(w, 1)
+        line["cpu_baseline"] = {
+            "value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"batch row 0, K/V head 0 of {w.name}, fp64 oracle decode, one pass, {dt:.2f} s wall"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -377,7 +567,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    from exact_io_aware_83_b200.inputs import WORKLOADS
+    from exact_io_aware_83_b200.inputs import DECODE_WORKLOADS, WORKLOADS
+    if args.workload in DECODE_WORKLOADS:
+        w = DECODE_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            return run_reference_decode(args, w)
+        return run_ours_decode(args, w)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

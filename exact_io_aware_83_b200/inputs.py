@@ -16,7 +16,20 @@ gpt_2k_causal         8   16   16   2048  128  yes     fwd+bwd    N(0,1)
 long_8k_causal        2   16   16   8192  128  yes     fwd+bwd    N(0,1)
 gqa_4k_causal_fwd     4   32   8    4096  128  yes     fwd        N(0,1)
 d256_4k_stress        2   8    8    4096  256  no      fwd+bwd    N(0,4^2)
+window_8k_1k          2   16   16   8192  128  band    fwd+bwd    N(0,1)
 ====================  ==  ===  ===  ====  ===  ======  =========  =====================
+
+window_8k_1k is local attention with the band i - 1023 <= j <= i (1024 keys per row,
+the row's own included).
+
+Decode workloads (a few new query rows against a key/value cache; K/V N(0,1)):
+
+=================  ==  ===  ===  ==  ======  ===
+name               B   Hq   Hkv  Nq  Nk      d
+=================  ==  ===  ===  ==  ======  ===
+decode_64k_gqa     4   32   8    1   65536   128
+decode_8k_batch    64  32   8    1   8192    128
+=================  ==  ===  ===  ==  ======  ===
 """
 from __future__ import annotations
 
@@ -38,6 +51,7 @@ class Workload:
     backward: bool
     q_std: float
     seed: int
+    window: tuple | None = None   # (left, right) key band, -1 = unlimited; None: causal flag
 
     @property
     def scale(self) -> float:
@@ -46,7 +60,16 @@ class Workload:
         return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
 
     def fwd_flops(self) -> float:
-        """4 B Hq N^2 d, halved when causal (the metric's convention)."""
+        """4 B Hq N^2 d, halved when causal (the metric's convention); with a key band,
+        4 B Hq d times the number of visible (query, key) pairs."""
+        if self.window is not None:
+            left, right = self.window
+            pairs = 0
+            for i in range(self.N):
+                lo = 0 if left < 0 else max(0, i - left)
+                hi = self.N - 1 if right < 0 else min(self.N - 1, i + right)
+                pairs += hi - lo + 1
+            return 4.0 * self.B * self.Hq * pairs * self.d
         f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
         return f / 2 if self.causal else f
 
@@ -63,6 +86,42 @@ WORKLOADS = {
         Workload("long_8k_causal", 2, 16, 16, 8192, 128, True, True, 1.0, 3),
         Workload("gqa_4k_causal_fwd", 4, 32, 8, 4096, 128, True, False, 1.0, 4),
         Workload("d256_4k_stress", 2, 8, 8, 4096, 256, False, True, 4.0, 5),
+        Workload("window_8k_1k", 2, 16, 16, 8192, 128, False, True, 1.0, 6, (1023, 0)),
+    )
+}
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
+
+    def cache_bytes(self) -> int:
+        """K and V of every cached row: what a decode step must read from HBM."""
+        return 2 * self.B * self.Hkv * self.Nk * self.d * 2
+
+    def io_bytes(self) -> int:
+        """Algorithmic bytes of one step: read the cache and Q, write O (bf16) and LSE."""
+        rows = self.B * self.Hq * self.Nq
+        return self.cache_bytes() + 2 * rows * self.d * 2 + rows * 4
+
+
+DECODE_WORKLOADS = {
+    w.name: w
+    for w in (
+        DecodeWorkload("decode_64k_gqa", 4, 32, 8, 1, 65536, 128, True, 7),
+        DecodeWorkload("decode_8k_batch", 64, 32, 8, 1, 8192, 128, True, 8),
     )
 }
 
