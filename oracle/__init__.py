@@ -8,8 +8,9 @@ Every function takes and returns numpy float64 arrays in the ``[B, H, N, d]`` la
 
 Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy example
 of the "Consideration"/FlashAttention article page, finite differences and invariants):
-``oracle_fwd``, ``oracle_bwd``, their key-window forms, ``oracle_decode``,
-``oracle_merge`` and ``online_softmax_stats`` all have pins; none is "parity unpinned".
+``oracle_fwd``, ``oracle_bwd``, their key-window and variable-length forms,
+``oracle_decode``, ``oracle_merge`` and ``online_softmax_stats`` all have pins; none is
+"parity unpinned".
 """
 from __future__ import annotations
 
@@ -47,6 +48,12 @@ def _lib():
         lib.oracle_decode.restype = ci
         lib.oracle_merge.argtypes = [dp, dp, ci, ctypes.c_longlong, ci, dp, dp]
         lib.oracle_merge.restype = ci
+        lib.oracle_fwd_varlen.argtypes = [dp, dp, dp, ip, ip, dp, dp, ci, ci, ci, ci, ci, ci,
+                                          ci, ci, ctypes.c_double]
+        lib.oracle_fwd_varlen.restype = ci
+        lib.oracle_bwd_varlen.argtypes = [dp, dp, dp, dp, ip, ip, dp, dp, dp, ci, ci, ci, ci,
+                                          ci, ci, ci, ci, ctypes.c_double]
+        lib.oracle_bwd_varlen.restype = ci
         lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
         lib.oracle_online_softmax_stats.restype = ci
         _LIB = lib
@@ -161,6 +168,52 @@ def attention_decode(q, k, v, lens, causal: bool, scale: float):
     if rc != 0:
         raise RuntimeError(f"oracle_decode failed with {rc}")
     return o, lse
+
+
+def _cu(cu):
+    a = np.ascontiguousarray(np.asarray(cu, dtype=np.int32).reshape(-1))
+    return a, a.ctypes.data_as(ctypes.POINTER(ctypes.c_int))
+
+
+def attention_fwd_varlen(q, k, v, cu_q, cu_k, left: int, right: int, scale: float):
+    """Packed sequences: q [total_q, Hq, d], k/v [total_k, Hkv, d], cu_* [B+1] row offsets.
+    The band i + dlt - left <= j <= i + dlt + right (dlt = Lk - Lq, -1 = unlimited) is
+    aligned to the end of each sequence.  Returns o [total_q, Hq, d], lse [total_q, Hq]."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    tq, Hq, d = q.shape
+    tk, Hkv, dk = k.shape
+    if dk != d or v.shape != k.shape:
+        raise ValueError("shape mismatch")
+    cq, cqp = _cu(cu_q)
+    ck, ckp = _cu(cu_k)
+    if cq.size != ck.size:
+        raise ValueError("cu_q and cu_k must have B+1 entries each")
+    o = np.empty_like(q)
+    lse = np.empty((tq, Hq), dtype=np.float64)
+    rc = _lib().oracle_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), cqp, ckp, _ptr(o), _ptr(lse),
+                                  cq.size - 1, Hq, Hkv, tq, tk, d, int(left), int(right),
+                                  float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_fwd_varlen failed with {rc}")
+    return o, lse
+
+
+def attention_bwd_varlen(q, k, v, dout, cu_q, cu_k, left: int, right: int, scale: float):
+    """Gradient of <O, dO> for packed sequences; returns dq, dk, dv."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    tq, Hq, d = q.shape
+    tk, Hkv, _ = k.shape
+    cq, cqp = _cu(cu_q)
+    ck, ckp = _cu(cu_k)
+    dq = np.empty_like(q)
+    dk = np.empty_like(k)
+    dv = np.empty_like(v)
+    rc = _lib().oracle_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), cqp, ckp, _ptr(dq),
+                                  _ptr(dk), _ptr(dv), cq.size - 1, Hq, Hkv, tq, tk, d,
+                                  int(left), int(right), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bwd_varlen failed with {rc}")
+    return dq, dk, dv
 
 
 def merge(o_parts, lse_parts):

@@ -372,3 +372,184 @@ int oracle_merge(const double *o_parts, const double *lse_parts, int S, long lon
     }
     return 0;
 }
+
+/*
+ * Variable-length batches: B sequences packed along the token axis.
+ *   q, o: [total_q, Hq, d];  k, v: [total_k, Hkv, d];  lse: [total_q, Hq]
+ *   sequence b owns query rows cu_q[b] .. cu_q[b+1]-1 and key rows cu_k[b] .. cu_k[b+1]-1.
+ * Lengths may differ (Lq = cu_q[b+1] - cu_q[b], Lk likewise); the key band is aligned to
+ * the END of both (bottom-right): with dlt = Lk - Lq, query i sees keys j with
+ *     i + dlt - left <= j <= i + dlt + right,  0 <= j < Lk
+ * (a negative bound is unlimited; causal is left < 0, right = 0).  Variable sequence
+ * lengths are named on the "FlashAttention1" Q&A page (question on scaling, item 2).  A
+ * query row that sees no key gets O = 0 and LSE = -inf.
+ */
+static void varlen_range(int i, int Lq, int Lk, int left, int right, int *lo, int *hi)
+{
+    const int c = i + (Lk - Lq);
+    *lo = (left < 0 || c - left < 0) ? 0 : c - left;
+    *hi = (right < 0 || c + right + 1 > Lk) ? Lk : c + right + 1;
+    if (*hi < *lo) *hi = *lo;
+}
+
+static int check_cu(const int *cu, int B, int total)
+{
+    if (!cu || cu[0] < 0) return -1;
+    for (int b = 0; b < B; ++b)
+        if (cu[b + 1] < cu[b]) return -1;
+    return cu[B] > total ? -1 : 0;
+}
+
+int oracle_fwd_varlen(const double *q, const double *k, const double *v, const int *cu_q,
+                      const int *cu_k, double *o, double *lse, int B, int Hq, int Hkv,
+                      int total_q, int total_k, int d, int left, int right, double scale)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv || !q || !k || !v || !o || !lse)
+        return -1;
+    if (check_cu(cu_q, B, total_q) || check_cu(cu_k, B, total_k)) return -1;
+    const int g = Hq / Hkv;
+    for (long long r = 0; r < (long long)total_q * Hq; ++r) lse[r] = -INFINITY;
+    for (long long r = 0; r < (long long)total_q * Hq * d; ++r) o[r] = 0.0;
+    int fail = 0;
+    for (int b = 0; b < B; ++b) {
+        const int Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
+        const long long rows = (long long)Lq * Hq;
+#pragma omp parallel reduction(|: fail)
+        {
+            double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+            if (!s) {
+                fail = 1;
+            } else {
+#pragma omp for schedule(dynamic, 8)
+                for (long long r = 0; r < rows; ++r) {
+                    const int i = (int)(r / Hq), h = (int)(r % Hq);
+                    int lo, hi;
+                    varlen_range(i, Lq, Lk, left, right, &lo, &hi);
+                    if (hi <= lo) continue;               /* no key: O = 0, LSE = -inf */
+                    const size_t qrow = (size_t)(cu_q[b] + i) * Hq + h;
+                    /* key row j of this head: k + ((cu_k[b] + j) * Hkv + h / g) * d */
+                    double m = -INFINITY;
+                    for (int j = lo; j < hi; ++j) {
+                        const double *kj = k + ((size_t)(cu_k[b] + j) * Hkv + h / g) * d;
+                        s[j - lo] = scale * dotd(q + qrow * d, kj, d);
+                        if (s[j - lo] > m) m = s[j - lo];
+                    }
+                    double l = 0.0;
+                    for (int j = lo; j < hi; ++j) l += exp(s[j - lo] - m);
+                    const double L = m + log(l);
+                    double *oi = o + qrow * d;
+                    for (int j = lo; j < hi; ++j) {
+                        const double p = exp(s[j - lo] - L);
+                        const double *vj = v + ((size_t)(cu_k[b] + j) * Hkv + h / g) * d;
+                        for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
+                    }
+                    lse[qrow] = L;
+                }
+                free(s);
+            }
+        }
+    }
+    return fail ? -2 : 0;
+}
+
+/*
+ * Gradient of <O, dO> for variable-length batches (layouts as oracle_fwd_varlen; dq like q,
+ * dk and dv like k).  Pass 1 runs over query rows (LSE, Delta, dQ); pass 2 over key rows,
+ * visiting every query row whose band contains the key.
+ */
+int oracle_bwd_varlen(const double *q, const double *k, const double *v, const double *dout,
+                      const int *cu_q, const int *cu_k, double *dq, double *dk, double *dv,
+                      int B, int Hq, int Hkv, int total_q, int total_k, int d, int left,
+                      int right, double scale)
+{
+    if (B < 1 || Hq < 1 || Hkv < 1 || d < 1 || Hq % Hkv || !q || !k || !v || !dout || !dq ||
+        !dk || !dv)
+        return -1;
+    if (check_cu(cu_q, B, total_q) || check_cu(cu_k, B, total_k)) return -1;
+    const int g = Hq / Hkv;
+    const long long nq = (long long)total_q * Hq;
+    double *L = (double *)malloc(sizeof(double) * (size_t)(nq > 0 ? nq : 1));
+    double *D = (double *)malloc(sizeof(double) * (size_t)(nq > 0 ? nq : 1));
+    if (!L || !D) { free(L); free(D); return -2; }
+    for (long long r = 0; r < nq * d; ++r) dq[r] = 0.0;
+    for (long long r = 0; r < (long long)total_k * Hkv * d; ++r) { dk[r] = 0.0; dv[r] = 0.0; }
+    for (long long r = 0; r < nq; ++r) { L[r] = -INFINITY; D[r] = 0.0; }
+    int fail = 0;
+    for (int b = 0; b < B && !fail; ++b) {
+        const int Lq = cu_q[b + 1] - cu_q[b], Lk = cu_k[b + 1] - cu_k[b];
+        const long long rows = (long long)Lq * Hq;
+        /* Pass 1: per query row. */
+#pragma omp parallel reduction(|: fail)
+        {
+            double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+            double *dp = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+            if (!s || !dp) {
+                fail = 1;
+            } else {
+#pragma omp for schedule(dynamic, 8)
+                for (long long r = 0; r < rows; ++r) {
+                    const int i = (int)(r / Hq), h = (int)(r % Hq);
+                    int lo, hi;
+                    varlen_range(i, Lq, Lk, left, right, &lo, &hi);
+                    if (hi <= lo) continue;
+                    const size_t qrow = (size_t)(cu_q[b] + i) * Hq + h;
+                    double m = -INFINITY;
+                    for (int j = lo; j < hi; ++j) {
+                        const double *kj = k + ((size_t)(cu_k[b] + j) * Hkv + h / g) * d;
+                        s[j - lo] = scale * dotd(q + qrow * d, kj, d);
+                        if (s[j - lo] > m) m = s[j - lo];
+                    }
+                    double l = 0.0;
+                    for (int j = lo; j < hi; ++j) l += exp(s[j - lo] - m);
+                    const double Li = m + log(l);
+                    double Di = 0.0;
+                    for (int j = lo; j < hi; ++j) {
+                        const double *vj = v + ((size_t)(cu_k[b] + j) * Hkv + h / g) * d;
+                        dp[j - lo] = dotd(dout + qrow * d, vj, d);
+                        Di += exp(s[j - lo] - Li) * dp[j - lo];
+                    }
+                    double *dqi = dq + qrow * d;
+                    for (int j = lo; j < hi; ++j) {
+                        const double dS = exp(s[j - lo] - Li) * (dp[j - lo] - Di);
+                        const double *kj = k + ((size_t)(cu_k[b] + j) * Hkv + h / g) * d;
+                        for (int c = 0; c < d; ++c) dqi[c] += dS * kj[c];
+                    }
+                    for (int c = 0; c < d; ++c) dqi[c] *= scale;
+                    L[qrow] = Li;
+                    D[qrow] = Di;
+                }
+            }
+            free(s);
+            free(dp);
+        }
+        if (fail) break;
+        /* Pass 2: per key row of each K/V head. */
+        const long long krows = (long long)Lk * Hkv;
+#pragma omp parallel for schedule(dynamic, 8)
+        for (long long r = 0; r < krows; ++r) {
+            const int j = (int)(r / Hkv), kvh = (int)(r % Hkv);
+            const size_t krow = (size_t)(cu_k[b] + j) * Hkv + kvh;
+            const double *kj = k + krow * d, *vj = v + krow * d;
+            double *dkj = dk + krow * d, *dvj = dv + krow * d;
+            for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
+                for (int i = 0; i < Lq; ++i) {
+                    int lo, hi;
+                    varlen_range(i, Lq, Lk, left, right, &lo, &hi);
+                    if (j < lo || j >= hi) continue;
+                    const size_t qrow = (size_t)(cu_q[b] + i) * Hq + h;
+                    const double *qi = q + qrow * d, *doi = dout + qrow * d;
+                    const double P = exp(scale * dotd(qi, kj, d) - L[qrow]);
+                    const double dS = P * (dotd(doi, vj, d) - D[qrow]);
+                    for (int c = 0; c < d; ++c) {
+                        dvj[c] += P * doi[c];
+                        dkj[c] += dS * qi[c];
+                    }
+                }
+            }
+            for (int c = 0; c < d; ++c) dkj[c] *= scale;
+        }
+    }
+    free(L);
+    free(D);
+    return fail ? -2 : 0;
+}

@@ -19,7 +19,10 @@ the causal mask on the wrong side, a missing scale) fails at least one test:
 * decode (queries at the end of a longer cache) against a bottom-right-masked softmax on
   the full score matrix, the square forward, and single-key / no-key closed forms;
 * the merge of partial results against attention over the union of the key ranges, and
-  closed forms (one part, equal weights, weights 1/4 and 3/4, all parts empty).
+  closed forms (one part, equal weights, weights 1/4 and 3/4, all parts empty);
+* packed variable-length batches against the dense oracle per sequence (equal lengths),
+  the decode oracle per sequence (unequal lengths, bottom-right band), a brute-force
+  masked softmax for banded windows, and central finite differences.
 """
 import math
 import os
@@ -531,3 +534,135 @@ def test_merge_closed_forms():
     ob, lb = oracle.merge(np.concatenate([o2, o1]), np.concatenate([l3, l1]))
     np.testing.assert_allclose(oa, ob, atol=1e-15)
     np.testing.assert_allclose(la, lb, atol=1e-15)
+
+
+# ---------------------------------------------------------------------------- variable length
+
+def _pack(rng, lens, H, d):
+    """[total, H, d] packed rows and the [B+1] offsets."""
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    return rng.normal(size=(int(cu[-1]), H, d)), cu
+
+
+def _seq(x, cu, b):
+    """Rows of sequence b as a dense [1, H, L, d] array."""
+    return np.ascontiguousarray(x[cu[b]:cu[b + 1]].transpose(1, 0, 2)[None])
+
+
+@pytest.mark.parametrize("left,right", [(-1, -1), (-1, 0), (3, 1), (0, 0)])
+def test_varlen_with_equal_lengths_is_the_dense_oracle_per_sequence(left, right):
+    r = _rng(61)
+    lens = [5, 1, 9]
+    q, cu = _pack(r, lens, 4, 6)
+    k, _ = _pack(r, lens, 2, 6)
+    v, _ = _pack(r, lens, 2, 6)
+    do, _ = _pack(r, lens, 4, 6)
+    o, lse = oracle.attention_fwd_varlen(q, k, v, cu, cu, left, right, 0.45)
+    dq, dk, dv = oracle.attention_bwd_varlen(q, k, v, do, cu, cu, left, right, 0.45)
+    for b in range(len(lens)):
+        o_b, l_b = oracle.attention_fwd_window(_seq(q, cu, b), _seq(k, cu, b), _seq(v, cu, b),
+                                               left, right, 0.45)
+        np.testing.assert_allclose(_seq(o, cu, b), o_b, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[cu[b]:cu[b + 1]].T[None], l_b, rtol=0, atol=1e-13)
+        g = oracle.attention_bwd_window(_seq(q, cu, b), _seq(k, cu, b), _seq(v, cu, b),
+                                        _seq(do, cu, b), left, right, 0.45)
+        for x, ref in ((dq, g[0]), (dk, g[1]), (dv, g[2])):
+            np.testing.assert_allclose(_seq(x, cu, b), ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_with_unequal_lengths_is_decode_per_sequence(causal):
+    # Lq != Lk: the band is aligned to the end of the sequence, which is exactly the
+    # decode oracle's bottom-right convention (Lq > Lk leaves early causal rows empty).
+    r = _rng(67)
+    lq, lk = [3, 7, 2, 4], [8, 7, 0, 2]
+    q, cq = _pack(r, lq, 4, 5)
+    k, ck = _pack(r, lk, 2, 5)
+    v, _ = _pack(r, lk, 2, 5)
+    o, lse = oracle.attention_fwd_varlen(q, k, v, cq, ck, -1, 0 if causal else -1, 0.6)
+    for b in range(4):
+        if lk[b] == 0:
+            assert np.all(_seq(o, cq, b) == 0) and np.all(np.isneginf(lse[cq[b]:cq[b + 1]]))
+            continue
+        o_b, l_b = oracle.attention_decode(_seq(q, cq, b), _seq(k, ck, b), _seq(v, ck, b), None,
+                                           causal, 0.6)
+        np.testing.assert_allclose(_seq(o, cq, b), o_b, rtol=0, atol=1e-13)
+        got = lse[cq[b]:cq[b + 1]].T[None]
+        np.testing.assert_array_equal(np.isneginf(got), np.isneginf(l_b))
+        fin = np.isfinite(l_b)
+        np.testing.assert_allclose(got[fin], l_b[fin], rtol=0, atol=1e-13)
+
+
+def _brute_varlen(q, k, v, cq, ck, left, right, scale):
+    o = np.zeros_like(q)
+    lse = np.full(q.shape[:2], -np.inf)
+    Hq, Hkv = q.shape[1], k.shape[1]
+    for b in range(len(cq) - 1):
+        Lq, Lk = cq[b + 1] - cq[b], ck[b + 1] - ck[b]
+        i = np.arange(Lq)[:, None] + (Lk - Lq)
+        j = np.arange(Lk)[None, :]
+        vis = np.ones((Lq, Lk), dtype=bool)
+        if left >= 0:
+            vis &= j >= i - left
+        if right >= 0:
+            vis &= j <= i + right
+        for h in range(Hq):
+            s = scale * q[cq[b]:cq[b + 1], h] @ k[ck[b]:ck[b + 1], h // (Hq // Hkv)].T
+            s = np.where(vis, s, -np.inf)
+            for t in range(Lq):
+                if vis[t].any():
+                    lse[cq[b] + t, h] = scipy.special.logsumexp(s[t])
+                    o[cq[b] + t, h] = np.exp(s[t] - lse[cq[b] + t, h]) @ v[ck[b]:ck[b + 1], h // (Hq // Hkv)]
+    return o, lse
+
+
+@pytest.mark.parametrize("left,right", [(2, 0), (1, 3), (-1, 2), (4, -1), (0, 0)])
+def test_varlen_window_equals_masked_softmax(left, right):
+    r = _rng(71)
+    lq, lk = [6, 2, 9], [4, 5, 9]
+    q, cq = _pack(r, lq, 2, 4)
+    k, ck = _pack(r, lk, 1, 4)
+    v, _ = _pack(r, lk, 1, 4)
+    o, lse = oracle.attention_fwd_varlen(q, k, v, cq, ck, left, right, 0.7)
+    o_ref, lse_ref = _brute_varlen(q, k, v, cq, ck, left, right, 0.7)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(lse_ref))
+    fin = np.isfinite(lse_ref)
+    np.testing.assert_allclose(lse[fin], lse_ref[fin], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=1e-12)
+
+
+def test_varlen_gradients_match_central_differences():
+    r = _rng(73)
+    lq, lk = [3, 4], [5, 2]
+    q, cq = _pack(r, lq, 2, 3)
+    k, ck = _pack(r, lk, 1, 3)
+    v, _ = _pack(r, lk, 1, 3)
+    do = r.normal(size=q.shape)
+    left, right, scale = 2, 1, 0.8
+
+    def loss(q_, k_, v_):
+        o_, _ = oracle.attention_fwd_varlen(q_, k_, v_, cq, ck, left, right, scale)
+        return float((o_ * do).sum())
+
+    dq, dk, dv = oracle.attention_bwd_varlen(q, k, v, do, cq, ck, left, right, scale)
+    eps = 1e-6
+    for x, g, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            args_p = [q.copy(), k.copy(), v.copy()]
+            args_m = [q.copy(), k.copy(), v.copy()]
+            args_p[which][idx] += eps
+            args_m[which][idx] -= eps
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7)
+
+
+def test_varlen_invalid_offsets_are_rejected():
+    r = _rng(79)
+    q, cq = _pack(r, [2, 3], 1, 4)
+    with pytest.raises(RuntimeError):
+        oracle.attention_fwd_varlen(q, q, q, [0, 3, 2], cq, -1, -1, 1.0)   # decreasing
+    with pytest.raises(RuntimeError):
+        oracle.attention_fwd_varlen(q, q, q, cq, [0, 2, 9], -1, -1, 1.0)   # past the end
