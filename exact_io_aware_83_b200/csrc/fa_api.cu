@@ -154,6 +154,22 @@ bool make_map_bf16(CUtensorMap *m, const void *ptr, int d, int N, long long head
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D bf16 tensor map over packed rows [total][H][d] (a tile = box_rows consecutive
+// rows of one head: box {64, 1, box_rows}), 128-byte swizzle.  The shared-memory image of
+// a box is the same [box_rows x 64] tile as that of make_map_bf16.
+bool make_map_packed(CUtensorMap *m, const void *ptr, int d, int H, int total, int box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total > 0 ? total : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[3] = {64u, 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides,
+                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- optional event pairs around the main kernels (fa_kernel_timing)
@@ -285,6 +301,64 @@ void launch_merge(const float *o_part, const float *lse_part, void *o, float *ls
   else fa::fa_merge_kernel<256><<<grid, 256, 0, s>>>(o_part, lse_part, ob, lse, S, rows);
 }
 
+// Launches the forward kernel for d (maps and parameters prepared by the caller).
+int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
+               FwdParams &p, int d, bool window, cudaStream_t s) {
+  const int g = p.Hq / p.Hkv;
+  const int tslot = timer_start(0, s);
+  if (d == 256) {
+    p.pair_heads = 0;
+    const unsigned units = static_cast<unsigned>(p.B) * p.Hq * p.nqb;
+    if (window)
+      fa::fa_fwd_d256_kernel<true><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
+          tq, tk, tv, to, p);
+    else
+      fa::fa_fwd_d256_kernel<false><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
+          tq, tk, tv, to, p);
+  } else {
+    p.pair_heads = (g % 2 == 0) ? 1 : 0;
+    const unsigned units = p.pair_heads ? static_cast<unsigned>(p.B) * (p.Hq / 2) * p.nqb
+                                        : static_cast<unsigned>(p.B) * p.Hq * ((p.nqb + 1) / 2);
+    if (d == 64) {
+      if (window)
+        fa::fa_fwd_kernel<64, true><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+      else
+        fa::fa_fwd_kernel<64, false><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+    } else {
+      if (window)
+        fa::fa_fwd_kernel<128, true><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+      else
+        fa::fa_fwd_kernel<128, false><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+    }
+  }
+  const bool launched = cuda_ok(cudaGetLastError(), "fa_fwd launch");
+  timer_stop(0, tslot, s);
+  return launched ? FA_OK : FA_ERR_CUDA;
+}
+
+// Packed-sequence sizes: totals up to 2^29 rows keep every band computation in int32.
+int check_varlen_sizes(int B, int Hq, int Hkv, int total_q, int total_k, int max_q, int max_k, int d,
+                       float scale) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || total_q < 0 || total_k < 0 || max_q < 0 || max_k < 0)
+    return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return FA_ERR_GQA;
+  if (total_q > (1 << 29) || total_k > (1 << 29) || max_q > (1 << 29) || max_k > (1 << 29) ||
+      static_cast<long long>(total_q) * Hq >= (1ll << 31) ||
+      static_cast<long long>(B) * Hq * ((max_q + 127) / 128) >= (1ll << 31) ||
+      static_cast<long long>(B) * Hkv * ((max_k + 127) / 128) * 2 >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// Window bound for packed sequences: a bound of max_q + max_k or more hides nothing.
+bool normalise_window_varlen(int w, int max_q, int max_k, int *out) {
+  if (w < -1) return false;
+  *out = (w < 0 || static_cast<long long>(w) >= static_cast<long long>(max_q) + max_k) ? -1 : w;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -302,6 +376,7 @@ const char *fa_status_string(int code) {
     case FA_ERR_CUDA: return "CUDA error (no sm_100 device or launch failure)";
     case FA_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
     case FA_ERR_SCRATCH_LIMIT: return "problem needs more scratch than the static no-alloc buffer holds";
+    case FA_ERR_SEQLENS: return "packed-sequence offsets inconsistent with the sizes given";
     default: return "unknown status";
   }
 }
@@ -338,51 +413,60 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *l
 
   FwdParams p;
   p.lse = lse;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.N = N;
+  p.total_q = p.total_k = 0;
   p.nqb = (N + 127) / 128;
   p.left = left;
   p.right = right;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int g = Hq / Hkv;
+  return launch_fwd(tq, tk, tv, to, p, d, window, static_cast<cudaStream_t>(stream));
+}
 
-  const int tslot = timer_start(0, s);
-  if (d == 256) {
-    p.pair_heads = 0;
-    const unsigned units = static_cast<unsigned>(B) * Hq * p.nqb;
-    if (window)
-      fa::fa_fwd_d256_kernel<true><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
-          tq, tk, tv, to, p);
-    else
-      fa::fa_fwd_d256_kernel<false><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
-          tq, tk, tv, to, p);
-  } else {
-    p.pair_heads = (g % 2 == 0) ? 1 : 0;
-    const unsigned units = p.pair_heads
-                               ? static_cast<unsigned>(B) * (Hq / 2) * p.nqb
-                               : static_cast<unsigned>(B) * Hq * ((p.nqb + 1) / 2);
-    if (d == 64) {
-      if (window)
-        fa::fa_fwd_kernel<64, true><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(
-            tq, tk, tv, to, p);
-      else
-        fa::fa_fwd_kernel<64, false><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(
-            tq, tk, tv, to, p);
-    } else {
-      if (window)
-        fa::fa_fwd_kernel<128, true><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(
-            tq, tk, tv, to, p);
-      else
-        fa::fa_fwd_kernel<128, false><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(
-            tq, tk, tv, to, p);
-    }
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int *cu_seqlens_q,
+                  const int *cu_seqlens_k, int B, int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q,
+                  int max_seqlen_k, int d, int window_left, int window_right, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return FA_ERR_INVALID_ARG;
+  int rc = check_varlen_sizes(B, Hq, Hkv, total_q, total_k, max_seqlen_q, max_seqlen_k, d, scale);
+  if (rc != FA_OK) return rc;
+  int left = -1, right = -1;
+  if (!normalise_window_varlen(window_left, max_seqlen_q, max_seqlen_k, &left) ||
+      !normalise_window_varlen(window_right, max_seqlen_q, max_seqlen_k, &right))
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  if (total_q == 0 || max_seqlen_q == 0) return FA_OK;  // no query rows
+
+  const int kv_rows = d == 256 ? 64 : 128;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map_packed(&tq, q, d, Hq, total_q, 128) || !make_map_packed(&tk, k, d, Hkv, total_k, kv_rows) ||
+      !make_map_packed(&tv, v, d, Hkv, total_k, kv_rows) || !make_map_packed(&to, o, d, Hq, total_q, 128)) {
+    if (debug_enabled()) std::fprintf(stderr, "[fa] cuTensorMapEncodeTiled failed (fa_fwd_varlen)\n");
+    return FA_ERR_CUDA;
   }
-  const bool launched = cuda_ok(cudaGetLastError(), "fa_fwd launch");
-  timer_stop(0, tslot, s);
-  return launched ? FA_OK : FA_ERR_CUDA;
+  FwdParams p;
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = 0;
+  p.total_q = total_q;
+  p.total_k = total_k;
+  p.nqb = (max_seqlen_q + 127) / 128;
+  p.left = left;
+  p.right = right;
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  return launch_fwd(tq, tk, tv, to, p, d, left >= 0 || right >= 0, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
@@ -416,6 +500,51 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, co
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, left, right,
                         scale, static_cast<cudaStream_t>(stream), encode_fn(), &timer_start,
                         &timer_stop);
+}
+
+size_t fa_bwd_varlen_workspace_bytes(int Hq, int total_q, int d) {
+  if (Hq < 1 || total_q < 0 || total_q > (1 << 29) || (d != 64 && d != 128 && d != 256) ||
+      static_cast<long long>(total_q) * Hq >= (1ll << 31))
+    return 0;
+  return fa::bwd_workspace_bytes(1, Hq, total_q, d);
+}
+
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+                  void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, const int *cu_seqlens_q,
+                  const int *cu_seqlens_k, int B, int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q,
+                  int max_seqlen_k, int d, int window_left, int window_right, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !cu_seqlens_q || !cu_seqlens_k)
+    return FA_ERR_INVALID_ARG;
+  int rc = check_varlen_sizes(B, Hq, Hkv, total_q, total_k, max_seqlen_q, max_seqlen_k, d, scale);
+  if (rc != FA_OK) return rc;
+  int left = -1, right = -1;
+  if (!normalise_window_varlen(window_left, max_seqlen_q, max_seqlen_k, &left) ||
+      !normalise_window_varlen(window_right, max_seqlen_q, max_seqlen_k, &right))
+    return FA_ERR_INVALID_ARG;
+  const size_t need = fa::bwd_workspace_bytes(1, Hq, total_q, d);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (total_k > 0 && (total_q == 0 || max_seqlen_q == 0 || max_seqlen_k == 0)) {
+    // No query row sees a key: dK = dV = 0 (and there is no dQ row to write).
+    if (!cuda_ok(cudaMemsetAsync(dk, 0, static_cast<size_t>(total_k) * Hkv * d * 2, s), "cudaMemsetAsync(dK)") ||
+        !cuda_ok(cudaMemsetAsync(dv, 0, static_cast<size_t>(total_k) * Hkv * d * 2, s), "cudaMemsetAsync(dV)"))
+      return FA_ERR_CUDA;
+  }
+  if (total_q == 0 || max_seqlen_q == 0 || max_seqlen_k == 0) {
+    if (total_q > 0 &&
+        !cuda_ok(cudaMemsetAsync(dq, 0, static_cast<size_t>(total_q) * Hq * d * 2, s), "cudaMemsetAsync(dQ)"))
+      return FA_ERR_CUDA;
+    return FA_OK;
+  }
+  const fa::PackedSeqs pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k};
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, 0, d, left, right, scale, s,
+                        encode_fn(), &timer_start, &timer_stop, &pk);
 }
 
 int fa_kernel_timing(int enable) {

@@ -95,12 +95,15 @@ __global__ void __launch_bounds__(256)
 // ============================================================================ main kernel
 
 struct BwdParams {
-  const float *lse;    // [B, Hq, N]
-  const float *delta;  // [B, Hq, N]
+  const float *lse;       // dense: [B, Hq, N]; packed sequences: [total_q, Hq]
+  const float *delta;     // same layout as lse
+  __nv_bfloat16 *dk, *dv; // packed sequences: for the rows of key blocks that end past a sequence
+  const int *cu_q, *cu_k; // packed sequences: [B + 1] row offsets (nullptr: dense [B, H, N, d])
   int B, Hq, Hkv, N;
-  int nkb;             // key blocks of 128
-  int left, right;     // key window: key j seen by query i iff i - left <= j <= i + right; -1 = unlimited
-  float sl2;           // scale * log2(e)
+  int total_q, total_k;
+  int nkb;                // key blocks of 128 per sequence (packed: of the longest)
+  int left, right;        // key band around the diagonal (see SeqGeom); -1 = unlimited
+  float sl2;              // scale * log2(e)
   float scale;
 };
 
@@ -205,14 +208,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int b = u / p.Hkv;
   const int g = p.Hq / p.Hkv;
   const int kv0 = kb * 128;
-  // Query blocks that can see some key of this block: queries i with
-  // j - right <= i <= j + left for a key j in [kv0, kv0 + 127].
-  const int kv1 = min(kv0 + 127, p.N - 1);
-  const int q_first = (p.right < 0 || kv0 <= p.right) ? 0 : (kv0 - p.right) / BQ;
-  const int q_last = (p.left < 0 || p.left >= p.N - 1 - kv1) ? (p.N - 1) / BQ : (kv1 + p.left) / BQ;
-  const int nq = q_last - q_first + 1;
+  const bool packed = p.cu_q != nullptr;
+  SeqGeom sg;
+  if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, INT_MAX, p.nkb * 128, b, sg)) return;
+  if (kv0 >= sg.Lk) return;  // packed: the block starts past the sequence's keys
+  // Query blocks that can see some key of this block: query i sits at key position
+  // i + dlt and sees key j iff j - right <= i + dlt <= j + left.
+  const int kv1 = min(kv0 + 127, sg.Lk - 1);
+  const int first_i = p.right < 0 ? 0 : max(0, kv0 - p.right - sg.dlt);
+  const int last_i = p.left < 0 ? sg.Lq - 1 : min(sg.Lq - 1, kv1 + p.left - sg.dlt);
+  const int q_first = first_i / BQ;
+  const int nq = last_i >= first_i ? last_i / BQ - q_first + 1 : 0;  // 0: dK = dV = 0
   const int T = g * nq;  // steps: (query head of the group, query block)
   const int dcol0 = half * DH;  // first output column owned by this CTA
+  // TMA coordinates (dimensions 1 and 2): dense maps are [B*H][N][cols], packed [total][H][cols].
+  auto q_coords = [&](int hh, int row, int &c1, int &c2) {
+    c1 = packed ? hh : row;
+    c2 = packed ? sg.q_base + row : b * p.Hq + hh;
+  };
+  const int kv_c1 = packed ? kvh : kv0, kv_c2 = packed ? sg.k_base + kv0 : b * p.Hkv + kvh;
+  // Row of query q of head hh in the LSE / Delta vectors.
+  auto vec_row = [&](int hh, int q) -> size_t {
+    return packed ? static_cast<size_t>(sg.q_base + q) * p.Hq + hh : static_cast<size_t>(b * p.Hq + hh) * p.N + q;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i) {
@@ -249,8 +267,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_arrive_expect_tx(bar(L::kBarKV), 2 * L::kKTile);
 #pragma unroll
       for (int c = 0; c < L::kChunks; ++c) {
-        tma_load_3d(sK + c * L::kKChunk, &tm_k, bar(L::kBarKV), c * 64, kv0, b * p.Hkv + kvh);
-        tma_load_3d(sV + c * L::kKChunk, &tm_v, bar(L::kBarKV), c * 64, kv0, b * p.Hkv + kvh);
+        tma_load_3d(sK + c * L::kKChunk, &tm_k, bar(L::kBarKV), c * 64, kv_c1, kv_c2);
+        tma_load_3d(sV + c * L::kKChunk, &tm_v, bar(L::kBarKV), c * 64, kv_c1, kv_c2);
       }
     }
     int issued = 0;
@@ -261,23 +279,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!ok) break;
       const int h = step_head(i), q0 = step_q0(i);
       if (lane == 0) {
+        int c1, c2;
+        q_coords(h, q0, c1, c2);
         mbar_arrive_expect_tx(bar(L::kBarQFull + st), 2 * L::kQTile);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c) {
-          tma_load_3d(sQ + st * L::kQTile + c * L::kQChunk, &tm_q, bar(L::kBarQFull + st), c * 64, q0,
-                      b * p.Hq + h);
-          tma_load_3d(sDO + st * L::kQTile + c * L::kQChunk, &tm_do, bar(L::kBarQFull + st), c * 64, q0,
-                      b * p.Hq + h);
+          tma_load_3d(sQ + st * L::kQTile + c * L::kQChunk, &tm_q, bar(L::kBarQFull + st), c * 64, c1, c2);
+          tma_load_3d(sDO + st * L::kQTile + c * L::kQChunk, &tm_do, bar(L::kBarQFull + st), c * 64, c1, c2);
         }
       }
-      const size_t rowbase = static_cast<size_t>(b * p.Hq + h) * p.N;
       float *lse2 = vec + (st * 2) * BQ;
       float *dl = vec + (st * 2 + 1) * BQ;
       for (int c = lane; c < BQ; c += 32) {
         const int q = q0 + c;
-        // Query rows past N get LSE = +inf, so their probabilities are exactly 0.
-        lse2[c] = q < p.N ? p.lse[rowbase + q] * 1.4426950408889634f : INFINITY;
-        dl[c] = q < p.N ? p.delta[rowbase + q] : 0.f;
+        // Query rows past the sequence get LSE = +inf, so their probabilities are exactly 0
+        // (and so are their dS and their dQ contributions).  A row that sees no key has
+        // LSE = -inf but is never inside this block's band.
+        const bool live = q < sg.Lq;
+        lse2[c] = live ? p.lse[vec_row(h, q)] * 1.4426950408889634f : INFINITY;
+        dl[c] = live ? p.delta[vec_row(h, q)] : 0.f;
       }
       // The stores above are ordered before lane 0's arrival by the warp barrier; the
       // barrier phase completes only when that arrival and the TMA bytes are both in.
@@ -307,8 +327,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       bool ok = wait_bounded(bar(L::kBarKV), 0, abort_flag, wait_site(3, L::kBarKV, 0));
-      if (ok) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
-      if (ok) {
+      if (ok && T > 0) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
+      if (ok && T > 0) {
         tc_fence_after_sync();
         issue_st(L::kTmS, sK, sQ);
         tc_commit(bar(L::kBarS));
@@ -377,7 +397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tS = tmem + L::kTmS + lane_off + c0;
     const uint32_t tDP = tmem + L::kTmDP + lane_off + c0;
-    const bool row_live = kv < p.N;
+    const bool row_live = kv < sg.Lk;
     const float sl2 = p.sl2;
     bool ok = true;
     for (int i = 0; ok && i < T; ++i) {
@@ -409,8 +429,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < HC; ++c) pr[c] = 0.f;
       } else if (WINDOW) {
-        const int c_lo = p.right < 0 ? INT_MIN : kv - p.right - q0;
-        const int c_hi = p.left < 0 ? INT_MAX : kv + p.left - q0;
+        const int c_lo = p.right < 0 ? INT_MIN : kv - p.right - sg.dlt - q0;
+        const int c_hi = p.left < 0 ? INT_MAX : kv + p.left - sg.dlt - q0;
         if (c_lo > 0 || c_hi < HC - 1) {
 #pragma unroll
           for (int c = 0; c < HC; ++c)
@@ -468,10 +488,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t tacc = tmem + (wg ? L::kTmDK : L::kTmDV) + lane_off;
       const float mul = wg ? p.scale : 1.f;
       const uint32_t stage = wg ? sK : sV;
+      // A packed key block that ends past its sequence stores its rows directly.
+      const bool direct = packed && kv0 + 128 > sg.Lk;
+      __nv_bfloat16 *drow = packed ? (wg ? p.dk : p.dv) + (static_cast<size_t>(sg.k_base + kv) * p.Hkv + kvh) * D + dcol0
+                                   : nullptr;
 #pragma unroll
       for (int cc = 0; cc < DH / 32; ++cc) {
         uint32_t o[32];
-        tmem_ld_x32(tacc + cc * 32, o);
+        if (T > 0) {
+          tmem_ld_x32(tacc + cc * 32, o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;  // no query sees this block
+        }
         const uint32_t rowbase = stage + (cc / 2) * L::kKChunk + r * 128;
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
@@ -481,19 +510,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int e = 0; e < 4; ++e)
             w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * mul,
                                __uint_as_float(o[8 * uu + 2 * e + 1]) * mul);
-          st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+          if (!direct)
+            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+          else if (row_live)
+            *reinterpret_cast<uint4 *>(drow + cc * 32 + uu * 8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 256);
-      if (threadIdx.x == 0) {
+      if (!direct) {
+        fence_proxy_async_smem();
+        named_bar_sync(1, 256);
+        if (threadIdx.x == 0) {
 #pragma unroll
-        for (int c = 0; c < DH / 64; ++c) {
-          tma_store_3d(&tm_dv, sV + c * L::kKChunk, dcol0 + c * 64, kv0, b * p.Hkv + kvh);
-          tma_store_3d(&tm_dk, sK + c * L::kKChunk, dcol0 + c * 64, kv0, b * p.Hkv + kvh);
+          for (int c = 0; c < DH / 64; ++c) {
+            tma_store_3d(&tm_dv, sV + c * L::kKChunk, dcol0 + c * 64, kv_c1, kv_c2);
+            tma_store_3d(&tm_dk, sK + c * L::kKChunk, dcol0 + c * 64, kv_c1, kv_c2);
+          }
+          bulk_commit_group();
+          bulk_wait_group_read0();
         }
-        bulk_commit_group();
-        bulk_wait_group_read0();
       }
     }
   } else {
@@ -537,7 +571,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_proxy_async_smem();
         named_bar_sync(2, 128);
         if (tid == 0) {
-          tma_reduce_add_3d(&tm_dqacc, sDQ, dcol0 + hp * L::kDQCols, q0, b * p.Hq + h);
+          int c1, c2;
+          q_coords(h, q0, c1, c2);
+          tma_reduce_add_3d(&tm_dqacc, sDQ, dcol0 + hp * L::kDQCols, c1, c2);
           bulk_commit_group();
         }
       }
@@ -582,6 +618,28 @@ inline bool bwd_map(EncodeTiledFnBwd enc, CUtensorMap *m, const void *ptr, bool 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same over packed rows [total][H][d]: a box is box_rows consecutive rows of one head.
+inline bool bwd_map_packed(EncodeTiledFnBwd enc, CUtensorMap *m, const void *ptr, bool f32, int d, int H,
+                           int total, int box_cols, int box_rows) {
+  const cuuint64_t esz = f32 ? 4 : 2;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(total > 0 ? total : 1)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * esz,
+                                 static_cast<cuuint64_t>(H) * static_cast<cuuint64_t>(d) * esz};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), 1u, static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+             const_cast<void *>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             f32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Packed variable-length sequences ([total, H, d] rows, [B + 1] offsets on the device).
+struct PackedSeqs {
+  const int *cu_q, *cu_k;
+  int total_q, total_k, max_q, max_k;
+};
+
 template <int D, int DH, int BQ, bool WINDOW>
 inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
@@ -597,18 +655,29 @@ template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                         int Hkv, int N, int left, int right, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
-                        TimerStartFn tstart, TimerStopFn tstop) {
-  const long long rows = static_cast<long long>(B) * Hq * N;
+                        TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk) {
+  const long long rows = pk ? static_cast<long long>(pk->total_q) * Hq : static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
   float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
   using L = BwdLayout<D, DH, BQ>;
   CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
-  const long long hq = static_cast<long long>(B) * Hq, hkv = static_cast<long long>(B) * Hkv;
-  if (!bwd_map(enc, &tq, q, false, D, N, hq, 64, BQ) || !bwd_map(enc, &tdo, dout, false, D, N, hq, 64, BQ) ||
-      !bwd_map(enc, &tk, k, false, D, N, hkv, 64, 128) || !bwd_map(enc, &tv, v, false, D, N, hkv, 64, 128) ||
-      !bwd_map(enc, &tdk, dk, false, D, N, hkv, 64, 128) || !bwd_map(enc, &tdv, dv, false, D, N, hkv, 64, 128) ||
-      !bwd_map(enc, &tdq, dqacc, true, D, N, hq, L::kDQCols, BQ))
-    return FA_ERR_CUDA;
+  if (pk) {
+    if (!bwd_map_packed(enc, &tq, q, false, D, Hq, pk->total_q, 64, BQ) ||
+        !bwd_map_packed(enc, &tdo, dout, false, D, Hq, pk->total_q, 64, BQ) ||
+        !bwd_map_packed(enc, &tk, k, false, D, Hkv, pk->total_k, 64, 128) ||
+        !bwd_map_packed(enc, &tv, v, false, D, Hkv, pk->total_k, 64, 128) ||
+        !bwd_map_packed(enc, &tdk, dk, false, D, Hkv, pk->total_k, 64, 128) ||
+        !bwd_map_packed(enc, &tdv, dv, false, D, Hkv, pk->total_k, 64, 128) ||
+        !bwd_map_packed(enc, &tdq, dqacc, true, D, Hq, pk->total_q, L::kDQCols, BQ))
+      return FA_ERR_CUDA;
+  } else {
+    const long long hq = static_cast<long long>(B) * Hq, hkv = static_cast<long long>(B) * Hkv;
+    if (!bwd_map(enc, &tq, q, false, D, N, hq, 64, BQ) || !bwd_map(enc, &tdo, dout, false, D, N, hq, 64, BQ) ||
+        !bwd_map(enc, &tk, k, false, D, N, hkv, 64, 128) || !bwd_map(enc, &tv, v, false, D, N, hkv, 64, 128) ||
+        !bwd_map(enc, &tdk, dk, false, D, N, hkv, 64, 128) || !bwd_map(enc, &tdv, dv, false, D, N, hkv, 64, 128) ||
+        !bwd_map(enc, &tdq, dqacc, true, D, N, hq, L::kDQCols, BQ))
+      return FA_ERR_CUDA;
+  }
 
   fa_bwd_pre_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
       static_cast<const __nv_bfloat16 *>(o), static_cast<const __nv_bfloat16 *>(dout), delta, dqacc, rows);
@@ -616,21 +685,29 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   BwdParams p;
   p.lse = lse;
   p.delta = delta;
+  p.dk = static_cast<__nv_bfloat16 *>(dk);
+  p.dv = static_cast<__nv_bfloat16 *>(dv);
+  p.cu_q = pk ? pk->cu_q : nullptr;
+  p.cu_k = pk ? pk->cu_k : nullptr;
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.N = N;
-  p.nkb = (N + 127) / 128;
+  p.N = pk ? 0 : N;
+  p.total_q = pk ? pk->total_q : 0;
+  p.total_k = pk ? pk->total_k : 0;
+  p.nkb = pk ? (pk->max_k + 127) / 128 : (N + 127) / 128;
   p.left = left;
   p.right = right;
   p.scale = scale;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
-  if (left >= 0 || right >= 0)
-    bwd_launch_main<D, DH, BQ, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
-  else
-    bwd_launch_main<D, DH, BQ, false>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+  if (grid > 0) {
+    if (left >= 0 || right >= 0)
+      bwd_launch_main<D, DH, BQ, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+    else
+      bwd_launch_main<D, DH, BQ, false>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+  }
   tstop(1, tslot, s);
 
   const long long n8 = rows * D / 8;
@@ -643,16 +720,16 @@ template <typename Enc>
 inline int bwd_launch(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                       int Hkv, int N, int d, int left, int right, float scale, cudaStream_t s, Enc enc,
-                      TimerStartFn tstart, TimerStopFn tstop) {
+                      TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk = nullptr) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
     return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop);
+                                    scale, s, e, tstart, tstop, pk);
   if (d == 128)
     return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                      scale, s, e, tstart, tstop);
+                                      scale, s, e, tstart, tstop, pk);
   return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop);
+                                    scale, s, e, tstart, tstop, pk);
 }
 
 }  // namespace fa

@@ -70,6 +70,38 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// The sequence a CTA works on.  Dense: Lq = Lk = N.  Packed: the lengths of sequence b and
+// its first rows in the packed tensors.  The keys are aligned to the END of the queries:
+// query i sits at key position c = i + dlt, dlt = Lk - Lq (0 for self-attention), and sees
+// the keys j with c - left <= j <= c + right, 0 <= j < Lk.
+struct SeqGeom {
+  int Lq, Lk, dlt, q_base, k_base;
+};
+
+// Records FA_ERR_SEQLENS when packed offsets are inconsistent (decreasing, past the packed
+// rows, or a sequence longer than the launch was sized for).
+__device__ __forceinline__ void report_bad_seqlens() {
+  if (atomicCAS(&g_fa_status, FA_OK, FA_ERR_SEQLENS) == FA_OK)
+    atomicExch(&g_fa_status_site, static_cast<unsigned long long>(blockIdx.x) << 32);
+}
+
+// Geometry of batch entry b; false (after reporting) when the offsets are inconsistent.
+__device__ __forceinline__ bool seq_geom(const int *cu_q, const int *cu_k, int N, int total_q,
+                                         int total_k, int max_lq, int max_lk, int b, SeqGeom &g) {
+  if (!cu_q) {
+    g = SeqGeom{N, N, 0, 0, 0};
+    return true;
+  }
+  const int q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_k[b], k1 = cu_k[b + 1];
+  if (q0 < 0 || q1 < q0 || q1 > total_q || k0 < 0 || k1 < k0 || k1 > total_k || q1 - q0 > max_lq ||
+      k1 - k0 > max_lk) {
+    report_bad_seqlens();
+    return false;
+  }
+  g = SeqGeom{q1 - q0, k1 - k0, (k1 - k0) - (q1 - q0), q0, k0};
+  return true;
+}
+
 // Self-test of the watchdog path: one thread waits, with a short limit, on an mbarrier
 // that nothing ever arrives at.  The wait must give up, record FA_ERR_DEVICE_TIMEOUT in
 // the status word, and return; no fault, trap or hang is involved.

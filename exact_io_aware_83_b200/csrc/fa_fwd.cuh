@@ -40,38 +40,47 @@
 namespace fa {
 
 struct FwdParams {
-  float *lse;       // [B, Hq, N] fp32
-  int B, Hq, Hkv, N;
-  int nqb;          // 128-row blocks per sequence, ceil(N / 128)
-  int pair_heads;   // 1: a unit is (2 heads, 1 query block); 0: (1 head, 2 query blocks)
-  int left, right;  // key window: j in [i - left, i + right]; -1 = unlimited (both < N)
-  float sl2;        // scale * log2(e)
+  float *lse;             // dense: [B, Hq, N]; packed sequences: [total_q, Hq]
+  __nv_bfloat16 *o;       // packed sequences: O, for the rows of tiles that end past a sequence
+  const int *cu_q, *cu_k; // packed sequences: [B + 1] row offsets (nullptr: dense [B, H, N, d])
+  int B, Hq, Hkv, N;      // dense: N = sequence length
+  int total_q, total_k;   // packed sequences: rows of the packed Q and K
+  int nqb;                // 128-row query blocks per sequence (packed: of the longest)
+  int pair_heads;         // 1: a unit is (2 heads, 1 query block); 0: (1 head, 2 query blocks)
+  int left, right;        // key band around the diagonal: [c - left, c + right]; -1 = unlimited
+  float sl2;              // scale * log2(e)
 };
 
-// First and last block of KB keys that some row of the 128-row query block qb can see.
-// Every row sees its own key, so the range is never empty and contains the diagonal.
+// Blocks of KB keys [lo, hi] that some row q0 .. min(q0 + 127, Lq - 1) of a query tile can
+// see; false when no row sees any key.
 template <int KB>
-__device__ __forceinline__ void key_block_range(const FwdParams &p, int qb, int &lo, int &hi) {
-  const int q0 = qb * 128, q1 = min(q0 + 127, p.N - 1);
-  lo = (p.left < 0 || q0 <= p.left) ? 0 : (q0 - p.left) / KB;
-  hi = (p.right < 0 || p.right >= p.N - 1 - q1) ? (p.N - 1) / KB : (q1 + p.right) / KB;
+__device__ __forceinline__ bool key_block_range(int left, int right, const SeqGeom &g, int q0, int &lo,
+                                                int &hi) {
+  const int c0 = q0 + g.dlt, c1 = min(q0 + 127, g.Lq - 1) + g.dlt;
+  const int first = (left < 0) ? 0 : max(0, c0 - left);
+  const int last = (right < 0) ? g.Lk - 1 : min(g.Lk - 1, c1 + right);
+  if (last < first) return false;
+  lo = first / KB;
+  hi = last / KB;
+  return true;
 }
 
 // True when some key of the block [kv0, kv0 + KB) is hidden from some row of the
-// 128-row query tile starting at q0 (window edge or the end of the sequence).
+// 128-row query tile whose first row sits at key position c0 (band edge or end of keys).
 template <int KB>
-__device__ __forceinline__ bool block_needs_mask(const FwdParams &p, int q0, int kv0) {
-  return kv0 + KB > p.N || (p.left >= 0 && q0 + 127 - kv0 > p.left) ||
-         (p.right >= 0 && kv0 + KB - 1 - q0 > p.right);
+__device__ __forceinline__ bool block_needs_mask(int left, int right, int Lk, int c0, int kv0) {
+  return kv0 + KB > Lk || (left >= 0 && c0 + 127 - kv0 > left) || (right >= 0 && kv0 + KB - 1 - c0 > right);
 }
 
-// Hides the scores of keys kv0 + c outside row qrow's window (or past N) with -inf.
+// Hides with -inf the scores of keys kv0 + c outside the band of the row at key position
+// c_row, and keys past Lk.
 template <int NC>
-__device__ __forceinline__ void mask_scores(uint32_t (&s)[NC], const FwdParams &p, int qrow, int kv0) {
+__device__ __forceinline__ void mask_scores(uint32_t (&s)[NC], int left, int right, int Lk, int c_row,
+                                            int kv0) {
   // key kv0 + c is visible iff c_lo <= c < c_hi
-  const int rel = qrow - kv0;
-  const int c_lo = p.left < 0 ? INT_MIN : rel - p.left;
-  const int c_hi = min(p.N - kv0, p.right < 0 ? INT_MAX : rel + p.right + 1);
+  const int rel = c_row - kv0;
+  const int c_lo = left < 0 ? INT_MIN : rel - left;
+  const int c_hi = min(Lk - kv0, right < 0 ? INT_MAX : rel + right + 1);
 #pragma unroll
   for (int c = 0; c < NC; ++c)
     if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
@@ -234,21 +243,40 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   }
   const int kvh = h[0] / g;
-  // Key blocks: the CTA walks the union [ulo, ulo + nu) of its tiles' ranges (contiguous,
-  // since both ranges contain their tile's diagonal block and the tiles are adjacent or
-  // equal); tile t takes part in the local blocks [a[t], a[t] + nblk[t]).
+  const bool packed = p.cu_q != nullptr;
+  SeqGeom sg;
+  if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, p.nqb * 128, INT_MAX, b, sg)) return;
+  // Packed sequences: tiles that start past the sequence's end have no rows.
+  valid[0] = valid[0] && qb[0] * 128 < sg.Lq;
+  valid[1] = valid[1] && qb[1] * 128 < sg.Lq;
+  if (!valid[0]) return;  // then tile 1 (same or later block) is past the end too
+  // Key blocks: the CTA walks the union [ulo, ulo + nu) of its tiles' ranges (contiguous:
+  // the tiles are the same rows or adjacent rows, and each range is an interval around
+  // its rows' key positions); tile t takes part in the local blocks [a[t], a[t] + nblk[t]).
+  // A tile whose rows see no key at all has nblk = 0 and only writes O = 0, LSE = -inf.
   int a[2], nblk[2], ulo, nu;
   {
-    int lo0, hi0, lo1, hi1;
-    key_block_range<128>(p, qb[0], lo0, hi0);
-    key_block_range<128>(p, valid[1] ? qb[1] : qb[0], lo1, hi1);
-    ulo = lo0 < lo1 ? lo0 : lo1;
-    nu = (hi0 > hi1 ? hi0 : hi1) - ulo + 1;
-    a[0] = lo0 - ulo;
-    nblk[0] = hi0 - lo0 + 1;
-    a[1] = lo1 - ulo;
-    nblk[1] = valid[1] ? hi1 - lo1 + 1 : 0;
+    int lo0 = 0, hi0 = -1, lo1 = 0, hi1 = -1;
+    const bool has0 = key_block_range<128>(p.left, p.right, sg, qb[0] * 128, lo0, hi0);
+    const bool has1 = valid[1] && key_block_range<128>(p.left, p.right, sg, qb[1] * 128, lo1, hi1);
+    ulo = has0 ? (has1 ? min(lo0, lo1) : lo0) : lo1;
+    const int uhi = has0 ? (has1 ? max(hi0, hi1) : hi0) : hi1;
+    nu = (has0 || has1) ? uhi - ulo + 1 : 0;
+    a[0] = has0 ? lo0 - ulo : 0;
+    nblk[0] = has0 ? hi0 - lo0 + 1 : 0;
+    a[1] = has1 ? lo1 - ulo : 0;
+    nblk[1] = has1 ? hi1 - lo1 + 1 : 0;
   }
+  // TMA coordinates (dimensions 1 and 2) of a 128-row tile: dense maps are [B*H][N][d],
+  // packed maps [total][H][d].
+  auto q_coords = [&](int hh, int row, int &c1, int &c2) {
+    c1 = packed ? hh : row;
+    c2 = packed ? sg.q_base + row : b * p.Hq + hh;
+  };
+  auto kv_coords = [&](int row, int &c1, int &c2) {
+    c1 = packed ? kvh : row;
+    c2 = packed ? sg.k_base + row : b * p.Hkv + kvh;
+  };
 
   // ---- barriers and tensor memory
   if (threadIdx.x == 0) {
@@ -280,12 +308,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tma_prefetch_desc(&tm_o);
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (!valid[t]) continue;
+        if (nblk[t] == 0) continue;
+        int c1, c2;
+        q_coords(h[t], qb[t] * 128, c1, c2);
         mbar_arrive_expect_tx(bar(L::kBarQ + t), L::kTileBytes);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
-          tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tm_q, bar(L::kBarQ + t), c * 64,
-                      qb[t] * 128, b * p.Hq + h[t]);
+          tma_load_3d(sQ + t * L::kTileBytes + c * L::kChunkBytes, &tm_q, bar(L::kBarQ + t), c * 64, c1, c2);
       }
       int issued = 0;
       bool ok = true;
@@ -300,10 +329,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kTileBytes);
           const CUtensorMap *m = kind ? &tm_v : &tm_k;
+          int c1, c2;
+          kv_coords((ulo + j) * 128, c1, c2);
 #pragma unroll
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_3d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, m, bar(L::kBarKVFull + slot),
-                        c * 64, (ulo + j) * 128, b * p.Hkv + kvh);
+                        c * 64, c1, c2);
           ++issued;
         }
       }
@@ -312,7 +343,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         wait_drain(bar(L::kBarKVFull + seq % S), (seq / S) & 1, 100000000ull);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (valid[t]) wait_drain(bar(L::kBarQ + t), 0, 100000000ull);
+        if (nblk[t] > 0) wait_drain(bar(L::kBarQ + t), 0, 100000000ull);
     }
     __syncwarp();
   } else if (warp == 8) {
@@ -345,17 +376,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (!first || kk > 0));
       };
 
-      bool ok = true;
+      bool ok = nu > 0;
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (ok && valid[t]) ok = wait_bounded(bar(L::kBarQ + t), 0, abort_flag, wait_site(1, L::kBarQ + t, 0));
+        if (ok && nblk[t] > 0) ok = wait_bounded(bar(L::kBarQ + t), 0, abort_flag, wait_site(1, L::kBarQ + t, 0));
       if (ok) ok = wait_bounded(bar(L::kBarKVFull + kslot(0)), kpar(0), abort_flag,
                                 wait_site(1, L::kBarKVFull + kslot(0), 0));
       if (ok) {
         tc_fence_after_sync();
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          if (!valid[t] || a[t] != 0) continue;
+          if (nblk[t] == 0 || a[t] != 0) continue;
           issue_qk(t, 0);
           tc_commit(bar(L::kBarS + t));
         }
@@ -374,7 +405,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // jt: block j counted from this tile's first block; -1 means only its first
           // S = Q K^T is due (K_{j+1} is the tile's first block).
           const int jt = j - a[t];
-          if (!ok || !valid[t] || jt + 1 < 0 || jt >= nblk[t]) continue;
+          if (!ok || nblk[t] == 0 || jt + 1 < 0 || jt >= nblk[t]) continue;
           if (jt >= 0) {
             if (!wait_bounded(bar(L::kBarP + t), jt & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
               ok = false;
@@ -448,8 +479,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_wait_ld_2x64(s0, s1);
       }
       const int kv0 = (my_j0 + j) * 128;
-      const bool masked = WINDOW ? block_needs_mask<128>(p, my_qb * 128, kv0) : kv0 + 128 > p.N;
-      if (masked) mask_scores<128>(s, p, qrow, kv0);
+      const bool masked =
+          WINDOW ? block_needs_mask<128>(p.left, p.right, sg.Lk, my_qb * 128 + sg.dlt, kv0) : kv0 + 128 > sg.Lk;
+      if (masked) mask_scores<128>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
       const float m_cand = row_max128(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       // 0 on a row's first visible block, else <= 1.  A window can hide a whole block from
@@ -487,18 +519,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (lane == 0) mbar_arrive(bar(L::kBarP + t));  // one arrival per warp
     }
 
-    // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store
+    // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store; a
+    // packed tile that ends past its sequence stores its rows directly instead, and a tile
+    // that sees no key writes O = 0 (no MMA ever touched its accumulator).
     if (my_valid) {
-      bool okw = ok && warp_wait_bounded(bar(L::kBarO + t), 0, abort_flag, wait_site(1, L::kBarO + t, 0));
+      bool okw = ok && (my_n == 0 || warp_wait_bounded(bar(L::kBarO + t), 0, abort_flag, wait_site(1, L::kBarO + t, 0)));
       okw = named_bar_and(1 + t, 128, okw && *abort_flag == 0);
       if (okw) {
         tc_fence_after_sync();
-        const float inv_l = 1.f / r_run;
+        const float inv_l = r_run > 0.f ? 1.f / r_run : 0.f;  // rows without keys: O = 0
         const uint32_t stage = sQ + t * L::kTileBytes;
+        const bool direct = packed && my_qb * 128 + 128 > sg.Lq;
+        const bool row_ok = qrow < sg.Lq;
+        __nv_bfloat16 *orow =
+            packed ? p.o + (static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h) * D : nullptr;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
-          tmem_ld_x32(tO + cc * 32, o);
+          if (my_n > 0) {
+            tmem_ld_x32(tO + cc * 32, o);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
+          }
           const uint32_t rowbase = stage + (cc / 2) * L::kChunkBytes + r * 128;
 #pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
@@ -508,20 +551,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 4; ++e)
               w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * inv_l,
                                  __uint_as_float(o[8 * uu + 2 * e + 1]) * inv_l);
-            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+            if (!direct)
+              st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+            else if (row_ok)
+              *reinterpret_cast<uint4 *>(orow + cc * 32 + uu * 8) = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
-        fence_proxy_async_smem();
-        named_bar_sync(1 + t, 128);
-        if (r == 0) {
+        if (!direct) {
+          fence_proxy_async_smem();
+          named_bar_sync(1 + t, 128);
+          if (r == 0) {
+            int c1, c2;
+            q_coords(my_h, my_qb * 128, c1, c2);
 #pragma unroll
-          for (int c = 0; c < L::kChunks; ++c)
-            tma_store_3d(&tm_o, stage + c * L::kChunkBytes, c * 64, my_qb * 128, b * p.Hq + my_h);
-          bulk_commit_group();
-          bulk_wait_group_read0();
+            for (int c = 0; c < L::kChunks; ++c) tma_store_3d(&tm_o, stage + c * L::kChunkBytes, c * 64, c1, c2);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
         }
-        if (qrow < p.N)
-          p.lse[static_cast<size_t>(b * p.Hq + my_h) * p.N + qrow] = (m_run + log2f(l_run)) * kLn2;
+        if (row_ok) {
+          const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+          if (packed)
+            p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h] = lse;
+          else
+            p.lse[static_cast<size_t>(b * p.Hq + my_h) * p.N + qrow] = lse;
+        }
       }
     }
   }

@@ -83,11 +83,21 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
   const int h = u % p.Hq;
   const int b = u / p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
+  const bool packed = p.cu_q != nullptr;
+  SeqGeom sg;
+  if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, p.nqb * 128, INT_MAX, b, sg)) return;
+  if (qb * 128 >= sg.Lq) return;  // packed: the block starts past the sequence's end
   // 64-key blocks [jlo, jlo + nblk) that some row of the query block can see; the loop
-  // index j below counts from jlo.
-  int jlo, jhi;
-  key_block_range<64>(p, qb, jlo, jhi);
+  // index j below counts from jlo.  nblk = 0: no row sees a key (O = 0, LSE = -inf).
+  int jlo = 0, jhi = -1;
+  key_block_range<64>(p.left, p.right, sg, qb * 128, jlo, jhi);
   const int nblk = jhi - jlo + 1;
+  // TMA coordinates (dimensions 1 and 2): dense maps are [B*H][N][d], packed [total][H][d].
+  const int q_c1 = packed ? h : qb * 128, q_c2 = packed ? sg.q_base + qb * 128 : b * p.Hq + h;
+  auto kv_coords = [&](int row, int &c1, int &c2) {
+    c1 = packed ? kvh : row;
+    c2 = packed ? sg.k_base + row : b * p.Hkv + kvh;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::kNumBars; ++i)
@@ -113,12 +123,14 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_o);
-      mbar_arrive_expect_tx(bar(L::kBarQ), L::kQBytes);
+      if (nblk > 0) {
+        mbar_arrive_expect_tx(bar(L::kBarQ), L::kQBytes);
 #pragma unroll
-      for (int c = 0; c < L::kChunks; ++c)
-        tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, bar(L::kBarQ), c * 64, qb * 128, b * p.Hq + h);
+        for (int c = 0; c < L::kChunks; ++c)
+          tma_load_3d(sQ + c * L::kQChunkBytes, &tm_q, bar(L::kBarQ), c * 64, q_c1, q_c2);
+      }
       int seq = 0;
-      bool ok = true;
+      bool ok = nblk > 0;
       auto produce = [&](bool is_v, int j) {
         const int slot = seq % S, use = seq / S;
         if (!wait_bounded(bar(L::kBarKVEmpty + slot), (use & 1) ^ 1, abort_flag,
@@ -128,13 +140,15 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
         }
         mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kKVBytes);
         const CUtensorMap *m = is_v ? &tm_v : &tm_k;
+        int c1, c2;
+        kv_coords((jlo + j) * 64, c1, c2);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(sKV + slot * L::kKVBytes + c * L::kKChunkBytes, m, bar(L::kBarKVFull + slot), c * 64,
-                      (jlo + j) * 64, b * p.Hkv + kvh);
+                      c1, c2);
         ++seq;
       };
-      produce(false, 0);
+      if (ok) produce(false, 0);
       if (ok && nblk > 1) produce(false, 1);
       for (int j = 0; ok && j < nblk; ++j) {
         produce(true, j);
@@ -142,7 +156,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       }
       for (int s2 = seq > S ? seq - S : 0; s2 < seq; ++s2)
         wait_drain(bar(L::kBarKVFull + s2 % S), (s2 / S) & 1, 100000000ull);
-      wait_drain(bar(L::kBarQ), 0, 100000000ull);
+      if (nblk > 0) wait_drain(bar(L::kBarQ), 0, 100000000ull);
     }
     __syncwarp();
   } else if (warp == 4) {
@@ -151,7 +165,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 64, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
       int seq = 0;
-      bool ok = wait_bounded(bar(L::kBarQ), 0, abort_flag, wait_site(2, L::kBarQ, 0));
+      bool ok = nblk > 0 && wait_bounded(bar(L::kBarQ), 0, abort_flag, wait_site(2, L::kBarQ, 0));
       // Take the next ring item: wait until it has landed; returns its slot.
       auto consume = [&](int j) -> int {
         const int slot = seq % S, use = seq / S;
@@ -227,8 +241,9 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       uint32_t s[64];
       tmem_ld_x64(tS, s);
       const int kv0 = (jlo + j) * 64;
-      const bool masked = WINDOW ? block_needs_mask<64>(p, qb * 128, kv0) : kv0 + 64 > p.N;
-      if (masked) mask_scores<64>(s, p, qrow, kv0);
+      const bool masked =
+          WINDOW ? block_needs_mask<64>(p.left, p.right, sg.Lk, qb * 128 + sg.dlt, kv0) : kv0 + 64 > sg.Lk;
+      if (masked) mask_scores<64>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
       const float m_cand = row_max<64>(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       // A window can hide a whole block from a row: while its max is still -inf the
@@ -270,15 +285,24 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       if (lane == 0) mbar_arrive(bar(L::kBarP + (j & 1)));  // one arrival per warp
     }
 
-    bool okw = ok && warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0));
+    bool okw = ok && (nblk == 0 || warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0)));
     okw = named_bar_and(1, 128, okw && *abort_flag == 0);
     if (okw) {
       tc_fence_after_sync();
-      const float inv_l = 1.f / r_run;
+      const float inv_l = r_run > 0.f ? 1.f / r_run : 0.f;  // rows without keys: O = 0
+      // A packed block that ends past its sequence stores its rows directly.
+      const bool direct = packed && qb * 128 + 128 > sg.Lq;
+      const bool row_ok = qrow < sg.Lq;
+      __nv_bfloat16 *orow = packed ? p.o + (static_cast<size_t>(sg.q_base + qrow) * p.Hq + h) * 256 : nullptr;
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         uint32_t o[32];
-        tmem_ld_x32(tO + cc * 32, o);
+        if (nblk > 0) {
+          tmem_ld_x32(tO + cc * 32, o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
         const uint32_t rowbase = sQ + (cc / 2) * L::kQChunkBytes + r * 128;
 #pragma unroll
         for (int uu = 0; uu < 4; ++uu) {
@@ -288,19 +312,29 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
           for (int e = 0; e < 4; ++e)
             w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * inv_l,
                                __uint_as_float(o[8 * uu + 2 * e + 1]) * inv_l);
-          st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+          if (!direct)
+            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+          else if (row_ok)
+            *reinterpret_cast<uint4 *>(orow + cc * 32 + uu * 8) = make_uint4(w[0], w[1], w[2], w[3]);
         }
       }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (r == 0) {
+      if (!direct) {
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (r == 0) {
 #pragma unroll
-        for (int c = 0; c < L::kChunks; ++c)
-          tma_store_3d(&tm_o, sQ + c * L::kQChunkBytes, c * 64, qb * 128, b * p.Hq + h);
-        bulk_commit_group();
-        bulk_wait_group_read0();
+          for (int c = 0; c < L::kChunks; ++c) tma_store_3d(&tm_o, sQ + c * L::kQChunkBytes, c * 64, q_c1, q_c2);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
       }
-      if (qrow < p.N) p.lse[static_cast<size_t>(b * p.Hq + h) * p.N + qrow] = (m_run + log2f(l_run)) * kLn2;
+      if (row_ok) {
+        const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        if (packed)
+          p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + h] = lse;
+        else
+          p.lse[static_cast<size_t>(b * p.Hq + h) * p.N + qrow] = lse;
+      }
     }
   }
 

@@ -10,9 +10,13 @@ Entry points mirror the C ABI names:
 * :func:`fa_fwd` / :func:`fa_bwd` - pointer-level calls (device pointers as ints);
 * :func:`fa_fwd_window` / :func:`fa_bwd_window` - the same for local attention (key j
   visible to query i iff i - left <= j <= i + right, -1 = unlimited);
+* :func:`fa_fwd_varlen` / :func:`fa_bwd_varlen` - packed variable-length sequences
+  ([total, H, d] rows, [B+1] offsets; query and key lengths may differ, the band being
+  aligned to the end of each sequence);
 * :func:`fa_decode` / :func:`fa_merge` - a few new query rows against a long key/value
   cache, split over the cache, and the merge of partial results;
-* :func:`fwd` / :func:`bwd` / :func:`decode` / :func:`merge` - tensor conveniences that
+* :func:`fwd` / :func:`bwd` / :func:`fwd_varlen` / :func:`bwd_varlen` / :func:`decode` /
+  :func:`merge` - tensor conveniences that
   allocate outputs with torch (``window=(left, right)`` selects local attention);
 * :func:`fa_bwd_workspace_bytes`, :func:`fa_device_status`, :func:`fa_status_string`.
 """
@@ -35,6 +39,7 @@ FA_ERR_WORKSPACE = 5
 FA_ERR_CUDA = 6
 FA_ERR_DEVICE_TIMEOUT = 7
 FA_ERR_SCRATCH_LIMIT = 8
+FA_ERR_SEQLENS = 9
 FA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -72,6 +77,14 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_bwd_window.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                       ci, ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd_window.restype = ci
+        lib.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci,
+                                      ci, ci, ci, cf, vp]
+        lib.fa_fwd_varlen.restype = ci
+        lib.fa_bwd_varlen_workspace_bytes.argtypes = [ci, ci, ci]
+        lib.fa_bwd_varlen_workspace_bytes.restype = sz
+        lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp,
+                                      ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cf, vp]
+        lib.fa_bwd_varlen.restype = ci
         lib.fa_decode_num_splits.argtypes = [ci, ci, ci, ci, ci, ci]
         lib.fa_decode_num_splits.restype = ci
         lib.fa_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci, ci]
@@ -147,6 +160,26 @@ def fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, 
     rule that calls overlapping on the GPU race on that buffer)."""
     _check(load().fa_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d,
                                  int(causal), float(scale), stream), "fa_bwd_noalloc")
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, Hq, Hkv, total_q, total_k, max_q, max_k, d,
+                  window_left, window_right, scale, stream) -> None:
+    _check(load().fa_fwd_varlen(q, k, v, o, lse, cu_q, cu_k, B, Hq, Hkv, total_q, total_k, max_q,
+                                max_k, d, int(window_left), int(window_right), float(scale),
+                                stream), "fa_fwd_varlen")
+
+
+def fa_bwd_varlen_workspace_bytes(Hq, total_q, d) -> int:
+    return int(load().fa_bwd_varlen_workspace_bytes(Hq, total_q, d))
+
+
+def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, cu_q, cu_k, B,
+                  Hq, Hkv, total_q, total_k, max_q, max_k, d, window_left, window_right, scale,
+                  stream) -> None:
+    _check(load().fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                                cu_q, cu_k, B, Hq, Hkv, total_q, total_k, max_q, max_k, d,
+                                int(window_left), int(window_right), float(scale), stream),
+           "fa_bwd_varlen")
 
 
 def fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d) -> int:
@@ -329,3 +362,62 @@ def merge(o_parts, lse_parts, out=None, lse=None):
     fa_merge(o_parts.data_ptr(), lse_parts.data_ptr(), o.data_ptr(), l.data_ptr(), S, rows, d,
              _stream_handle(o_parts))
     return o, l
+
+
+def _varlen_args(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, window):
+    import torch
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n)
+    if q.dim() != 3 or k.dim() != 3 or v.shape != k.shape or q.shape[2] != k.shape[2]:
+        raise ValueError("expected q [total_q, Hq, d] and k, v [total_k, Hkv, d]")
+    for c, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k")):
+        if not c.is_cuda or c.dtype != torch.int32 or not c.is_contiguous() or c.dim() != 1:
+            raise ValueError(f"{n} must be a contiguous int32 CUDA vector of B + 1 offsets")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 >= 2 offsets")
+    if window is not None and causal:
+        raise ValueError("give either causal=True or window=(left, right), not both")
+    left, right = (int(w) for w in window) if window is not None else (-1, 0 if causal else -1)
+    return (cu_seqlens_q.numel() - 1, q.shape[1], k.shape[1], q.shape[0], k.shape[0],
+            int(max_seqlen_q), int(max_seqlen_k), q.shape[2], left, right)
+
+
+def fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+               causal: bool = False, scale: float | None = None, window=None, out=None, lse=None):
+    """Attention over packed sequences: q [total_q, Hq, d], k/v [total_k, Hkv, d] bf16,
+    cu_seqlens_* int32 [B+1] on the GPU.  Returns O [total_q, Hq, d] and LSE [total_q, Hq].
+    causal / window bands are aligned to the end of each sequence."""
+    import torch
+    B, Hq, Hkv, tq, tk, mq, mk, d, left, right = _varlen_args(
+        q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, window)
+    scale = default_scale(d) if scale is None else scale
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((tq, Hq), dtype=torch.float32, device=q.device) if lse is None else lse
+    fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                  cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, Hq, Hkv, tq, tk, mq, mk, d,
+                  left, right, scale, _stream_handle(q))
+    return o, l
+
+
+def bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+               causal: bool = False, scale: float | None = None, window=None, workspace=None,
+               dq=None, dk=None, dv=None):
+    """dQ, dK, dV of <O, dO> for packed sequences (same arguments as fwd_varlen)."""
+    import torch
+    B, Hq, Hkv, tq, tk, mq, mk, d, left, right = _varlen_args(
+        q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal, window)
+    _need(o, "o")
+    _need(dout, "dout")
+    scale = default_scale(d) if scale is None else scale
+    nbytes = fa_bwd_varlen_workspace_bytes(Hq, tq, d)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                  workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                  cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(), B, Hq, Hkv, tq, tk, mq, mk, d,
+                  left, right, scale, _stream_handle(q))
+    return dq, dk, dv

@@ -163,3 +163,31 @@ def draw_decode(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, seed: int,
     k = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
     v = torch.randn((B, Hkv, Nk, d), generator=g, dtype=torch.float32)
     return q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)
+
+
+def draw_packed(lens_q, lens_k, Hq: int, Hkv: int, d: int, seed: int, q_std: float = 1.0):
+    """Packed variable-length sequences: bf16 CPU tensors q [total_q, Hq, d], k, v
+    [total_k, Hkv, d], dout like q, and int32 offsets cu_q, cu_k [B + 1] (starting at 0)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    cu_q = torch.tensor([0] + list(lens_q), dtype=torch.int64).cumsum(0).to(torch.int32)
+    cu_k = torch.tensor([0] + list(lens_k), dtype=torch.int64).cumsum(0).to(torch.int32)
+    tq, tk = int(cu_q[-1]), int(cu_k[-1])
+    q = torch.randn((tq, Hq, d), generator=g, dtype=torch.float32)
+    if q_std != 1.0:
+        q = q * q_std
+    k = torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32)
+    v = torch.randn((tk, Hkv, d), generator=g, dtype=torch.float32)
+    do = torch.randn((tq, Hq, d), generator=g, dtype=torch.float32)
+    bf = lambda t: t.to(torch.bfloat16)
+    return bf(q), bf(k), bf(v), bf(do), cu_q, cu_k
+
+
+def packed_lengths(n: int, mean: int, seed: int, lo: int = 16, hi: int = 8192):
+    """n sequence lengths with a long-tailed (log-normal) mix around `mean`, clipped to
+    [lo, hi]: the ragged batches that packing serves."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    x = torch.randn(n, generator=g, dtype=torch.float64) * 0.8
+    lens = (torch.exp(x) * mean / math.exp(0.32)).round().clamp(lo, hi).to(torch.int64)
+    return [int(v) for v in lens]

@@ -66,7 +66,8 @@ enum fa_status {
     FA_ERR_WORKSPACE = 5,      /* workspace missing or smaller than fa_bwd_workspace_bytes() */
     FA_ERR_CUDA = 6,           /* CUDA runtime/driver error (no sm_100 device, launch failure) */
     FA_ERR_DEVICE_TIMEOUT = 7, /* a kernel's bounded pipeline wait expired (device watchdog) */
-    FA_ERR_SCRATCH_LIMIT = 8   /* fa_bwd_noalloc: problem needs more than FA_NOALLOC_SCRATCH_BYTES */
+    FA_ERR_SCRATCH_LIMIT = 8,  /* fa_bwd_noalloc: problem needs more than FA_NOALLOC_SCRATCH_BYTES */
+    FA_ERR_SEQLENS = 9         /* packed-sequence offsets inconsistent (found on the device) */
 };
 
 /*
@@ -95,6 +96,30 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *l
                   float scale, void *stream);
 
 /*
+ * Forward pass over a batch of variable-length sequences packed along the token axis
+ * (the "FlashAttention1" Q&A page names variable sequence lengths among the scaling
+ * challenges, item 2; the packing and alignment below are this library's reading).
+ *   q, o [total_q, Hq, d] bf16;  k, v [total_k, Hkv, d] bf16;  lse [total_q, Hq] fp32 out
+ *   cu_seqlens_q, cu_seqlens_k: DEVICE int32 [B + 1] (4-byte aligned), nondecreasing row
+ *        offsets: sequence b owns query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1 and key
+ *        rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 (the offsets need not start at 0).
+ *   max_seqlen_q, max_seqlen_k: upper bounds on the per-sequence lengths (they size the
+ *        launch); total_q, total_k: rows of the packed tensors (<= 2^29 each).
+ * Query and key lengths may differ.  The key band is aligned to the END of both (bottom
+ * right): with dlt = Lk - Lq, query i sees keys j with
+ *     i + dlt - window_left <= j <= i + dlt + window_right,  0 <= j < Lk,
+ * a bound of -1 being unlimited (causal: window_left = -1, window_right = 0; full
+ * attention: both -1).  A query row that sees no key gets O = 0 and LSE = -inf.
+ * Offsets that are decreasing, exceed total_q / total_k, or describe a sequence longer
+ * than max_seqlen_q rows are reported on the device as FA_ERR_SEQLENS (fa_device_status);
+ * the affected sequences are left unwritten.
+ */
+int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                  const int *cu_seqlens_q, const int *cu_seqlens_k, int B, int Hq, int Hkv,
+                  int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                  int window_left, int window_right, float scale, void *stream);
+
+/*
  * Size in bytes of the fp32 scratch that fa_bwd needs: Delta_i = <dO_i, O_i> per query
  * row ([B, Hq, N] fp32) plus a dQ accumulator ([B, Hq, N, d] fp32), each padded to
  * 256 bytes.  Returns 0 for invalid sizes.
@@ -115,6 +140,23 @@ int fa_bwd(const void *q, const void *k, const void *v, const void *o, const flo
            const void *dout, void *dq, void *dk, void *dv, void *workspace,
            size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
            float scale, void *stream);
+
+/* Scratch bytes fa_bwd_varlen needs: Delta ([total_q, Hq] fp32) and a dQ accumulator
+ * ([total_q, Hq, d] fp32), each padded to 256 bytes.  0 for invalid sizes. */
+size_t fa_bwd_varlen_workspace_bytes(int Hq, int total_q, int d);
+
+/*
+ * Backward pass of fa_fwd_varlen: arguments as fa_fwd_varlen plus dout [total_q, Hq, d],
+ * dq [total_q, Hq, d], dk and dv [total_k, Hkv, d] (bf16; dK, dV summed over the query
+ * heads of each K/V head) and a workspace of fa_bwd_varlen_workspace_bytes() bytes.  A key
+ * that no query sees gets dK = dV = 0.  Offsets are checked as in the forward, with
+ * max_seqlen_k bounding the key lengths.
+ */
+int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                  const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                  size_t workspace_bytes, const int *cu_seqlens_q, const int *cu_seqlens_k, int B,
+                  int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
+                  int d, int window_left, int window_right, float scale, void *stream);
 
 /*
  * Backward pass of local attention: arguments as fa_bwd, with the window bounds of
@@ -209,7 +251,7 @@ int fa_merge(const float *o_parts, const float *lse_parts, void *o, float *lse, 
 
 /*
  * Synchronises `stream`, returns the device status word of the current device
- * (FA_OK or FA_ERR_DEVICE_TIMEOUT) and clears it.  Returns FA_ERR_CUDA if the
+ * (FA_OK, FA_ERR_DEVICE_TIMEOUT or FA_ERR_SEQLENS) and clears it.  Returns FA_ERR_CUDA if the
  * synchronisation itself fails.
  */
 int fa_device_status(void *stream);
