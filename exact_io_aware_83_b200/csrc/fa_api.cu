@@ -105,24 +105,32 @@ bool device_ready() {
       return;
     }
     bool ok = encode_fn() != nullptr;
-    ok = ok && set_smem(fa::fa_fwd_kernel<64, false>, fa::FwdLayout<64>::kSmemBytes);
-    ok = ok && set_smem(fa::fa_fwd_kernel<64, true>, fa::FwdLayout<64>::kSmemBytes);
-    ok = ok && set_smem(fa::fa_fwd_kernel<128, false>, fa::FwdLayout<128>::kSmemBytes);
-    ok = ok && set_smem(fa::fa_fwd_kernel<128, true>, fa::FwdLayout<128>::kSmemBytes);
-    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, false>, fa::kFwdRegsLaunch);
-    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, true>, fa::kFwdRegsLaunch);
-    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, false>, fa::kFwdRegsLaunch);
-    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, true>, fa::kFwdRegsLaunch);
-    ok = ok && set_smem(fa::fa_fwd_d256_kernel<false>, fa::FwdD256Layout::kSmemBytes);
-    ok = ok && set_smem(fa::fa_fwd_d256_kernel<true>, fa::FwdD256Layout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, fa::kAttnFull>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, fa::kAttnCausal>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, fa::kAttnGeneral>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnFull>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnCausal>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnGeneral>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnFull>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnCausal>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnGeneral>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnFull>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnCausal>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnGeneral>, fa::kFwdRegsLaunch);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnFull>, fa::FwdD256Layout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnCausal>, fa::FwdD256Layout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnGeneral>, fa::FwdD256Layout::kSmemBytes);
     using fa::BwdLayout;
     using fa::fa_bwd_main_kernel;
-    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, false>, BwdLayout<64, 64, 64>::kSmemBytes);
-    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, true>, BwdLayout<64, 64, 64>::kSmemBytes);
-    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, false>, BwdLayout<128, 128, 64>::kSmemBytes);
-    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, true>, BwdLayout<128, 128, 64>::kSmemBytes);
-    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, false>, BwdLayout<256, 128, 32>::kSmemBytes);
-    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, true>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnFull>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnCausal>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnGeneral>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, fa::kAttnFull>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, fa::kAttnCausal>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, fa::kAttnGeneral>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnFull>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnCausal>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnGeneral>, BwdLayout<256, 128, 32>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<64, 16>, fa::DecodeLayout<64, 16>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<64, 32>, fa::DecodeLayout<64, 32>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<64, 64>, fa::DecodeLayout<64, 64>::kSmemBytes);
@@ -303,32 +311,39 @@ void launch_merge(const float *o_part, const float *lse_part, void *o, float *ls
 
 // Launches the forward kernel for d (maps and parameters prepared by the caller).
 int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
-               FwdParams &p, int d, bool window, cudaStream_t s) {
+               FwdParams &p, int d, int mode, cudaStream_t s) {
   const int g = p.Hq / p.Hkv;
   const int tslot = timer_start(0, s);
   if (d == 256) {
     p.pair_heads = 0;
     const unsigned units = static_cast<unsigned>(p.B) * p.Hq * p.nqb;
-    if (window)
-      fa::fa_fwd_d256_kernel<true><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
-          tq, tk, tv, to, p);
+    constexpr int sm = fa::FwdD256Layout::kSmemBytes;
+    if (mode == fa::kAttnGeneral)
+      fa::fa_fwd_d256_kernel<fa::kAttnGeneral><<<units, fa::kFwdD256Threads, sm, s>>>(tq, tk, tv, to, p);
+    else if (mode == fa::kAttnCausal)
+      fa::fa_fwd_d256_kernel<fa::kAttnCausal><<<units, fa::kFwdD256Threads, sm, s>>>(tq, tk, tv, to, p);
     else
-      fa::fa_fwd_d256_kernel<false><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
-          tq, tk, tv, to, p);
+      fa::fa_fwd_d256_kernel<fa::kAttnFull><<<units, fa::kFwdD256Threads, sm, s>>>(tq, tk, tv, to, p);
   } else {
     p.pair_heads = (g % 2 == 0) ? 1 : 0;
     const unsigned units = p.pair_heads ? static_cast<unsigned>(p.B) * (p.Hq / 2) * p.nqb
                                         : static_cast<unsigned>(p.B) * p.Hq * ((p.nqb + 1) / 2);
     if (d == 64) {
-      if (window)
-        fa::fa_fwd_kernel<64, true><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+      constexpr int sm = fa::FwdLayout<64>::kSmemBytes;
+      if (mode == fa::kAttnGeneral)
+        fa::fa_fwd_kernel<64, fa::kAttnGeneral><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
+      else if (mode == fa::kAttnCausal)
+        fa::fa_fwd_kernel<64, fa::kAttnCausal><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
       else
-        fa::fa_fwd_kernel<64, false><<<units, fa::kFwdThreads, fa::FwdLayout<64>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+        fa::fa_fwd_kernel<64, fa::kAttnFull><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
     } else {
-      if (window)
-        fa::fa_fwd_kernel<128, true><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+      constexpr int sm = fa::FwdLayout<128>::kSmemBytes;
+      if (mode == fa::kAttnGeneral)
+        fa::fa_fwd_kernel<128, fa::kAttnGeneral><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
+      else if (mode == fa::kAttnCausal)
+        fa::fa_fwd_kernel<128, fa::kAttnCausal><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
       else
-        fa::fa_fwd_kernel<128, false><<<units, fa::kFwdThreads, fa::FwdLayout<128>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+        fa::fa_fwd_kernel<128, fa::kAttnFull><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
     }
   }
   const bool launched = cuda_ok(cudaGetLastError(), "fa_fwd launch");
@@ -425,7 +440,9 @@ int fa_fwd_window(const void *q, const void *k, const void *v, void *o, float *l
   p.left = left;
   p.right = right;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  return launch_fwd(tq, tk, tv, to, p, d, window, static_cast<cudaStream_t>(stream));
+  // Dense full and causal attention have their own kernel variants; other bands the general one.
+  const int mode = !window ? fa::kAttnFull : (left < 0 && right == 0 ? fa::kAttnCausal : fa::kAttnGeneral);
+  return launch_fwd(tq, tk, tv, to, p, d, mode, static_cast<cudaStream_t>(stream));
 }
 
 int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse, const int *cu_seqlens_q,
@@ -466,7 +483,7 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
   p.left = left;
   p.right = right;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  return launch_fwd(tq, tk, tv, to, p, d, left >= 0 || right >= 0, static_cast<cudaStream_t>(stream));
+  return launch_fwd(tq, tk, tv, to, p, d, fa::kAttnGeneral, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {

@@ -172,7 +172,9 @@ struct BwdLayout {
 // Warps 0-7: two elementwise warpgroups; 8-11: dQ drain; 12: MMA; 13: loader.
 constexpr int kBwdThreads = 448;
 
-template <int D, int DH, int BQ, bool WINDOW>
+// Kernel variants (kAttnFull, kAttnCausal, kAttnGeneral, see fa_common.cuh): dense full and
+// dense causal attention, and the general form (packed sequences and/or a key band).
+template <int D, int DH, int BQ, int MODE>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -208,17 +210,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int b = u / p.Hkv;
   const int g = p.Hq / p.Hkv;
   const int kv0 = kb * 128;
-  const bool packed = p.cu_q != nullptr;
-  SeqGeom sg;
-  if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, INT_MAX, p.nkb * 128, b, sg)) return;
-  if (kv0 >= sg.Lk) return;  // packed: the block starts past the sequence's keys
-  // Query blocks that can see some key of this block: query i sits at key position
-  // i + dlt and sees key j iff j - right <= i + dlt <= j + left.
-  const int kv1 = min(kv0 + 127, sg.Lk - 1);
-  const int first_i = p.right < 0 ? 0 : max(0, kv0 - p.right - sg.dlt);
-  const int last_i = p.left < 0 ? sg.Lq - 1 : min(sg.Lq - 1, kv1 + p.left - sg.dlt);
-  const int q_first = first_i / BQ;
-  const int nq = last_i >= first_i ? last_i / BQ - q_first + 1 : 0;  // 0: dK = dV = 0
+  constexpr bool GEN = MODE == kAttnGeneral;
+  const bool packed = GEN && p.cu_q != nullptr;
+  SeqGeom sg{p.N, p.N, 0, 0, 0};
+  int q_first, nq;
+  if constexpr (GEN) {
+    if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, INT_MAX, p.nkb * 128, b, sg)) return;
+    if (kv0 >= sg.Lk) return;  // packed: the block starts past the sequence's keys
+    // Query blocks that can see some key of this block: query i sits at key position
+    // i + dlt and sees key j iff j - right <= i + dlt <= j + left.
+    const int kv1 = min(kv0 + 127, sg.Lk - 1);
+    const int first_i = p.right < 0 ? 0 : max(0, kv0 - p.right - sg.dlt);
+    const int last_i = p.left < 0 ? sg.Lq - 1 : min(sg.Lq - 1, kv1 + p.left - sg.dlt);
+    q_first = first_i / BQ;
+    nq = last_i >= first_i ? last_i / BQ - q_first + 1 : 0;  // 0: dK = dV = 0
+  } else {
+    q_first = MODE == kAttnCausal ? kv0 / BQ : 0;
+    nq = (p.N + BQ - 1) / BQ - q_first;
+  }
   const int T = g * nq;  // steps: (query head of the group, query block)
   const int dcol0 = half * DH;  // first output column owned by this CTA
   // TMA coordinates (dimensions 1 and 2): dense maps are [B*H][N][cols], packed [total][H][cols].
@@ -327,8 +336,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       bool ok = wait_bounded(bar(L::kBarKV), 0, abort_flag, wait_site(3, L::kBarKV, 0));
-      if (ok && T > 0) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
-      if (ok && T > 0) {
+      if (ok && (!GEN || T > 0)) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
+      if (ok && (!GEN || T > 0)) {
         tc_fence_after_sync();
         issue_st(L::kTmS, sK, sQ);
         tc_commit(bar(L::kBarS));
@@ -428,7 +437,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!row_live) {
 #pragma unroll
         for (int c = 0; c < HC; ++c) pr[c] = 0.f;
-      } else if (WINDOW) {
+      } else if (GEN && (p.left >= 0 || p.right >= 0)) {
         const int c_lo = p.right < 0 ? INT_MIN : kv - p.right - sg.dlt - q0;
         const int c_hi = p.left < 0 ? INT_MAX : kv + p.left - sg.dlt - q0;
         if (c_lo > 0 || c_hi < HC - 1) {
@@ -436,6 +445,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int c = 0; c < HC; ++c)
             if (c < c_lo || c > c_hi) pr[c] = 0.f;
         }
+      } else if (MODE == kAttnCausal && q0 < kv) {
+#pragma unroll
+        for (int c = 0; c < HC; ++c)
+          if (q0 + c < kv) pr[c] = 0.f;
       }
       {
         uint32_t pk[HC / 2];
@@ -495,7 +508,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < DH / 32; ++cc) {
         uint32_t o[32];
-        if (T > 0) {
+        if (!GEN || T > 0) {
           tmem_ld_x32(tacc + cc * 32, o);
         } else {
 #pragma unroll
@@ -640,11 +653,11 @@ struct PackedSeqs {
   int total_q, total_k, max_q, max_k;
 };
 
-template <int D, int DH, int BQ, bool WINDOW>
+template <int D, int DH, int BQ, int MODE>
 inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
                             const CUtensorMap &tdq, const BwdParams &p, unsigned grid, cudaStream_t s) {
-  fa_bwd_main_kernel<D, DH, BQ, WINDOW><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
+  fa_bwd_main_kernel<D, DH, BQ, MODE><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
       tq, tk, tv, tdo, tdk, tdv, tdq, p);
 }
 
@@ -703,10 +716,14 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
   if (grid > 0) {
-    if (left >= 0 || right >= 0)
-      bwd_launch_main<D, DH, BQ, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+    // Dense full and causal attention have their own variants; packed sequences and other
+    // bands take the general one.
+    if (pk || (left >= 0 || (right >= 0 && right != 0)))
+      bwd_launch_main<D, DH, BQ, kAttnGeneral>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+    else if (right == 0)
+      bwd_launch_main<D, DH, BQ, kAttnCausal>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
     else
-      bwd_launch_main<D, DH, BQ, false>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+      bwd_launch_main<D, DH, BQ, kAttnFull>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
   }
   tstop(1, tslot, s);
 

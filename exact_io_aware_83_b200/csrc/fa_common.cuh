@@ -70,6 +70,11 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// Kernel variants: dense attention over every key, dense causal attention, and the general
+// form (packed variable-length sequences and/or a key band), whose extra bookkeeping the
+// two common dense cases do not pay for.
+constexpr int kAttnFull = 0, kAttnCausal = 1, kAttnGeneral = 2;
+
 // The sequence a CTA works on.  Dense: Lq = Lk = N.  Packed: the lengths of sequence b and
 // its first rows in the packed tensors.  The keys are aligned to the END of the queries:
 // query i sits at key position c = i + dlt, dlt = Lk - Lq (0 for self-attention), and sees

@@ -79,11 +79,17 @@ __device__ __forceinline__ void mask_scores(uint32_t (&s)[NC], int left, int rig
                                             int kv0) {
   // key kv0 + c is visible iff c_lo <= c < c_hi
   const int rel = c_row - kv0;
-  const int c_lo = left < 0 ? INT_MIN : rel - left;
   const int c_hi = min(Lk - kv0, right < 0 ? INT_MAX : rel + right + 1);
+  if (left < 0) {  // causal and right-bounded bands: one comparison per key
 #pragma unroll
-  for (int c = 0; c < NC; ++c)
-    if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
+    for (int c = 0; c < NC; ++c)
+      if (c >= c_hi) s[c] = __float_as_uint(-INFINITY);
+  } else {
+    const int c_lo = rel - left;
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+      if (c < c_lo || c >= c_hi) s[c] = __float_as_uint(-INFINITY);
+  }
 }
 
 constexpr float kLn2 = 0.693147180559945309f;
@@ -194,7 +200,40 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
   rsum = a + b;
 }
 
-template <int D, bool WINDOW>
+// Epilogue of the uncommon tiles: O / sum (0 for rows without keys, or all 0 when the tile
+// saw no key) either into the tile's swizzled staging rows (`direct` false, for a TMA
+// store) or straight to this thread's row of O in global memory (`row_ok` rows only).
+template <int D>
+__device__ __noinline__ void fwd_epilogue_rows(uint32_t tO, bool has_keys, float r_run, bool row_ok,
+                                               bool direct, uint32_t stage, int r, __nv_bfloat16 *orow) {
+  using L = FwdLayout<D>;
+  const float inv_l = r_run > 0.f ? 1.f / r_run : 0.f;
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    if (has_keys) {
+      tmem_ld_x32(tO + cc * 32, o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0u;
+    }
+    const uint32_t rowbase = stage + (cc / 2) * L::kChunkBytes + r * 128;
+#pragma unroll
+    for (int uu = 0; uu < 4; ++uu) {
+      const int unit = (cc % 2) * 4 + uu;
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * inv_l, __uint_as_float(o[8 * uu + 2 * e + 1]) * inv_l);
+      if (!direct)
+        st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
+      else if (row_ok)
+        *reinterpret_cast<uint4 *>(orow + cc * 32 + uu * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -243,19 +282,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   }
   const int kvh = h[0] / g;
-  const bool packed = p.cu_q != nullptr;
-  SeqGeom sg;
-  if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, p.nqb * 128, INT_MAX, b, sg)) return;
-  // Packed sequences: tiles that start past the sequence's end have no rows.
-  valid[0] = valid[0] && qb[0] * 128 < sg.Lq;
-  valid[1] = valid[1] && qb[1] * 128 < sg.Lq;
-  if (!valid[0]) return;  // then tile 1 (same or later block) is past the end too
+  constexpr bool GEN = MODE == kAttnGeneral;
+  const bool packed = GEN && p.cu_q != nullptr;
+  SeqGeom sg{p.N, p.N, 0, 0, 0};
   // Key blocks: the CTA walks the union [ulo, ulo + nu) of its tiles' ranges (contiguous:
   // the tiles are the same rows or adjacent rows, and each range is an interval around
   // its rows' key positions); tile t takes part in the local blocks [a[t], a[t] + nblk[t]).
   // A tile whose rows see no key at all has nblk = 0 and only writes O = 0, LSE = -inf.
-  int a[2], nblk[2], ulo, nu;
-  {
+  int a[2] = {0, 0}, nblk[2], ulo = 0, nu;
+  if constexpr (GEN) {
+    if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, p.nqb * 128, INT_MAX, b, sg)) return;
+    // Packed sequences: tiles that start past the sequence's end have no rows.
+    valid[0] = valid[0] && qb[0] * 128 < sg.Lq;
+    valid[1] = valid[1] && qb[1] * 128 < sg.Lq;
+    if (!valid[0]) return;  // then tile 1 (same or later block) is past the end too
     int lo0 = 0, hi0 = -1, lo1 = 0, hi1 = -1;
     const bool has0 = key_block_range<128>(p.left, p.right, sg, qb[0] * 128, lo0, hi0);
     const bool has1 = valid[1] && key_block_range<128>(p.left, p.right, sg, qb[1] * 128, lo1, hi1);
@@ -266,6 +306,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     nblk[0] = has0 ? hi0 - lo0 + 1 : 0;
     a[1] = has1 ? lo1 - ulo : 0;
     nblk[1] = has1 ? hi1 - lo1 + 1 : 0;
+  } else {
+#pragma unroll
+    for (int t = 0; t < 2; ++t) nblk[t] = !valid[t] ? 0 : (MODE == kAttnCausal ? qb[t] + 1 : p.nqb);
+    nu = nblk[0] > nblk[1] ? nblk[0] : nblk[1];
   }
   // TMA coordinates (dimensions 1 and 2) of a 128-row tile: dense maps are [B*H][N][d],
   // packed maps [total][H][d].
@@ -376,6 +420,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (!first || kk > 0));
       };
 
+      // Local block range of each tile (an empty tile gets an empty range; in the dense
+      // variants every tile starts at block 0).
+      const int first[2] = {!GEN ? 0 : (nblk[0] > 0 ? a[0] : 1 << 30), !GEN ? 0 : (nblk[1] > 0 ? a[1] : 1 << 30)};
+      const int last[2] = {a[0] + nblk[0] - 1, a[1] + nblk[1] - 1};
       bool ok = nu > 0;
 #pragma unroll
       for (int t = 0; t < 2; ++t)
@@ -402,19 +450,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bool knext = false;
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          // jt: block j counted from this tile's first block; -1 means only its first
-          // S = Q K^T is due (K_{j+1} is the tile's first block).
-          const int jt = j - a[t];
-          if (!ok || nblk[t] == 0 || jt + 1 < 0 || jt >= nblk[t]) continue;
-          if (jt >= 0) {
-            if (!wait_bounded(bar(L::kBarP + t), jt & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
+          // Tile t takes part in blocks first[t] .. last[t]; at j = first[t] - 1 only its
+          // first S = Q K^T is due.
+          if (!ok || j + 1 < first[t] || j > last[t]) continue;
+          if (j >= first[t]) {
+            if (!wait_bounded(bar(L::kBarP + t), (j - first[t]) & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
               ok = false;
               continue;
             }
             tc_fence_after_sync();
-            issue_pv(t, j, jt == 0);
+            issue_pv(t, j, j == first[t]);
           }
-          if (jt + 1 < nblk[t]) {
+          if (j < last[t]) {
             if (!knext) {
               if (!wait_bounded(bar(L::kBarKVFull + kslot(j + 1)), kpar(j + 1), abort_flag,
                                 wait_site(1, L::kBarKVFull + kslot(j + 1), j + 1))) {
@@ -479,17 +526,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_wait_ld_2x64(s0, s1);
       }
       const int kv0 = (my_j0 + j) * 128;
-      const bool masked =
-          WINDOW ? block_needs_mask<128>(p.left, p.right, sg.Lk, my_qb * 128 + sg.dlt, kv0) : kv0 + 128 > sg.Lk;
-      if (masked) mask_scores<128>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
+      bool masked;
+      if constexpr (GEN) {
+        masked = block_needs_mask<128>(p.left, p.right, sg.Lk, my_qb * 128 + sg.dlt, kv0);
+        if (masked) mask_scores<128>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
+      } else {
+        masked = (MODE == kAttnCausal && j == my_qb) || kv0 + 128 > p.N;
+        if (masked) {
+          const int lim = MODE == kAttnCausal ? min(qrow + 1, p.N) : p.N;  // keys kv < lim are visible
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
+        }
+      }
       const float m_cand = row_max128(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
-      // 0 on a row's first visible block, else <= 1.  A window can hide a whole block from
+      // 0 on a row's first visible block, else <= 1.  A band can hide a whole block from
       // a row; while its max is still -inf the offset stays 0 and alpha 1 (no inf - inf).
-      const float alpha = (WINDOW && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
+      const float alpha = (GEN && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
       float lsum, rsum;
       if (masked)
-        exp_block<128, false>(s, sl2, (WINDOW && m_new == -INFINITY) ? 0.f : m_new, tS, lsum,
+        exp_block<128, false>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum,
                               rsum);   // exact zeros for masked keys
       else
         exp_block<128, true>(s, sl2, m_new, tS, lsum, rsum);
@@ -519,29 +576,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (lane == 0) mbar_arrive(bar(L::kBarP + t));  // one arrival per warp
     }
 
-    // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store; a
-    // packed tile that ends past its sequence stores its rows directly instead, and a tile
-    // that sees no key writes O = 0 (no MMA ever touched its accumulator).
+    // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store.  Two
+    // cases take a separate path: a packed tile that ends past its sequence stores its
+    // rows directly, and a tile that sees no key writes O = 0 (no MMA touched it).
     if (my_valid) {
-      bool okw = ok && (my_n == 0 || warp_wait_bounded(bar(L::kBarO + t), 0, abort_flag, wait_site(1, L::kBarO + t, 0)));
+      bool okw = ok && ((GEN && my_n == 0) ||
+                        warp_wait_bounded(bar(L::kBarO + t), 0, abort_flag, wait_site(1, L::kBarO + t, 0)));
       okw = named_bar_and(1 + t, 128, okw && *abort_flag == 0);
-      if (okw) {
+      const bool direct = packed && my_qb * 128 + 128 > sg.Lq;
+      if (okw && (!GEN || (!direct && my_n > 0))) {
         tc_fence_after_sync();
-        const float inv_l = r_run > 0.f ? 1.f / r_run : 0.f;  // rows without keys: O = 0
+        const float inv_l = (!GEN || r_run > 0.f) ? 1.f / r_run : 0.f;  // rows without keys: O = 0
         const uint32_t stage = sQ + t * L::kTileBytes;
-        const bool direct = packed && my_qb * 128 + 128 > sg.Lq;
-        const bool row_ok = qrow < sg.Lq;
-        __nv_bfloat16 *orow =
-            packed ? p.o + (static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h) * D : nullptr;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
-          if (my_n > 0) {
-            tmem_ld_x32(tO + cc * 32, o);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0u;
-          }
+          tmem_ld_x32(tO + cc * 32, o);
           const uint32_t rowbase = stage + (cc / 2) * L::kChunkBytes + r * 128;
 #pragma unroll
           for (int uu = 0; uu < 4; ++uu) {
@@ -551,12 +601,22 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 4; ++e)
               w[e] = pack_bf16x2(__uint_as_float(o[8 * uu + 2 * e]) * inv_l,
                                  __uint_as_float(o[8 * uu + 2 * e + 1]) * inv_l);
-            if (!direct)
-              st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
-            else if (row_ok)
-              *reinterpret_cast<uint4 *>(orow + cc * 32 + uu * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+            st_shared_v4(rowbase + ((unit ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
           }
         }
+        fence_proxy_async_smem();
+        named_bar_sync(1 + t, 128);
+        if (r == 0) {
+          int c1, c2;
+          q_coords(my_h, my_qb * 128, c1, c2);
+#pragma unroll
+          for (int c = 0; c < L::kChunks; ++c) tma_store_3d(&tm_o, stage + c * L::kChunkBytes, c * 64, c1, c2);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+        }
+      } else if (GEN && okw) {
+        fwd_epilogue_rows<D>(tO, my_n > 0, r_run, qrow < sg.Lq, direct, sQ + t * L::kTileBytes, r,
+                             p.o + (static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h) * D);
         if (!direct) {
           fence_proxy_async_smem();
           named_bar_sync(1 + t, 128);
@@ -564,18 +624,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             int c1, c2;
             q_coords(my_h, my_qb * 128, c1, c2);
 #pragma unroll
-            for (int c = 0; c < L::kChunks; ++c) tma_store_3d(&tm_o, stage + c * L::kChunkBytes, c * 64, c1, c2);
+            for (int c = 0; c < L::kChunks; ++c)
+              tma_store_3d(&tm_o, sQ + t * L::kTileBytes + c * L::kChunkBytes, c * 64, c1, c2);
             bulk_commit_group();
             bulk_wait_group_read0();
           }
         }
-        if (row_ok) {
-          const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-          if (packed)
-            p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h] = lse;
-          else
-            p.lse[static_cast<size_t>(b * p.Hq + my_h) * p.N + qrow] = lse;
-        }
+      }
+      if (okw && qrow < sg.Lq) {
+        const float lse = (!GEN || l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        if (packed)
+          p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h] = lse;
+        else
+          p.lse[static_cast<size_t>(b * p.Hq + my_h) * p.N + qrow] = lse;
       }
     }
   }

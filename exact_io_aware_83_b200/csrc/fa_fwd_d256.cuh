@@ -56,7 +56,7 @@ struct FwdD256Layout {
 
 constexpr int kFwdD256Threads = 192;  // warps 0-3 softmax, 4 MMA, 5 TMA
 
-template <bool WINDOW>
+template <int MODE>  // kAttnFull, kAttnCausal or kAttnGeneral (see fa_common.cuh)
 __global__ void __launch_bounds__(kFwdD256Threads, 1)
     fa_fwd_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -83,15 +83,22 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
   const int h = u % p.Hq;
   const int b = u / p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
-  const bool packed = p.cu_q != nullptr;
-  SeqGeom sg;
-  if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, p.nqb * 128, INT_MAX, b, sg)) return;
-  if (qb * 128 >= sg.Lq) return;  // packed: the block starts past the sequence's end
+  constexpr bool GEN = MODE == kAttnGeneral;
+  const bool packed = GEN && p.cu_q != nullptr;
+  SeqGeom sg{p.N, p.N, 0, 0, 0};
   // 64-key blocks [jlo, jlo + nblk) that some row of the query block can see; the loop
   // index j below counts from jlo.  nblk = 0: no row sees a key (O = 0, LSE = -inf).
-  int jlo = 0, jhi = -1;
-  key_block_range<64>(p.left, p.right, sg, qb * 128, jlo, jhi);
-  const int nblk = jhi - jlo + 1;
+  int jlo = 0, nblk;
+  if constexpr (GEN) {
+    if (!seq_geom(p.cu_q, p.cu_k, p.N, p.total_q, p.total_k, p.nqb * 128, INT_MAX, b, sg)) return;
+    if (qb * 128 >= sg.Lq) return;  // packed: the block starts past the sequence's end
+    int jhi = -1;
+    key_block_range<64>(p.left, p.right, sg, qb * 128, jlo, jhi);
+    nblk = jhi - jlo + 1;
+  } else {
+    const int nkb_all = (p.N + 63) / 64;
+    nblk = MODE == kAttnCausal ? min(2 * qb + 2, nkb_all) : nkb_all;
+  }
   // TMA coordinates (dimensions 1 and 2): dense maps are [B*H][N][d], packed [total][H][d].
   const int q_c1 = packed ? h : qb * 128, q_c2 = packed ? sg.q_base + qb * 128 : b * p.Hq + h;
   auto kv_coords = [&](int row, int &c1, int &c2) {
@@ -241,17 +248,27 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       uint32_t s[64];
       tmem_ld_x64(tS, s);
       const int kv0 = (jlo + j) * 64;
-      const bool masked =
-          WINDOW ? block_needs_mask<64>(p.left, p.right, sg.Lk, qb * 128 + sg.dlt, kv0) : kv0 + 64 > sg.Lk;
-      if (masked) mask_scores<64>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
+      bool masked;
+      if constexpr (GEN) {
+        masked = block_needs_mask<64>(p.left, p.right, sg.Lk, qb * 128 + sg.dlt, kv0);
+        if (masked) mask_scores<64>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
+      } else {
+        masked = (MODE == kAttnCausal && kv0 + 63 > qb * 128) || kv0 + 64 > p.N;
+        if (masked) {
+          const int lim = MODE == kAttnCausal ? min(qrow + 1, p.N) : p.N;  // keys kv < lim are visible
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
+        }
+      }
       const float m_cand = row_max<64>(s) * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
-      // A window can hide a whole block from a row: while its max is still -inf the
-      // offset stays 0 and alpha 1.
-      const float alpha = (WINDOW && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
+      // A band can hide a whole block from a row: while its max is still -inf the offset
+      // stays 0 and alpha 1.
+      const float alpha = (GEN && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
       float lsum, rsum;
       if (masked)
-        exp_block<64, false>(s, sl2, (WINDOW && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum);
+        exp_block<64, false>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum);
       else
         exp_block<64, true>(s, sl2, m_new, tS, lsum, rsum);
       l_run = l_run * alpha + lsum;
@@ -285,11 +302,11 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       if (lane == 0) mbar_arrive(bar(L::kBarP + (j & 1)));  // one arrival per warp
     }
 
-    bool okw = ok && (nblk == 0 || warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0)));
+    bool okw = ok && ((GEN && nblk == 0) || warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0)));
     okw = named_bar_and(1, 128, okw && *abort_flag == 0);
     if (okw) {
       tc_fence_after_sync();
-      const float inv_l = r_run > 0.f ? 1.f / r_run : 0.f;  // rows without keys: O = 0
+      const float inv_l = (!GEN || r_run > 0.f) ? 1.f / r_run : 0.f;  // rows without keys: O = 0
       // A packed block that ends past its sequence stores its rows directly.
       const bool direct = packed && qb * 128 + 128 > sg.Lq;
       const bool row_ok = qrow < sg.Lq;
@@ -297,7 +314,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         uint32_t o[32];
-        if (nblk > 0) {
+        if (!GEN || nblk > 0) {
           tmem_ld_x32(tO + cc * 32, o);
         } else {
 #pragma unroll
@@ -329,7 +346,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
         }
       }
       if (row_ok) {
-        const float lse = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        const float lse = (!GEN || l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         if (packed)
           p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + h] = lse;
         else
