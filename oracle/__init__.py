@@ -8,9 +8,10 @@ Every function takes and returns numpy float64 arrays in the ``[B, H, N, d]`` la
 
 Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy example
 of the "Consideration"/FlashAttention article page, finite differences and invariants):
-``oracle_fwd``, ``oracle_bwd``, their key-window and variable-length forms,
+``oracle_fwd``, ``oracle_bwd``, their key-window, variable-length and dropout forms,
 ``oracle_decode``, ``oracle_merge`` and ``online_softmax_stats`` all have pins; none is
-"parity unpinned".
+"parity unpinned".  The dropout generator itself (Philox4x32-10) is pinned by statistics
+(keep rate, uniformity, independence), not by known-answer vectors.
 """
 from __future__ import annotations
 
@@ -54,6 +55,16 @@ def _lib():
         lib.oracle_bwd_varlen.argtypes = [dp, dp, dp, dp, ip, ip, dp, dp, dp, ci, ci, ci, ci,
                                           ci, ci, ci, ci, ctypes.c_double]
         lib.oracle_bwd_varlen.restype = ci
+        u8p = ctypes.POINTER(ctypes.c_ubyte)
+        u64 = ctypes.c_uint64
+        lib.oracle_dropout_mask.argtypes = [u8p, ci, ci, ctypes.c_double, u64]
+        lib.oracle_dropout_mask.restype = ci
+        lib.oracle_fwd_dropout.argtypes = [dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, ci,
+                                           ctypes.c_double, ctypes.c_double, u64]
+        lib.oracle_fwd_dropout.restype = ci
+        lib.oracle_bwd_dropout.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, ci,
+                                           ctypes.c_double, ctypes.c_double, u64]
+        lib.oracle_bwd_dropout.restype = ci
         lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
         lib.oracle_online_softmax_stats.restype = ci
         _LIB = lib
@@ -213,6 +224,43 @@ def attention_bwd_varlen(q, k, v, dout, cu_q, cu_k, left: int, right: int, scale
                                   int(left), int(right), float(scale))
     if rc != 0:
         raise RuntimeError(f"oracle_bwd_varlen failed with {rc}")
+    return dq, dk, dv
+
+
+def dropout_keep_mask(BH: int, N: int, p: float, seed: int):
+    """uint8 [BH, N, N]: 1 where the probability of (query head bh, row i, key j) is kept."""
+    keep = np.empty((BH, N, N), dtype=np.uint8)
+    rc = _lib().oracle_dropout_mask(keep.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte)), BH, N,
+                                    float(p), int(seed) & 0xFFFFFFFFFFFFFFFF)
+    if rc != 0:
+        raise RuntimeError(f"oracle_dropout_mask failed with {rc}")
+    return keep
+
+
+def attention_fwd_dropout(q, k, v, causal: bool, scale: float, p: float, seed: int):
+    """O = (P * Z / (1 - p)) V with the Philox4x32-10 keep mask Z; LSE without dropout."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    rc = _lib().oracle_fwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N,
+                                   d, int(bool(causal)), float(scale), float(p),
+                                   int(seed) & 0xFFFFFFFFFFFFFFFF)
+    if rc != 0:
+        raise RuntimeError(f"oracle_fwd_dropout failed with {rc}")
+    return o, lse
+
+
+def attention_bwd_dropout(q, k, v, dout, causal: bool, scale: float, p: float, seed: int):
+    """dq, dk, dv of <O, dO> for attention_fwd_dropout with the same seed."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = _lib().oracle_bwd_dropout(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), B, Hq, Hkv, N, d, int(bool(causal)), float(scale),
+                                   float(p), int(seed) & 0xFFFFFFFFFFFFFFFF)
+    if rc != 0:
+        raise RuntimeError(f"oracle_bwd_dropout failed with {rc}")
     return dq, dk, dv
 
 

@@ -42,6 +42,7 @@
  * -2 when scratch memory cannot be obtained.
  */
 #include <math.h>
+#include <stdint.h>
 #include <stdlib.h>
 #include <stddef.h>
 
@@ -552,4 +553,194 @@ int oracle_bwd_varlen(const double *q, const double *k, const double *v, const d
     free(L);
     free(D);
     return fail ? -2 : 0;
+}
+
+/*
+ * Attention dropout.  The deep-dive page names dropout among the memory-bound steps of
+ * standard attention ("Quantitative Evidence") but gives no generator; the reading here:
+ * every probability P_ij of query head bh is kept with probability 1 - p and kept values
+ * are scaled by 1 / (1 - p), so
+ *     O_i = sum_j P_ij Z_ij / (1 - p) v_j,   Z_ij in {0, 1},
+ * while LSE_i is the logsumexp of the scores (dropout does not enter the normaliser).
+ * Z comes from the counter-based generator Philox4x32-10 (Salmon, Moraes, Dror and Shaw,
+ * "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011), written from its published
+ * definition: key (seed low 32 bits, seed high 32 bits), counter (j / 4, i, bh, 0); the
+ * 32-bit output word j % 4 is compared with thr = min(floor(p 2^32), 2^32 - 1) and the
+ * element is kept iff word >= thr.  The decision is integer-only, so any implementation
+ * of the same definition reproduces it bit for bit.
+ */
+static void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
+                          uint32_t k1, uint32_t out[4])
+{
+    for (int round = 0; round < 10; ++round) {
+        /* one Philox round: two 32x32 -> 64-bit products, then mix with the key */
+        const uint64_t prod0 = (uint64_t)0xD2511F53u * x0;
+        const uint64_t prod1 = (uint64_t)0xCD9E8D57u * x2;
+        const uint32_t y0 = (uint32_t)(prod1 >> 32) ^ x1 ^ k0;
+        const uint32_t y1 = (uint32_t)prod1;
+        const uint32_t y2 = (uint32_t)(prod0 >> 32) ^ x3 ^ k1;
+        const uint32_t y3 = (uint32_t)prod0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+        k0 += 0x9E3779B9u;  /* key schedule: Weyl sequence */
+        k1 += 0xBB67AE85u;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+static uint32_t drop_threshold(double p)
+{
+    const double t = floor(p * 4294967296.0);
+    return t >= 4294967295.0 ? 0xFFFFFFFFu : (uint32_t)t;
+}
+
+/* 1 when element (bh, i, j) is kept, 0 when dropped. */
+static int drop_keep(uint64_t seed, uint32_t thr, uint32_t bh, int i, int j)
+{
+    uint32_t w[4];
+    philox4x32_10((uint32_t)j >> 2, (uint32_t)i, bh, 0u, (uint32_t)seed, (uint32_t)(seed >> 32), w);
+    return w[j & 3] >= thr;
+}
+
+/* keep[bh][i][j] for BH query heads of N rows and N keys (uint8). */
+int oracle_dropout_mask(unsigned char *keep, int BH, int N, double p, uint64_t seed)
+{
+    if (!keep || BH < 1 || N < 1 || !(p >= 0.0 && p < 1.0)) return -1;
+    const uint32_t thr = drop_threshold(p);
+#pragma omp parallel for schedule(static)
+    for (long long r = 0; r < (long long)BH * N; ++r)
+        for (int j = 0; j < N; ++j)
+            keep[(size_t)r * N + j] = (unsigned char)drop_keep(seed, thr, (uint32_t)(r / N), (int)(r % N), j);
+    return 0;
+}
+
+int oracle_fwd_dropout(const double *q, const double *k, const double *v, double *o, double *lse,
+                       int B, int Hq, int Hkv, int N, int d, int causal, double scale, double p,
+                       uint64_t seed)
+{
+    if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !o || !lse || !(p >= 0.0 && p < 1.0))
+        return -1;
+    const int g = Hq / Hkv;
+    const uint32_t thr = drop_threshold(p);
+    const double inv_keep = 1.0 / (1.0 - p);
+    const long long rows = (long long)B * Hq * N;
+    int fail = 0;
+#pragma omp parallel reduction(|: fail)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!s) {
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < rows; ++r) {
+                const int i = (int)(r % N);
+                const long long bh = r / N;
+                const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+                const double *kh = k + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+                const double *vh = v + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+                const int hi = causal ? i + 1 : N;
+                const double L = scores_and_lse(q + (size_t)r * d, kh, 0, hi, d, scale, s);
+                double *oi = o + (size_t)r * d;
+                for (int c = 0; c < d; ++c) oi[c] = 0.0;
+                for (int j = 0; j < hi; ++j) {
+                    if (!drop_keep(seed, thr, (uint32_t)bh, i, j)) continue;
+                    const double pz = exp(s[j] - L) * inv_keep;
+                    const double *vj = vh + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) oi[c] += pz * vj[c];
+                }
+                lse[r] = L;
+            }
+            free(s);
+        }
+    }
+    return fail ? -2 : 0;
+}
+
+/*
+ * Gradient of <O, dO> for the dropout forward above (the mask is a fixed function of the
+ * seed): with Zs_ij = Z_ij / (1 - p),
+ *     dP_ij = Zs_ij <do_i, v_j>,  Delta_i = sum_j P_ij dP_ij (= <do_i, o_i>),
+ *     dS_ij = P_ij (dP_ij - Delta_i),
+ *     dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,  dV_j = sum_i P_ij Zs_ij do_i.
+ */
+int oracle_bwd_dropout(const double *q, const double *k, const double *v, const double *dout,
+                       double *dq, double *dk, double *dv, int B, int Hq, int Hkv, int N, int d,
+                       int causal, double scale, double p, uint64_t seed)
+{
+    if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !dout || !dq || !dk || !dv ||
+        !(p >= 0.0 && p < 1.0))
+        return -1;
+    const int g = Hq / Hkv;
+    const uint32_t thr = drop_threshold(p);
+    const double inv_keep = 1.0 / (1.0 - p);
+    const long long qrows = (long long)B * Hq * N;
+    double *Lv = (double *)malloc(sizeof(double) * (size_t)qrows);
+    double *Dv = (double *)malloc(sizeof(double) * (size_t)qrows);
+    if (!Lv || !Dv) { free(Lv); free(Dv); return -2; }
+    int fail = 0;
+#pragma omp parallel reduction(|: fail)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        double *dp = (double *)malloc(sizeof(double) * (size_t)N);
+        if (!s || !dp) {
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < qrows; ++r) {
+                const int i = (int)(r % N);
+                const long long bh = r / N;
+                const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+                const double *kh = k + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+                const double *vh = v + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+                const int hi = causal ? i + 1 : N;
+                const double Li = scores_and_lse(q + (size_t)r * d, kh, 0, hi, d, scale, s);
+                double Di = 0.0;
+                for (int j = 0; j < hi; ++j) {
+                    const double zs = drop_keep(seed, thr, (uint32_t)bh, i, j) ? inv_keep : 0.0;
+                    dp[j] = zs * dotd(dout + (size_t)r * d, vh + (size_t)j * d, d);
+                    Di += exp(s[j] - Li) * dp[j];
+                }
+                double *dqi = dq + (size_t)r * d;
+                for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+                for (int j = 0; j < hi; ++j) {
+                    const double dS = exp(s[j] - Li) * (dp[j] - Di);
+                    const double *kj = kh + (size_t)j * d;
+                    for (int c = 0; c < d; ++c) dqi[c] += dS * kj[c];
+                }
+                for (int c = 0; c < d; ++c) dqi[c] *= scale;
+                Lv[r] = Li;
+                Dv[r] = Di;
+            }
+        }
+        free(s);
+        free(dp);
+    }
+    if (fail) { free(Lv); free(Dv); return -2; }
+    const long long krows = (long long)B * Hkv * N;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long r = 0; r < krows; ++r) {
+        const int j = (int)(r % N);
+        const long long bk = r / N;
+        const int kvh = (int)(bk % Hkv), b = (int)(bk / Hkv);
+        const double *kj = k + (size_t)r * d, *vj = v + (size_t)r * d;
+        double *dkj = dk + (size_t)r * d, *dvj = dv + (size_t)r * d;
+        for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+        for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
+            const long long bh = (long long)b * Hq + h;
+            for (int i = causal ? j : 0; i < N; ++i) {
+                const size_t qr = (size_t)bh * N + i;
+                const double *qi = q + qr * d, *doi = dout + qr * d;
+                const double P = exp(scale * dotd(qi, kj, d) - Lv[qr]);
+                const double zs = drop_keep(seed, thr, (uint32_t)bh, i, j) ? inv_keep : 0.0;
+                const double dS = P * (zs * dotd(doi, vj, d) - Dv[qr]);
+                for (int c = 0; c < d; ++c) {
+                    dvj[c] += P * zs * doi[c];
+                    dkj[c] += dS * qi[c];
+                }
+            }
+        }
+        for (int c = 0; c < d; ++c) dkj[c] *= scale;
+    }
+    free(Lv);
+    free(Dv);
+    return 0;
 }

@@ -22,7 +22,11 @@ the causal mask on the wrong side, a missing scale) fails at least one test:
   closed forms (one part, equal weights, weights 1/4 and 3/4, all parts empty);
 * packed variable-length batches against the dense oracle per sequence (equal lengths),
   the decode oracle per sequence (unequal lengths, bottom-right band), a brute-force
-  masked softmax for banded windows, and central finite differences.
+  masked softmax for banded windows, and central finite differences;
+* dropout: p = 0 is plain attention, the forward equals the reweighted masked softmax
+  built from the keep mask, it is unbiased over seeds, its gradient matches central
+  differences, and the keep mask has the right rate for six p and no visible correlation
+  between neighbouring keys, rows, heads or seeds.
 """
 import math
 import os
@@ -666,3 +670,92 @@ def test_varlen_invalid_offsets_are_rejected():
         oracle.attention_fwd_varlen(q, q, q, [0, 3, 2], cq, -1, -1, 1.0)   # decreasing
     with pytest.raises(RuntimeError):
         oracle.attention_fwd_varlen(q, q, q, cq, [0, 2, 9], -1, -1, 1.0)   # past the end
+
+
+# ---------------------------------------------------------------------------- dropout
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_dropout_with_p_zero_is_plain_attention(causal):
+    r = _rng(83)
+    q, k, v, do = (r.normal(size=(1, 4, 9, 5)) for _ in range(4))
+    k, v = k[:, :2], v[:, :2]
+    o1, l1 = oracle.attention_fwd_dropout(q, k, v, causal, 0.5, 0.0, 77)
+    o2, l2 = oracle.attention_fwd(q, k, v, causal, 0.5)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    g1 = oracle.attention_bwd_dropout(q, k, v, do, causal, 0.5, 0.0, 77)
+    g2 = oracle.attention_bwd(q, k, v, do, causal, 0.5)[:3]
+    for a, b in zip(g1, g2):
+        np.testing.assert_allclose(a, b, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("p", [0.05, 0.1, 0.25, 0.5, 0.75, 0.9])
+def test_dropout_keep_rate_tracks_one_minus_p(p):
+    # The keep rate as a function of p is the complement of the 32-bit words' CDF: it
+    # must follow 1 - p within 5 standard errors over 4 x 256 x 256 elements.
+    keep = oracle.dropout_keep_mask(4, 256, p, seed=2024)
+    n = keep.size
+    assert abs(keep.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
+
+
+def test_dropout_mask_has_no_visible_correlation():
+    keep = oracle.dropout_keep_mask(2, 256, 0.5, seed=99).astype(np.float64) - 0.5
+    n = keep[:, :, 1:].size
+    bound = 5 * 0.25 / math.sqrt(n)          # 5 standard errors of a covariance of +-1/2 bits
+    assert abs((keep[:, :, 1:] * keep[:, :, :-1]).mean()) < bound    # neighbouring keys
+    assert abs((keep[:, 1:, :] * keep[:, :-1, :]).mean()) < bound    # neighbouring rows
+    assert abs((keep[1] * keep[0]).mean()) < 5 * 0.25 / math.sqrt(keep[0].size)  # heads
+    other = oracle.dropout_keep_mask(2, 256, 0.5, seed=100).astype(np.float64) - 0.5
+    assert abs((keep * other).mean()) < 5 * 0.25 / math.sqrt(keep.size)         # seeds
+    # Same seed, same mask: the generator is a pure function of (seed, head, row, key).
+    again = oracle.dropout_keep_mask(2, 256, 0.5, seed=99).astype(np.float64) - 0.5
+    np.testing.assert_array_equal(keep, again)
+
+
+def test_dropout_forward_is_the_masked_reweighted_softmax():
+    # Brute force from the keep mask: O = (softmax(S) * Z / (1 - p)) V, LSE unchanged.
+    r = _rng(89)
+    q, k, v = r.normal(size=(1, 2, 7, 4)), r.normal(size=(1, 2, 7, 4)), r.normal(size=(1, 2, 7, 4))
+    p, seed = 0.3, 5
+    o, lse = oracle.attention_fwd_dropout(q, k, v, True, 0.8, p, seed)
+    keep = oracle.dropout_keep_mask(2, 7, p, seed)
+    for h in range(2):
+        s = 0.8 * q[0, h] @ k[0, h].T
+        s = np.where(np.tril(np.ones((7, 7), dtype=bool)), s, -np.inf)
+        P = np.exp(s - scipy.special.logsumexp(s, axis=1, keepdims=True))
+        np.testing.assert_allclose(o[0, h], (P * keep[h] / (1 - p)) @ v[0, h], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[0, h], scipy.special.logsumexp(s, axis=1), atol=1e-13)
+
+
+def test_dropout_is_unbiased_over_seeds():
+    # E_Z[O] = O without dropout: the mean over 400 seeds lies within 5 standard errors.
+    r = _rng(97)
+    q, k, v = r.normal(size=(1, 1, 6, 3)), r.normal(size=(1, 1, 6, 3)), r.normal(size=(1, 1, 6, 3))
+    outs = np.stack([oracle.attention_fwd_dropout(q, k, v, False, 0.7, 0.4, s)[0]
+                     for s in range(400)])
+    ref, _ = oracle.attention_fwd(q, k, v, False, 0.7)
+    se = outs.std(axis=0) / math.sqrt(len(outs))
+    assert np.all(np.abs(outs.mean(axis=0) - ref) <= 5 * se + 1e-12)
+
+
+def test_dropout_gradients_match_central_differences():
+    r = _rng(101)
+    q, k, v, do = (r.normal(size=(1, 2, 5, 3)) for _ in range(4))
+    k, v = k[:, :1], v[:, :1]
+    p, seed, scale = 0.35, 123, 0.9
+    for causal in (False, True):
+        dq, dk, dv = oracle.attention_bwd_dropout(q, k, v, do, causal, scale, p, seed)
+        loss = lambda q_, k_, v_: float(
+            (oracle.attention_fwd_dropout(q_, k_, v_, causal, scale, p, seed)[0] * do).sum())
+        eps = 1e-6
+        for x, g, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+            num = np.zeros_like(x)
+            it = np.nditer(x, flags=["multi_index"])
+            for _ in it:
+                idx = it.multi_index
+                args_p = [q.copy(), k.copy(), v.copy()]
+                args_m = [q.copy(), k.copy(), v.copy()]
+                args_p[which][idx] += eps
+                args_m[which][idx] -= eps
+                num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+            np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7)
