@@ -117,6 +117,16 @@ bool device_ready() {
     ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnFull>, fa::kFwdRegsLaunch);
     ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnCausal>, fa::kFwdRegsLaunch);
     ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnGeneral>, fa::kFwdRegsLaunch);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, fa::kAttnFull, true>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, fa::kAttnCausal, true>, fa::FwdLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnFull, true>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnCausal, true>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnFull, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnCausal, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnFull, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_kernel<128, fa::kAttnCausal, true>, fa::kFwdRegsLaunch);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnFull, true>, fa::FwdD256Layout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnCausal, true>, fa::FwdD256Layout::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnFull>, fa::FwdD256Layout::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnCausal>, fa::FwdD256Layout::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnGeneral>, fa::FwdD256Layout::kSmemBytes);
@@ -131,6 +141,12 @@ bool device_ready() {
     ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnFull>, BwdLayout<256, 128, 32>::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnCausal>, BwdLayout<256, 128, 32>::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnGeneral>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnFull, true>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnCausal, true>, BwdLayout<64, 64, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, fa::kAttnFull, true>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, fa::kAttnCausal, true>, BwdLayout<128, 128, 64>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnFull, true>, BwdLayout<256, 128, 32>::kSmemBytes);
+    ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnCausal, true>, BwdLayout<256, 128, 32>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<64, 16>, fa::DecodeLayout<64, 16>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<64, 32>, fa::DecodeLayout<64, 32>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<64, 64>, fa::DecodeLayout<64, 64>::kSmemBytes);
@@ -310,45 +326,60 @@ void launch_merge(const float *o_part, const float *lse_part, void *o, float *ls
 }
 
 // Launches the forward kernel for d (maps and parameters prepared by the caller).
+template <int D, int MODE, bool DROP>
+void launch_fwd_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
+                  const FwdParams &p, unsigned units, cudaStream_t s) {
+  if constexpr (D == 256)
+    fa::fa_fwd_d256_kernel<MODE, DROP><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
+        tq, tk, tv, to, p);
+  else
+    fa::fa_fwd_kernel<D, MODE, DROP><<<units, fa::kFwdThreads, fa::FwdLayout<D>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+}
+
+template <int D>
+void launch_fwd_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
+                     const FwdParams &p, unsigned units, int mode, bool drop, cudaStream_t s) {
+  if (drop && mode == fa::kAttnCausal) launch_fwd_d<D, fa::kAttnCausal, true>(tq, tk, tv, to, p, units, s);
+  else if (drop) launch_fwd_d<D, fa::kAttnFull, true>(tq, tk, tv, to, p, units, s);
+  else if (mode == fa::kAttnGeneral) launch_fwd_d<D, fa::kAttnGeneral, false>(tq, tk, tv, to, p, units, s);
+  else if (mode == fa::kAttnCausal) launch_fwd_d<D, fa::kAttnCausal, false>(tq, tk, tv, to, p, units, s);
+  else launch_fwd_d<D, fa::kAttnFull, false>(tq, tk, tv, to, p, units, s);
+}
+
+// Launches the forward kernel for d (maps and parameters prepared by the caller).  With
+// `drop`, mode must be kAttnFull or kAttnCausal.
 int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
-               FwdParams &p, int d, int mode, cudaStream_t s) {
+               FwdParams &p, int d, int mode, cudaStream_t s, const fa::DropCfg *drop = nullptr) {
   const int g = p.Hq / p.Hkv;
+  p.drop = drop ? *drop : fa::DropCfg{};
   const int tslot = timer_start(0, s);
   if (d == 256) {
     p.pair_heads = 0;
     const unsigned units = static_cast<unsigned>(p.B) * p.Hq * p.nqb;
-    constexpr int sm = fa::FwdD256Layout::kSmemBytes;
-    if (mode == fa::kAttnGeneral)
-      fa::fa_fwd_d256_kernel<fa::kAttnGeneral><<<units, fa::kFwdD256Threads, sm, s>>>(tq, tk, tv, to, p);
-    else if (mode == fa::kAttnCausal)
-      fa::fa_fwd_d256_kernel<fa::kAttnCausal><<<units, fa::kFwdD256Threads, sm, s>>>(tq, tk, tv, to, p);
-    else
-      fa::fa_fwd_d256_kernel<fa::kAttnFull><<<units, fa::kFwdD256Threads, sm, s>>>(tq, tk, tv, to, p);
+    launch_fwd_mode<256>(tq, tk, tv, to, p, units, mode, drop != nullptr, s);
   } else {
     p.pair_heads = (g % 2 == 0) ? 1 : 0;
     const unsigned units = p.pair_heads ? static_cast<unsigned>(p.B) * (p.Hq / 2) * p.nqb
                                         : static_cast<unsigned>(p.B) * p.Hq * ((p.nqb + 1) / 2);
-    if (d == 64) {
-      constexpr int sm = fa::FwdLayout<64>::kSmemBytes;
-      if (mode == fa::kAttnGeneral)
-        fa::fa_fwd_kernel<64, fa::kAttnGeneral><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
-      else if (mode == fa::kAttnCausal)
-        fa::fa_fwd_kernel<64, fa::kAttnCausal><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
-      else
-        fa::fa_fwd_kernel<64, fa::kAttnFull><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
-    } else {
-      constexpr int sm = fa::FwdLayout<128>::kSmemBytes;
-      if (mode == fa::kAttnGeneral)
-        fa::fa_fwd_kernel<128, fa::kAttnGeneral><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
-      else if (mode == fa::kAttnCausal)
-        fa::fa_fwd_kernel<128, fa::kAttnCausal><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
-      else
-        fa::fa_fwd_kernel<128, fa::kAttnFull><<<units, fa::kFwdThreads, sm, s>>>(tq, tk, tv, to, p);
-    }
+    if (d == 64)
+      launch_fwd_mode<64>(tq, tk, tv, to, p, units, mode, drop != nullptr, s);
+    else
+      launch_fwd_mode<128>(tq, tk, tv, to, p, units, mode, drop != nullptr, s);
   }
   const bool launched = cuda_ok(cudaGetLastError(), "fa_fwd launch");
   timer_stop(0, tslot, s);
   return launched ? FA_OK : FA_ERR_CUDA;
+}
+
+// Dropout configuration: keep iff the Philox word >= floor(p 2^32) (capped at 2^32 - 1).
+bool make_drop(float p, unsigned long long seed, fa::DropCfg *out) {
+  if (!(p >= 0.f) || !(p < 1.f)) return false;
+  const double t = std::floor(static_cast<double>(p) * 4294967296.0);
+  out->thr = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  out->k0 = static_cast<uint32_t>(seed);
+  out->k1 = static_cast<uint32_t>(seed >> 32);
+  out->inv_keep = static_cast<float>(1.0 / (1.0 - static_cast<double>(p)));
+  return true;
 }
 
 // Packed-sequence sizes: totals up to 2^29 rows keep every band computation in int32.
@@ -562,6 +593,63 @@ int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, co
   const fa::PackedSeqs pk{cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k};
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, 0, d, left, right, scale, s,
                         encode_fn(), &timer_start, &timer_stop, &pk);
+}
+
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq, int Hkv,
+                   int N, int d, int causal, float dropout_p, unsigned long long seed, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  fa::DropCfg drop;
+  if (!make_drop(dropout_p, seed, &drop)) return FA_ERR_INVALID_ARG;
+  if (dropout_p == 0.f) return fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream);
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  const int kv_rows = d == 256 ? 64 : 128;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map_bf16(&tq, q, d, N, static_cast<long long>(B) * Hq, 128) ||
+      !make_map_bf16(&tk, k, d, N, static_cast<long long>(B) * Hkv, kv_rows) ||
+      !make_map_bf16(&tv, v, d, N, static_cast<long long>(B) * Hkv, kv_rows) ||
+      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, 128))
+    return FA_ERR_CUDA;
+  FwdParams p;
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.cu_q = p.cu_k = nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.total_q = p.total_k = 0;
+  p.nqb = (N + 127) / 128;
+  p.left = -1;
+  p.right = causal ? 0 : -1;
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  return launch_fwd(tq, tk, tv, to, p, d, causal ? fa::kAttnCausal : fa::kAttnFull, static_cast<cudaStream_t>(stream),
+                    &drop);
+}
+
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const float *lse, const void *dout,
+                   void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes, int B, int Hq, int Hkv,
+                   int N, int d, int causal, float dropout_p, unsigned long long seed, float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  fa::DropCfg drop;
+  if (!make_drop(dropout_p, seed, &drop)) return FA_ERR_INVALID_ARG;
+  if (dropout_p == 0.f)
+    return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N, d, causal, scale,
+                  stream);
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(B, Hq, N, d)) return FA_ERR_WORKSPACE;
+  const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  // N = 1 with causal is full attention (normalise_window's rule); the mask is the same.
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
+                        static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop, nullptr, &drop);
 }
 
 int fa_kernel_timing(int enable) {

@@ -105,6 +105,7 @@ struct BwdParams {
   int left, right;        // key band around the diagonal (see SeqGeom); -1 = unlimited
   float sl2;              // scale * log2(e)
   float scale;
+  DropCfg drop;           // dropout (kernels instantiated with DROP only)
 };
 
 // D: head dimension (contraction of S^T and dP^T); DH: output columns owned by a CTA
@@ -174,7 +175,7 @@ constexpr int kBwdThreads = 448;
 
 // Kernel variants (kAttnFull, kAttnCausal, kAttnGeneral, see fa_common.cuh): dense full and
 // dense causal attention, and the general form (packed sequences and/or a key band).
-template <int D, int DH, int BQ, int MODE>
+template <int D, int DH, int BQ, int MODE, bool DROP = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -450,10 +451,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < HC; ++c)
           if (q0 + c < kv) pr[c] = 0.f;
       }
+      // Dropout: bit c of `keep` is set when (query q0 + c, this key) is kept.  One Philox
+      // call gives the mask words of four consecutive keys for one query; the four lanes of
+      // a key group each call it for a different query and swap words in four shuffles.
+      uint32_t keep = 0xFFFFFFFFu;
+      if constexpr (DROP) {
+        keep = 0u;
+        const int m = lane & 3;  // == kv & 3
+        const uint32_t bh = static_cast<uint32_t>(b * p.Hq + step_head(i));
+#pragma unroll
+        for (int t = 0; t < HC / 4; ++t) {
+          uint32_t w[4];
+          philox4x32_10(static_cast<uint32_t>(kv) >> 2, static_cast<uint32_t>(q0 + 4 * t + m), bh, 0u, p.drop.k0,
+                        p.drop.k1, w);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const int si = (m + kk) & 3;  // word this lane sends: the key of lane (m + kk) & 3
+            const uint32_t sv = si == 0 ? w[0] : si == 1 ? w[1] : si == 2 ? w[2] : w[3];
+            const int from = (m - kk) & 3;  // that lane computed query q0 + 4t + from
+            const uint32_t rv = __shfl_sync(0xffffffffu, sv, (lane & ~3) | from);
+            keep |= (rv >= p.drop.thr ? 1u : 0u) << (4 * t + from);
+          }
+        }
+      }
       {
+        // P^T as the A operand of dV += P^T dO: dropped entries are 0 (the 1 / (1 - p)
+        // factor is applied to dV in the epilogue).
         uint32_t pk[HC / 2];
 #pragma unroll
-        for (int c = 0; c < HC / 2; ++c) pk[c] = pack_bf16x2(pr[2 * c], pr[2 * c + 1]);
+        for (int c = 0; c < HC / 2; ++c)
+          pk[c] = pack_bf16x2(((keep >> (2 * c)) & 1u) ? pr[2 * c] : 0.f, ((keep >> (2 * c + 1)) & 1u) ? pr[2 * c + 1] : 0.f);
         if constexpr (HC == 32) tmem_st_x16(tS, pk); else tmem_st_x8(tS, pk);
       }
       tmem_wait_st();
@@ -467,6 +494,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       {
         uint32_t rr[HC];
         if constexpr (HC == 32) tmem_ld_x32(tDP, rr); else tmem_ld_x16(tDP, rr);
+        if constexpr (DROP) {
+          // dS = P (Z dP / (1 - p) - Delta) with the dropout mask Z.
+#pragma unroll
+          for (int c = 0; c < HC; ++c)
+            rr[c] = __float_as_uint(((keep >> c) & 1u) ? __uint_as_float(rr[c]) * p.drop.inv_keep : 0.f);
+        }
 #pragma unroll
         for (int c4 = 0; c4 < HC / 4; ++c4) {
           const float4 dd = dl4[c4];
@@ -499,7 +532,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (okw) {
       tc_fence_after_sync();
       const uint32_t tacc = tmem + (wg ? L::kTmDK : L::kTmDV) + lane_off;
-      const float mul = wg ? p.scale : 1.f;
+      const float mul = wg ? p.scale : (DROP ? p.drop.inv_keep : 1.f);
       const uint32_t stage = wg ? sK : sV;
       // A packed key block that ends past its sequence stores its rows directly.
       const bool direct = packed && kv0 + 128 > sg.Lk;
@@ -653,11 +686,11 @@ struct PackedSeqs {
   int total_q, total_k, max_q, max_k;
 };
 
-template <int D, int DH, int BQ, int MODE>
+template <int D, int DH, int BQ, int MODE, bool DROP = false>
 inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
                             const CUtensorMap &tdq, const BwdParams &p, unsigned grid, cudaStream_t s) {
-  fa_bwd_main_kernel<D, DH, BQ, MODE><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
+  fa_bwd_main_kernel<D, DH, BQ, MODE, DROP><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
       tq, tk, tv, tdo, tdk, tdv, tdq, p);
 }
 
@@ -668,7 +701,7 @@ template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                         int Hkv, int N, int left, int right, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
-                        TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk) {
+                        TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk, const DropCfg *drop) {
   const long long rows = pk ? static_cast<long long>(pk->total_q) * Hq : static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
   float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
@@ -713,12 +746,17 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.right = right;
   p.scale = scale;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.drop = drop ? *drop : DropCfg{};
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
   if (grid > 0) {
     // Dense full and causal attention have their own variants; packed sequences and other
     // bands take the general one.
-    if (pk || (left >= 0 || (right >= 0 && right != 0)))
+    if (drop && right == 0)  // dropout: dense attention only (the host checks)
+      bwd_launch_main<D, DH, BQ, kAttnCausal, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+    else if (drop)
+      bwd_launch_main<D, DH, BQ, kAttnFull, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+    else if (pk || (left >= 0 || (right >= 0 && right != 0)))
       bwd_launch_main<D, DH, BQ, kAttnGeneral>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
     else if (right == 0)
       bwd_launch_main<D, DH, BQ, kAttnCausal>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
@@ -737,16 +775,17 @@ template <typename Enc>
 inline int bwd_launch(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                       int Hkv, int N, int d, int left, int right, float scale, cudaStream_t s, Enc enc,
-                      TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk = nullptr) {
+                      TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk = nullptr,
+                      const DropCfg *drop = nullptr) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
     return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk);
+                                    scale, s, e, tstart, tstop, pk, drop);
   if (d == 128)
     return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                      scale, s, e, tstart, tstop, pk);
+                                      scale, s, e, tstart, tstop, pk, drop);
   return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk);
+                                    scale, s, e, tstart, tstop, pk, drop);
 }
 
 }  // namespace fa

@@ -70,6 +70,38 @@ __device__ __forceinline__ void wait_drain(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// Counter-based generator Philox4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel Random
+// Numbers: As Easy as 1, 2, 3", SC 2011), written from its published definition: ten
+// rounds of two 32 x 32 -> 64-bit products mixed with the key, the key advanced by a Weyl
+// sequence between rounds.  Used for the attention-dropout keep mask.
+__device__ __forceinline__ void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
+                                              uint32_t k1, uint32_t (&out)[4]) {
+#pragma unroll
+  for (int round = 0; round < 10; ++round) {
+    const uint32_t hi0 = __umulhi(0xD2511F53u, x0), lo0 = 0xD2511F53u * x0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, x2), lo1 = 0xCD9E8D57u * x2;
+    const uint32_t y0 = hi1 ^ x1 ^ k0, y2 = hi0 ^ x3 ^ k1;
+    x0 = y0;
+    x1 = lo1;
+    x2 = y2;
+    x3 = lo0;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+// Dropout keep mask: probability (row i, key j) of query head bh is kept iff output word
+// j % 4 of Philox4x32-10(counter = (j / 4, i, bh, 0), key = (k0, k1)) is >= thr, where
+// thr = min(floor(p 2^32), 2^32 - 1); kept values are scaled by inv_keep = 1 / (1 - p).
+struct DropCfg {
+  uint32_t k0, k1, thr;
+  float inv_keep;
+};
+
 // Kernel variants: dense attention over every key, dense causal attention, and the general
 // form (packed variable-length sequences and/or a key band), whose extra bookkeeping the
 // two common dense cases do not pay for.

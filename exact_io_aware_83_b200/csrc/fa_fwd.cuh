@@ -49,6 +49,7 @@ struct FwdParams {
   int pair_heads;         // 1: a unit is (2 heads, 1 query block); 0: (1 head, 2 query blocks)
   int left, right;        // key band around the diagonal: [c - left, c + right]; -1 = unlimited
   float sl2;              // scale * log2(e)
+  DropCfg drop;           // dropout (kernels instantiated with DROP only)
 };
 
 // Blocks of KB keys [lo, hi] that some row q0 .. min(q0 + 127, Lq - 1) of a query tile can
@@ -158,18 +159,26 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) { return r
 // (f2_exp2_poly) instead of the MUFU unit, which is the forward's scarcest resource;
 // blocks containing masked keys use the MUFU path only so masked keys give exact zeros.
 // The caller waits for the stores (tcgen05.wait::st) before signalling the MMA warp.
-template <int N, bool POLY>
+// With DROP, P = 0 for keys the dropout mask drops (the sums keep every key: they
+// normalise the softmax, dropout only reweights it); dcnt = (first key / 4, row, head)
+// counter words of the mask for this row.
+template <int N, bool POLY, bool DROP = false>
 __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, float m, uint32_t tP, float &lsum,
-                                          float &rsum) {
+                                          float &rsum, const DropCfg &dc = DropCfg{}, uint32_t dkey4 = 0,
+                                          uint32_t drow = 0, uint32_t dbh = 0) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
   const uint64_t negm2 = f2_pack(-m, -m);
   uint64_t l0 = 0, l1 = 0, r0 = 0, r1 = 0;  // packed (0.f, 0.f)
 #pragma unroll
   for (int h = 0; h < N / 64; ++h) {
     uint32_t pk[32];
+    uint32_t dw[4];  // mask words of the current group of four keys
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
       const int pp = h * 32 + q;
+      if constexpr (DROP) {
+        if ((q & 1) == 0) philox4x32_10(dkey4 + static_cast<uint32_t>(pp / 2), drow, dbh, 0u, dc.k0, dc.k1, dw);
+      }
       const uint64_t x =
           f2_fma(f2_pack(__uint_as_float(s[2 * pp]), __uint_as_float(s[2 * pp + 1])), sl2x2, negm2);
       uint64_t pr;
@@ -189,6 +198,10 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
       } else {
         l0 = f2_add(l0, pr);
         r0 = f2_add(r0, bf16x2_widen(pk[q]));
+      }
+      if constexpr (DROP) {
+        const uint32_t wa = (q & 1) ? dw[2] : dw[0], wb = (q & 1) ? dw[3] : dw[1];
+        pk[q] &= (wa >= dc.thr ? 0x0000FFFFu : 0u) | (wb >= dc.thr ? 0xFFFF0000u : 0u);
       }
     }
     tmem_st_x32(tP + h * 32, pk);
@@ -233,7 +246,7 @@ __device__ __noinline__ void fwd_epilogue_rows(uint32_t tO, bool has_keys, float
   }
 }
 
-template <int D, int MODE>
+template <int D, int MODE, bool DROP = false>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -546,10 +559,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const float alpha = (GEN && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
       float lsum, rsum;
       if (masked)
-        exp_block<128, false>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum,
-                              rsum);   // exact zeros for masked keys
+        exp_block<128, false, DROP>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum, p.drop,
+                                    kv0 >> 2, qrow, b * p.Hq + my_h);   // exact zeros for masked keys
       else
-        exp_block<128, true>(s, sl2, m_new, tS, lsum, rsum);
+        exp_block<128, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 2, qrow, b * p.Hq + my_h);
       l_run = l_run * alpha + lsum;
       r_run = r_run * alpha + rsum;
       m_run = m_new;
@@ -586,7 +599,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool direct = packed && my_qb * 128 + 128 > sg.Lq;
       if (okw && (!GEN || (!direct && my_n > 0))) {
         tc_fence_after_sync();
-        const float inv_l = (!GEN || r_run > 0.f) ? 1.f / r_run : 0.f;  // rows without keys: O = 0
+        // rows without keys: O = 0; dropout scales the kept probabilities by 1 / (1 - p)
+        const float inv_l = (!GEN || r_run > 0.f) ? (DROP ? p.drop.inv_keep : 1.f) / r_run : 0.f;
         const uint32_t stage = sQ + t * L::kTileBytes;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {

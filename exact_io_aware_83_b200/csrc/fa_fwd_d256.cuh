@@ -56,7 +56,7 @@ struct FwdD256Layout {
 
 constexpr int kFwdD256Threads = 192;  // warps 0-3 softmax, 4 MMA, 5 TMA
 
-template <int MODE>  // kAttnFull, kAttnCausal or kAttnGeneral (see fa_common.cuh)
+template <int MODE, bool DROP = false>  // MODE: kAttnFull, kAttnCausal or kAttnGeneral (fa_common.cuh)
 __global__ void __launch_bounds__(kFwdD256Threads, 1)
     fa_fwd_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -268,9 +268,10 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       const float alpha = (GEN && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
       float lsum, rsum;
       if (masked)
-        exp_block<64, false>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum);
+        exp_block<64, false, DROP>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum, p.drop,
+                                   kv0 >> 2, qrow, b * p.Hq + h);
       else
-        exp_block<64, true>(s, sl2, m_new, tS, lsum, rsum);
+        exp_block<64, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 2, qrow, b * p.Hq + h);
       l_run = l_run * alpha + lsum;
       r_run = r_run * alpha + rsum;
       m_run = m_new;
@@ -306,7 +307,8 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
     okw = named_bar_and(1, 128, okw && *abort_flag == 0);
     if (okw) {
       tc_fence_after_sync();
-      const float inv_l = (!GEN || r_run > 0.f) ? 1.f / r_run : 0.f;  // rows without keys: O = 0
+      // rows without keys: O = 0; dropout scales the kept probabilities by 1 / (1 - p)
+      const float inv_l = (!GEN || r_run > 0.f) ? (DROP ? p.drop.inv_keep : 1.f) / r_run : 0.f;
       // A packed block that ends past its sequence stores its rows directly.
       const bool direct = packed && qb * 128 + 128 > sg.Lq;
       const bool row_ok = qrow < sg.Lq;

@@ -85,6 +85,12 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp,
                                       ci, ci, ci, ci, ci, ci, ci, ci, ci, ci, cf, vp]
         lib.fa_bwd_varlen.restype = ci
+        u64 = ctypes.c_ulonglong
+        lib.fa_fwd_dropout.argtypes = [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, u64, cf, vp]
+        lib.fa_fwd_dropout.restype = ci
+        lib.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                       ci, ci, ci, ci, ci, ci, cf, u64, cf, vp]
+        lib.fa_bwd_dropout.restype = ci
         lib.fa_decode_num_splits.argtypes = [ci, ci, ci, ci, ci, ci]
         lib.fa_decode_num_splits.restype = ci
         lib.fa_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci, ci]
@@ -182,6 +188,21 @@ def fa_bwd_varlen(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
            "fa_bwd_varlen")
 
 
+def fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, dropout_p, seed, scale,
+                   stream) -> None:
+    _check(load().fa_fwd_dropout(q, k, v, o, lse, B, Hq, Hkv, N, d, int(causal), float(dropout_p),
+                                 int(seed) & 0xFFFFFFFFFFFFFFFF, float(scale), stream),
+           "fa_fwd_dropout")
+
+
+def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, Hq, Hkv, N,
+                   d, causal, dropout_p, seed, scale, stream) -> None:
+    _check(load().fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                                 B, Hq, Hkv, N, d, int(causal), float(dropout_p),
+                                 int(seed) & 0xFFFFFFFFFFFFFFFF, float(scale), stream),
+           "fa_bwd_dropout")
+
+
 def fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d) -> int:
     return int(load().fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d))
 
@@ -260,10 +281,11 @@ def _window(causal, window):
 
 
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-        window=None):
+        window=None, dropout_p: float = 0.0, seed: int = 0):
     """O, LSE = attention(q, k, v); q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 on one GPU.
     ``window=(left, right)``: local attention, key j visible to query i iff
-    i - left <= j <= i + right (-1 = unlimited on that side)."""
+    i - left <= j <= i + right (-1 = unlimited on that side).  ``dropout_p`` > 0: attention
+    dropout with the Philox4x32-10 mask of ``seed`` (full or causal attention)."""
     import torch
     win = _window(causal, window)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -274,7 +296,12 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     scale = default_scale(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    if win is None:
+    if dropout_p:
+        if win is not None:
+            raise ValueError("dropout is supported with full or causal attention only")
+        fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                       B, Hq, Hkv, N, d, causal, dropout_p, seed, scale, _stream_handle(q))
+    elif win is None:
         fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
                B, Hq, Hkv, N, d, causal, scale, _stream_handle(q))
     else:
@@ -284,7 +311,8 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
 
 
 def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
-        workspace=None, dq=None, dk=None, dv=None, window=None):
+        workspace=None, dq=None, dk=None, dv=None, window=None, dropout_p: float = 0.0,
+        seed: int = 0):
     """dQ, dK, dV of <O, dO> given the forward's O and LSE (same causal / window)."""
     import torch
     win = _window(causal, window)
@@ -301,7 +329,11 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
             dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
             workspace.numel() * workspace.element_size(), B, Hq, Hkv, N, d)
-    if win is None:
+    if dropout_p:
+        if win is not None:
+            raise ValueError("dropout is supported with full or causal attention only")
+        fa_bwd_dropout(*ptrs, causal, dropout_p, seed, scale, _stream_handle(q))
+    elif win is None:
         fa_bwd(*ptrs, causal, scale, _stream_handle(q))
     else:
         fa_bwd_window(*ptrs, win[0], win[1], scale, _stream_handle(q))

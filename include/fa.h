@@ -16,6 +16,8 @@
  *  - exactness (the blocked result equals standard attention): the same Q&A, question
  *    on the key algorithmic innovations; the deep-dive page, section "Algorithm behind
  *    the article";
+ *  - attention dropout: named by the deep-dive page ("Quantitative Evidence"); the mask
+ *    generator is Philox4x32-10 (see fa_fwd_dropout);
  *  - grouped- and multi-query attention and head dimensions up to 256: the
  *    FlashAttention-2 page, "FlashAttention-2: Enhanced Performance";
  *  - causal masking: the deep-dive page names masking among the memory-bound steps
@@ -120,6 +122,23 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
                   int window_left, int window_right, float scale, void *stream);
 
 /*
+ * Forward pass with attention dropout.  The deep-dive page names dropout among the
+ * memory-bound steps of standard attention ("Quantitative Evidence") without specifying
+ * it; this library's reading: each probability P_ij of query head bh = b * Hq + h is kept
+ * with probability 1 - dropout_p and kept ones are scaled by 1 / (1 - dropout_p):
+ *     O_i = sum_j P_ij Z_ij / (1 - p) v_j,   LSE_i as without dropout.
+ * The keep mask Z is a pure function of (seed, bh, i, j): Philox4x32-10 (Salmon et al.,
+ * SC 2011) with key (seed & 0xffffffff, seed >> 32) and counter (j / 4, i, bh, 0); output
+ * word j % 4 keeps the element iff it is >= min(floor(p * 2^32), 2^32 - 1).  fa_bwd_dropout
+ * regenerates the same mask, so nothing N x N is stored.
+ * Arguments as fa_fwd, plus dropout_p in [0, 1) (0 runs fa_fwd) and the 64-bit seed.
+ * Dense layout; full or causal attention.
+ */
+int fa_fwd_dropout(const void *q, const void *k, const void *v, void *o, float *lse, int B,
+                   int Hq, int Hkv, int N, int d, int causal, float dropout_p,
+                   unsigned long long seed, float scale, void *stream);
+
+/*
  * Size in bytes of the fp32 scratch that fa_bwd needs: Delta_i = <dO_i, O_i> per query
  * row ([B, Hq, N] fp32) plus a dQ accumulator ([B, Hq, N, d] fp32), each padded to
  * 256 bytes.  Returns 0 for invalid sizes.
@@ -157,6 +176,15 @@ int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, co
                   size_t workspace_bytes, const int *cu_seqlens_q, const int *cu_seqlens_k, int B,
                   int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k,
                   int d, int window_left, int window_right, float scale, void *stream);
+
+/*
+ * Backward pass of fa_fwd_dropout (same dropout_p and seed; O and LSE from it): arguments
+ * as fa_bwd.  dV = sum_i P Z / (1 - p) dO, dS = P (Z dP / (1 - p) - Delta).
+ */
+int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                   const void *dout, void *dq, void *dk, void *dv, void *workspace,
+                   size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int causal,
+                   float dropout_p, unsigned long long seed, float scale, void *stream);
 
 /*
  * Backward pass of local attention: arguments as fa_bwd, with the window bounds of

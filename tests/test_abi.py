@@ -26,6 +26,7 @@ def _declared_functions():
 def test_header_declares_the_boundary():
     names = _declared_functions()
     for required in ("fa_fwd", "fa_bwd", "fa_fwd_window", "fa_bwd_window", "fa_decode",
+                     "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_dropout", "fa_bwd_dropout",
                      "fa_decode_num_splits", "fa_decode_workspace_bytes", "fa_merge",
                      "fa_bwd_workspace_bytes", "fa_device_status", "fa_status_string",
                      "fa_version"):
@@ -205,6 +206,18 @@ def test_merge_argument_errors(kw, code):
     a.update(kw)
     assert fa.load().fa_merge(a["op"], a["lp"], a["o"], a["lse"], a["parts"], a["rows"], a["d"],
                               None) == code
+
+
+@pytest.mark.parametrize("p_drop,causal,code", [
+    (-0.1, 0, fa.FA_ERR_INVALID_ARG), (1.0, 0, fa.FA_ERR_INVALID_ARG),
+    (float("nan"), 0, fa.FA_ERR_INVALID_ARG), (0.1, 2, fa.FA_ERR_INVALID_ARG),
+])
+def test_dropout_argument_errors(p_drop, causal, code):
+    lib = fa.load()
+    assert lib.fa_fwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 2, 1, 16, 128, causal, p_drop, 7,
+                              0.125, None) == code
+    assert lib.fa_bwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                              1, 2, 1, 16, 128, causal, p_drop, 7, 0.125, None) == code
 
 
 def test_workspace_size():
