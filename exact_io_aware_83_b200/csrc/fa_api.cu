@@ -371,14 +371,16 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   return launched ? FA_OK : FA_ERR_CUDA;
 }
 
-// Dropout configuration: keep iff the Philox word >= floor(p 2^32) (capped at 2^32 - 1).
+// Dropout configuration: keep iff the 16-bit Philox value >= floor(p 2^16) (capped at
+// 2^16 - 1); kept values are scaled by the inverse of the exact keep probability.
 bool make_drop(float p, unsigned long long seed, fa::DropCfg *out) {
   if (!(p >= 0.f) || !(p < 1.f)) return false;
-  const double t = std::floor(static_cast<double>(p) * 4294967296.0);
-  out->thr = t >= 4294967295.0 ? 0xFFFFFFFFu : static_cast<uint32_t>(t);
+  const double t = std::floor(static_cast<double>(p) * 65536.0);
+  out->thr = t >= 65535.0 ? 65535u : static_cast<uint32_t>(t);
+  out->thr2 = out->thr | (out->thr << 16);
   out->k0 = static_cast<uint32_t>(seed);
   out->k1 = static_cast<uint32_t>(seed >> 32);
-  out->inv_keep = static_cast<float>(1.0 / (1.0 - static_cast<double>(p)));
+  out->inv_keep = static_cast<float>(65536.0 / (65536.0 - static_cast<double>(out->thr)));
   return true;
 }
 

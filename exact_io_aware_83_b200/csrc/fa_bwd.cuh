@@ -452,25 +452,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (q0 + c < kv) pr[c] = 0.f;
       }
       // Dropout: bit c of `keep` is set when (query q0 + c, this key) is kept.  One Philox
-      // call gives the mask words of four consecutive keys for one query; the four lanes of
-      // a key group each call it for a different query and swap words in four shuffles.
+      // call gives the mask values of eight consecutive keys for one query; the eight
+      // lanes of a key group each call it for a different query and swap values in eight
+      // shuffles.
       uint32_t keep = 0xFFFFFFFFu;
       if constexpr (DROP) {
         keep = 0u;
-        const int m = lane & 3;  // == kv & 3
+        const int m = lane & 7;  // == kv & 7
         const uint32_t bh = static_cast<uint32_t>(b * p.Hq + step_head(i));
 #pragma unroll
-        for (int t = 0; t < HC / 4; ++t) {
+        for (int t = 0; t < HC / 8; ++t) {
           uint32_t w[4];
-          philox4x32_10(static_cast<uint32_t>(kv) >> 2, static_cast<uint32_t>(q0 + 4 * t + m), bh, 0u, p.drop.k0,
+          philox4x32_10(static_cast<uint32_t>(kv) >> 3, static_cast<uint32_t>(q0 + 8 * t + m), bh, 0u, p.drop.k0,
                         p.drop.k1, w);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const int si = (m + kk) & 3;  // word this lane sends: the key of lane (m + kk) & 3
-            const uint32_t sv = si == 0 ? w[0] : si == 1 ? w[1] : si == 2 ? w[2] : w[3];
-            const int from = (m - kk) & 3;  // that lane computed query q0 + 4t + from
-            const uint32_t rv = __shfl_sync(0xffffffffu, sv, (lane & ~3) | from);
-            keep |= (rv >= p.drop.thr ? 1u : 0u) << (4 * t + from);
+          for (int kk = 0; kk < 8; ++kk) {
+            const int si = (m + kk) & 7;  // value this lane sends: the key of lane (m + kk) & 7
+            const uint32_t sw = (si >> 1) == 0 ? w[0] : (si >> 1) == 1 ? w[1] : (si >> 1) == 2 ? w[2] : w[3];
+            const uint32_t sv = (si & 1) ? (sw >> 16) : (sw & 0xFFFFu);
+            const int from = (m - kk) & 7;  // that lane drew for query q0 + 8t + from
+            const uint32_t rv = __shfl_sync(0xffffffffu, sv, (lane & ~7) | from);
+            keep |= (rv >= p.drop.thr ? 1u : 0u) << (8 * t + from);
           }
         }
       }

@@ -94,11 +94,13 @@ __device__ __forceinline__ void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t
   out[3] = x3;
 }
 
-// Dropout keep mask: probability (row i, key j) of query head bh is kept iff output word
-// j % 4 of Philox4x32-10(counter = (j / 4, i, bh, 0), key = (k0, k1)) is >= thr, where
-// thr = min(floor(p 2^32), 2^32 - 1); kept values are scaled by inv_keep = 1 / (1 - p).
+// Dropout keep mask: probability (row i, key j) of query head bh is kept iff the 16-bit
+// value j % 8 of Philox4x32-10(counter = (j / 8, i, bh, 0), key = (k0, k1)) - the low (even
+// j) or high (odd j) half of output word (j % 8) / 2 - is >= thr = min(floor(p 2^16),
+// 2^16 - 1).  Kept values are scaled by inv_keep = 2^16 / (2^16 - thr), the inverse of the
+// exact keep probability.  thr2 holds thr in both halves, for packed halfword compares.
 struct DropCfg {
-  uint32_t k0, k1, thr;
+  uint32_t k0, k1, thr, thr2;
   float inv_keep;
 };
 

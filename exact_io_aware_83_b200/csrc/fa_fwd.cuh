@@ -160,11 +160,11 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) { return r
 // blocks containing masked keys use the MUFU path only so masked keys give exact zeros.
 // The caller waits for the stores (tcgen05.wait::st) before signalling the MMA warp.
 // With DROP, P = 0 for keys the dropout mask drops (the sums keep every key: they
-// normalise the softmax, dropout only reweights it); dcnt = (first key / 4, row, head)
-// counter words of the mask for this row.
+// normalise the softmax, dropout only reweights it); (dkey8, drow, dbh) = (first key / 8,
+// row, query head) are the mask's counter words for this row.
 template <int N, bool POLY, bool DROP = false>
 __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, float m, uint32_t tP, float &lsum,
-                                          float &rsum, const DropCfg &dc = DropCfg{}, uint32_t dkey4 = 0,
+                                          float &rsum, const DropCfg &dc = DropCfg{}, uint32_t dkey8 = 0,
                                           uint32_t drow = 0, uint32_t dbh = 0) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
   const uint64_t negm2 = f2_pack(-m, -m);
@@ -172,12 +172,12 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
 #pragma unroll
   for (int h = 0; h < N / 64; ++h) {
     uint32_t pk[32];
-    uint32_t dw[4];  // mask words of the current group of four keys
+    uint32_t dw[4];  // mask values of the current group of eight keys (two per word)
 #pragma unroll
     for (int q = 0; q < 32; ++q) {
       const int pp = h * 32 + q;
       if constexpr (DROP) {
-        if ((q & 1) == 0) philox4x32_10(dkey4 + static_cast<uint32_t>(pp / 2), drow, dbh, 0u, dc.k0, dc.k1, dw);
+        if ((q & 3) == 0) philox4x32_10(dkey8 + static_cast<uint32_t>(pp / 4), drow, dbh, 0u, dc.k0, dc.k1, dw);
       }
       const uint64_t x =
           f2_fma(f2_pack(__uint_as_float(s[2 * pp]), __uint_as_float(s[2 * pp + 1])), sl2x2, negm2);
@@ -199,10 +199,7 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
         l0 = f2_add(l0, pr);
         r0 = f2_add(r0, bf16x2_widen(pk[q]));
       }
-      if constexpr (DROP) {
-        const uint32_t wa = (q & 1) ? dw[2] : dw[0], wb = (q & 1) ? dw[3] : dw[1];
-        pk[q] &= (wa >= dc.thr ? 0x0000FFFFu : 0u) | (wb >= dc.thr ? 0xFFFF0000u : 0u);
-      }
+      if constexpr (DROP) pk[q] &= __vcmpgeu2(dw[q & 3], dc.thr2);  // keys 2pp, 2pp+1 = low, high half
     }
     tmem_st_x32(tP + h * 32, pk);
   }
@@ -560,9 +557,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float lsum, rsum;
       if (masked)
         exp_block<128, false, DROP>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum, p.drop,
-                                    kv0 >> 2, qrow, b * p.Hq + my_h);   // exact zeros for masked keys
+                                    kv0 >> 3, qrow, b * p.Hq + my_h);   // exact zeros for masked keys
       else
-        exp_block<128, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 2, qrow, b * p.Hq + my_h);
+        exp_block<128, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 3, qrow, b * p.Hq + my_h);
       l_run = l_run * alpha + lsum;
       r_run = r_run * alpha + rsum;
       m_run = m_new;

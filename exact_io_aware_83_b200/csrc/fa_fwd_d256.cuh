@@ -269,9 +269,9 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       float lsum, rsum;
       if (masked)
         exp_block<64, false, DROP>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum, p.drop,
-                                   kv0 >> 2, qrow, b * p.Hq + h);
+                                   kv0 >> 3, qrow, b * p.Hq + h);
       else
-        exp_block<64, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 2, qrow, b * p.Hq + h);
+        exp_block<64, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 3, qrow, b * p.Hq + h);
       l_run = l_run * alpha + lsum;
       r_run = r_run * alpha + rsum;
       m_run = m_new;

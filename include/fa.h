@@ -125,12 +125,14 @@ int fa_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *l
  * Forward pass with attention dropout.  The deep-dive page names dropout among the
  * memory-bound steps of standard attention ("Quantitative Evidence") without specifying
  * it; this library's reading: each probability P_ij of query head bh = b * Hq + h is kept
- * with probability 1 - dropout_p and kept ones are scaled by 1 / (1 - dropout_p):
- *     O_i = sum_j P_ij Z_ij / (1 - p) v_j,   LSE_i as without dropout.
+ * with probability 1 - p' and kept ones are scaled by 1 / (1 - p'):
+ *     O_i = sum_j P_ij Z_ij / (1 - p') v_j,   LSE_i as without dropout,
+ * where p' = thr / 2^16, thr = min(floor(dropout_p * 2^16), 2^16 - 1) (|p' - p| < 2^-16).
  * The keep mask Z is a pure function of (seed, bh, i, j): Philox4x32-10 (Salmon et al.,
- * SC 2011) with key (seed & 0xffffffff, seed >> 32) and counter (j / 4, i, bh, 0); output
- * word j % 4 keeps the element iff it is >= min(floor(p * 2^32), 2^32 - 1).  fa_bwd_dropout
- * regenerates the same mask, so nothing N x N is stored.
+ * SC 2011) with key (seed & 0xffffffff, seed >> 32) and counter (j / 8, i, bh, 0); its
+ * four output words hold eight 16-bit values, value j % 8 being the low (even j) or high
+ * (odd j) half of word (j % 8) / 2, and the element is kept iff that value is >= thr.
+ * fa_bwd_dropout regenerates the same mask, so nothing N x N is stored.
  * Arguments as fa_fwd, plus dropout_p in [0, 1) (0 runs fa_fwd) and the 64-bit seed.
  * Dense layout; full or causal attention.
  */
@@ -179,7 +181,7 @@ int fa_bwd_varlen(const void *q, const void *k, const void *v, const void *o, co
 
 /*
  * Backward pass of fa_fwd_dropout (same dropout_p and seed; O and LSE from it): arguments
- * as fa_bwd.  dV = sum_i P Z / (1 - p) dO, dS = P (Z dP / (1 - p) - Delta).
+ * as fa_bwd.  dV = sum_i P Z / (1 - p') dO, dS = P (Z dP / (1 - p') - Delta).
  */
 int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, const float *lse,
                    const void *dout, void *dq, void *dk, void *dv, void *workspace,

@@ -564,10 +564,13 @@ int oracle_bwd_varlen(const double *q, const double *k, const double *v, const d
  * while LSE_i is the logsumexp of the scores (dropout does not enter the normaliser).
  * Z comes from the counter-based generator Philox4x32-10 (Salmon, Moraes, Dror and Shaw,
  * "Parallel Random Numbers: As Easy as 1, 2, 3", SC 2011), written from its published
- * definition: key (seed low 32 bits, seed high 32 bits), counter (j / 4, i, bh, 0); the
- * 32-bit output word j % 4 is compared with thr = min(floor(p 2^32), 2^32 - 1) and the
- * element is kept iff word >= thr.  The decision is integer-only, so any implementation
- * of the same definition reproduces it bit for bit.
+ * definition: key (seed low 32 bits, seed high 32 bits), counter (j / 8, i, bh, 0).  The
+ * four 32-bit output words hold eight 16-bit values, value j % 8 being the low (even) or
+ * high (odd) half of word (j % 8) / 2; the element is kept iff that value is >= thr =
+ * min(floor(p 2^16), 2^16 - 1), so the keep probability is exactly 1 - thr / 2^16 and the
+ * kept values are scaled by its inverse, 2^16 / (2^16 - thr) (unbiased; within 2^-16 of
+ * 1 / (1 - p)).  The decision is integer-only, so any implementation of the same
+ * definition reproduces it bit for bit.
  */
 static void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, uint32_t k0,
                           uint32_t k1, uint32_t out[4])
@@ -589,16 +592,18 @@ static void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, ui
 
 static uint32_t drop_threshold(double p)
 {
-    const double t = floor(p * 4294967296.0);
-    return t >= 4294967295.0 ? 0xFFFFFFFFu : (uint32_t)t;
+    const double t = floor(p * 65536.0);
+    return t >= 65535.0 ? 65535u : (uint32_t)t;
 }
 
 /* 1 when element (bh, i, j) is kept, 0 when dropped. */
 static int drop_keep(uint64_t seed, uint32_t thr, uint32_t bh, int i, int j)
 {
     uint32_t w[4];
-    philox4x32_10((uint32_t)j >> 2, (uint32_t)i, bh, 0u, (uint32_t)seed, (uint32_t)(seed >> 32), w);
-    return w[j & 3] >= thr;
+    philox4x32_10((uint32_t)j >> 3, (uint32_t)i, bh, 0u, (uint32_t)seed, (uint32_t)(seed >> 32), w);
+    const uint32_t word = w[(j & 7) >> 1];
+    const uint32_t value = (j & 1) ? (word >> 16) : (word & 0xFFFFu);
+    return value >= thr;
 }
 
 /* keep[bh][i][j] for BH query heads of N rows and N keys (uint8). */
@@ -621,7 +626,7 @@ int oracle_fwd_dropout(const double *q, const double *k, const double *v, double
         return -1;
     const int g = Hq / Hkv;
     const uint32_t thr = drop_threshold(p);
-    const double inv_keep = 1.0 / (1.0 - p);
+    const double inv_keep = 65536.0 / (65536.0 - (double)thr);
     const long long rows = (long long)B * Hq * N;
     int fail = 0;
 #pragma omp parallel reduction(|: fail)
@@ -657,7 +662,7 @@ int oracle_fwd_dropout(const double *q, const double *k, const double *v, double
 
 /*
  * Gradient of <O, dO> for the dropout forward above (the mask is a fixed function of the
- * seed): with Zs_ij = Z_ij / (1 - p),
+ * seed): with Zs_ij = Z_ij / keep probability,
  *     dP_ij = Zs_ij <do_i, v_j>,  Delta_i = sum_j P_ij dP_ij (= <do_i, o_i>),
  *     dS_ij = P_ij (dP_ij - Delta_i),
  *     dQ_i = scale sum_j dS_ij k_j,  dK_j = scale sum_i dS_ij q_i,  dV_j = sum_i P_ij Zs_ij do_i.
@@ -671,7 +676,7 @@ int oracle_bwd_dropout(const double *q, const double *k, const double *v, const 
         return -1;
     const int g = Hq / Hkv;
     const uint32_t thr = drop_threshold(p);
-    const double inv_keep = 1.0 / (1.0 - p);
+    const double inv_keep = 65536.0 / (65536.0 - (double)thr);
     const long long qrows = (long long)B * Hq * N;
     double *Lv = (double *)malloc(sizeof(double) * (size_t)qrows);
     double *Dv = (double *)malloc(sizeof(double) * (size_t)qrows);

@@ -1,7 +1,7 @@
 """GPU parity of attention dropout (forward and backward) against the fp64 oracle.
 
-The keep mask is a pure function of (seed, head, row, key) (Philox4x32-10, integer
-threshold), so the kernel's mask must equal the oracle's bit for bit; that is checked
+The keep mask is a pure function of (seed, head, row, key) (Philox4x32-10, 16-bit values
+against an integer threshold), so the kernel's mask must equal the oracle's bit for bit; that is checked
 directly with Q = 0 and V = I (then O = P Z / (1 - p) exposes Z), and through dV with
 dO = I.  Outputs and gradients use the dense tolerances.
 """

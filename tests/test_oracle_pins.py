@@ -691,7 +691,7 @@ def test_dropout_with_p_zero_is_plain_attention(causal):
 
 @pytest.mark.parametrize("p", [0.05, 0.1, 0.25, 0.5, 0.75, 0.9])
 def test_dropout_keep_rate_tracks_one_minus_p(p):
-    # The keep rate as a function of p is the complement of the 32-bit words' CDF: it
+    # The keep rate as a function of p is the complement of the 16-bit values' CDF: it
     # must follow 1 - p within 5 standard errors over 4 x 256 x 256 elements.
     keep = oracle.dropout_keep_mask(4, 256, p, seed=2024)
     n = keep.size
@@ -723,7 +723,9 @@ def test_dropout_forward_is_the_masked_reweighted_softmax():
         s = 0.8 * q[0, h] @ k[0, h].T
         s = np.where(np.tril(np.ones((7, 7), dtype=bool)), s, -np.inf)
         P = np.exp(s - scipy.special.logsumexp(s, axis=1, keepdims=True))
-        np.testing.assert_allclose(o[0, h], (P * keep[h] / (1 - p)) @ v[0, h], rtol=0, atol=1e-13)
+        # kept values are scaled by the inverse of the exact keep probability 1 - thr / 2^16
+        inv_keep = 65536.0 / (65536.0 - math.floor(p * 65536.0))
+        np.testing.assert_allclose(o[0, h], (P * keep[h] * inv_keep) @ v[0, h], rtol=0, atol=1e-13)
         np.testing.assert_allclose(lse[0, h], scipy.special.logsumexp(s, axis=1), atol=1e-13)
 
 
