@@ -168,7 +168,8 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
                                           uint32_t drow = 0, uint32_t dbh = 0) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
   const uint64_t negm2 = f2_pack(-m, -m);
-  uint64_t l0 = 0, l1 = 0, r0 = 0, r1 = 0;  // packed (0.f, 0.f)
+  uint64_t l0 = 0, l1 = 0;  // packed (0.f, 0.f)
+  float ra0 = 0.f, ra1 = 0.f, rb0 = 0.f, rb1 = 0.f;
 #pragma unroll
   for (int h = 0; h < N / 64; ++h) {
     uint32_t pk[32];
@@ -192,12 +193,13 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
       float p0, p1;
       f2_unpack(pr, p0, p1);
       pk[q] = pack_bf16x2(p0, p1);
+      // Mixed-precision adds take the bf16 halves as they are (no widening to fp32 first).
       if (pp & 1) {
         l1 = f2_add(l1, pr);
-        r1 = f2_add(r1, bf16x2_widen(pk[q]));
+        add_bf16x2_f32(rb0, rb1, pk[q]);
       } else {
         l0 = f2_add(l0, pr);
-        r0 = f2_add(r0, bf16x2_widen(pk[q]));
+        add_bf16x2_f32(ra0, ra1, pk[q]);
       }
       if constexpr (DROP) pk[q] &= __vcmpgeu2(dw[q & 3], dc.thr2);  // keys 2pp, 2pp+1 = low, high half
     }
@@ -206,8 +208,7 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
   float a, b;
   f2_unpack(f2_add(l0, l1), a, b);
   lsum = a + b;
-  f2_unpack(f2_add(r0, r1), a, b);
-  rsum = a + b;
+  rsum = (ra0 + ra1) + (rb0 + rb1);
 }
 
 // Epilogue of the uncommon tiles: O / sum (0 for rows without keys, or all 0 when the tile
