@@ -153,23 +153,30 @@ __device__ __forceinline__ float row_max(const uint32_t (&s)[N]) {
 __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) { return row_max<128>(s); }
 
 // P = 2^(s * sl2 - m) for N scores, packed to bf16 pairs and stored to TMEM at tP (32
-// packed columns at a time, so few packed words are live at once), with the fp32 sum
-// (lsum, for the LSE) and the sum of the bf16-rounded values (rsum, the weights the
-// P V product uses).  With POLY, every fourth pair is evaluated on the FMA pipe
-// (f2_exp2_poly) instead of the MUFU unit, which is the forward's scarcest resource;
-// blocks containing masked keys use the MUFU path only so masked keys give exact zeros.
-// The caller waits for the stores (tcgen05.wait::st) before signalling the MMA warp.
+// packed columns at a time, so few packed words are live at once), and the fp32 sum
+// lsum.  With POLY, every fourth pair is evaluated on the FMA pipe (f2_exp2_poly) instead
+// of the MUFU unit, which is the forward's scarcest resource; blocks containing masked
+// keys use the MUFU path only so masked keys give exact zeros.  The caller waits for the
+// stores (tcgen05.wait::st) before signalling the MMA warp.
+//
+// O is normalised by the sum of the probabilities as the P V product saw them, i.e. after
+// rounding to bf16.  That sum differs from lsum mostly through the rounding of each
+// block's largest probability (in nearly one-hot rows it is the whole sum), so the
+// caller adds that one rounding error, bf16(p_max) - p_max, to lsum instead of summing
+// every rounded value (which would cost two more adds per pair).
 // With DROP, P = 0 for keys the dropout mask drops (the sums keep every key: they
 // normalise the softmax, dropout only reweights it); (dkey8, drow, dbh) = (first key / 8,
 // row, query head) are the mask's counter words for this row.
+// ppmax: the largest probability evaluated on the FMA pipe (0 without POLY), so the
+// caller can tell which evaluation produced the block's largest probability.
 template <int N, bool POLY, bool DROP = false>
 __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, float m, uint32_t tP, float &lsum,
-                                          float &rsum, const DropCfg &dc = DropCfg{}, uint32_t dkey8 = 0,
+                                          float &ppmax, const DropCfg &dc = DropCfg{}, uint32_t dkey8 = 0,
                                           uint32_t drow = 0, uint32_t dbh = 0) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
   const uint64_t negm2 = f2_pack(-m, -m);
   uint64_t l0 = 0, l1 = 0;  // packed (0.f, 0.f)
-  float ra0 = 0.f, ra1 = 0.f, rb0 = 0.f, rb1 = 0.f;
+  float pm = 0.f;
 #pragma unroll
   for (int h = 0; h < N / 64; ++h) {
     uint32_t pk[32];
@@ -185,6 +192,9 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
       uint64_t pr;
       if (POLY && (pp & 3) == 3) {
         pr = f2_exp2_poly(x);
+        float a0, a1;
+        f2_unpack(pr, a0, a1);
+        pm = fmax3(pm, a0, a1);
       } else {
         float x0, x1;
         f2_unpack(x, x0, x1);
@@ -193,14 +203,10 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
       float p0, p1;
       f2_unpack(pr, p0, p1);
       pk[q] = pack_bf16x2(p0, p1);
-      // Mixed-precision adds take the bf16 halves as they are (no widening to fp32 first).
-      if (pp & 1) {
+      if (pp & 1)
         l1 = f2_add(l1, pr);
-        add_bf16x2_f32(rb0, rb1, pk[q]);
-      } else {
+      else
         l0 = f2_add(l0, pr);
-        add_bf16x2_f32(ra0, ra1, pk[q]);
-      }
       if constexpr (DROP) pk[q] &= __vcmpgeu2(dw[q & 3], dc.thr2);  // keys 2pp, 2pp+1 = low, high half
     }
     tmem_st_x32(tP + h * 32, pk);
@@ -208,7 +214,17 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
   float a, b;
   f2_unpack(f2_add(l0, l1), a, b);
   lsum = a + b;
-  rsum = (ra0 + ra1) + (rb0 + rb1);
+  ppmax = pm;
+}
+
+// bf16 rounding error of the probability of a block's largest score (raw maximum smax,
+// offset m).  The largest probability was evaluated either on the MUFU path, which this
+// repeats bit for bit, or on the FMA pipe, in which case it is (within the polynomial's
+// ~1e-4 relative error) ppmax, the largest of those values.
+__device__ __forceinline__ float pmax_rounding(float smax, float sl2, float m, float ppmax) {
+  const float pmufu = ex2_approx(fmaf(smax, sl2, -m));
+  const float pmax = ppmax >= pmufu * 0.9990234375f ? ppmax : pmufu;  // 1 - 2^-10
+  return __bfloat162float(__float2bfloat16_rn(pmax)) - pmax;
 }
 
 // Epilogue of the uncommon tiles: O / sum (0 for rows without keys, or all 0 when the tile
@@ -515,9 +531,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const bool my_valid = t ? valid[1] : valid[0];
     const int qrow = my_qb * 128 + r;
     bool ok = my_valid;
-    // l_run: sum of the fp32 probabilities (for the LSE); r_run: sum of the same
-    // probabilities after rounding to bf16, i.e. of the weights the P V product
-    // actually used, so that O / r_run is a properly normalised average.
+    // l_run: sum of the fp32 probabilities (for the LSE); r_run: the same with each
+    // block's largest probability counted as rounded to bf16, i.e. (to within the other,
+    // much smaller rounding errors) the weights the P V product actually used, so that
+    // O / r_run is a properly normalised average.
     float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float sl2 = p.sl2;
     for (int j = 0; ok && j < my_n; ++j) {
@@ -550,19 +567,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
         }
       }
-      const float m_cand = row_max128(s) * sl2;
+      const float smax = row_max128(s);
+      const float m_cand = smax * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       // 0 on a row's first visible block, else <= 1.  A band can hide a whole block from
       // a row; while its max is still -inf the offset stays 0 and alpha 1 (no inf - inf).
       const float alpha = (GEN && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
-      float lsum, rsum;
+      const float m_use = (GEN && m_new == -INFINITY) ? 0.f : m_new;
+      float lsum, ppmax;
       if (masked)
-        exp_block<128, false, DROP>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum, p.drop,
-                                    kv0 >> 3, qrow, b * p.Hq + my_h);   // exact zeros for masked keys
+        exp_block<128, false, DROP>(s, sl2, m_use, tS, lsum, ppmax, p.drop, kv0 >> 3, qrow,
+                                    b * p.Hq + my_h);   // exact zeros for masked keys
       else
-        exp_block<128, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 3, qrow, b * p.Hq + my_h);
+        exp_block<128, true, DROP>(s, sl2, m_new, tS, lsum, ppmax, p.drop, kv0 >> 3, qrow, b * p.Hq + my_h);
       l_run = l_run * alpha + lsum;
-      r_run = r_run * alpha + rsum;
+      r_run = r_run * alpha + (lsum + pmax_rounding(smax, sl2, m_use, ppmax));
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O was last written by P V of block j-1, which completed before S_j was ready.

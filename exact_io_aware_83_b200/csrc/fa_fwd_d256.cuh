@@ -232,9 +232,8 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
     const uint32_t tO = tmem + L::kTmO + lane_off;
     const int qrow = qb * 128 + r;
     bool ok = true;
-    // l_run: sum of the fp32 probabilities (for the LSE); r_run: sum of the same
-    // probabilities after rounding to bf16, i.e. of the weights the P V product
-    // actually used, so that O / r_run is a properly normalised average.
+    // l_run: sum of the fp32 probabilities (for the LSE); r_run: the same with each
+    // block's largest probability counted as rounded to bf16 (see pmax_rounding).
     float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float sl2 = p.sl2;
     for (int j = 0; ok && j < nblk; ++j) {
@@ -261,19 +260,20 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
         }
       }
-      const float m_cand = row_max<64>(s) * sl2;
+      const float smax = row_max<64>(s);
+      const float m_cand = smax * sl2;
       const float m_new = (m_cand > m_run + kRescaleThreshold) ? m_cand : m_run;
       // A band can hide a whole block from a row: while its max is still -inf the offset
       // stays 0 and alpha 1.
       const float alpha = (GEN && m_new == m_run) ? 1.f : ex2_approx(m_run - m_new);
-      float lsum, rsum;
+      const float m_use = (GEN && m_new == -INFINITY) ? 0.f : m_new;
+      float lsum, ppmax;
       if (masked)
-        exp_block<64, false, DROP>(s, sl2, (GEN && m_new == -INFINITY) ? 0.f : m_new, tS, lsum, rsum, p.drop,
-                                   kv0 >> 3, qrow, b * p.Hq + h);
+        exp_block<64, false, DROP>(s, sl2, m_use, tS, lsum, ppmax, p.drop, kv0 >> 3, qrow, b * p.Hq + h);
       else
-        exp_block<64, true, DROP>(s, sl2, m_new, tS, lsum, rsum, p.drop, kv0 >> 3, qrow, b * p.Hq + h);
+        exp_block<64, true, DROP>(s, sl2, m_new, tS, lsum, ppmax, p.drop, kv0 >> 3, qrow, b * p.Hq + h);
       l_run = l_run * alpha + lsum;
-      r_run = r_run * alpha + rsum;
+      r_run = r_run * alpha + (lsum + pmax_rounding(smax, sl2, m_use, ppmax));
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // P V of block j-1 must have finished before O is rescaled.
