@@ -154,8 +154,9 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) { return r
 
 // P = 2^(s * sl2 - m) for N scores, packed to bf16 pairs and stored to TMEM at tP (32
 // packed columns at a time, so few packed words are live at once), and the fp32 sum
-// lsum.  With POLY, every fourth pair is evaluated on the FMA pipe (f2_exp2_poly) instead
-// of the MUFU unit, which is the forward's scarcest resource; blocks containing masked
+// lsum.  With POLY, every sixteenth pair is evaluated on the FMA pipe (f2_exp2_poly)
+// instead of the MUFU unit, to balance the two pipes (measured: 1/16 beats 0, 1/8, 1/4,
+// 3/8 and 1/2 now that the row sums are cheap); blocks containing masked
 // keys use the MUFU path only so masked keys give exact zeros.  The caller waits for the
 // stores (tcgen05.wait::st) before signalling the MMA warp.
 //
@@ -190,7 +191,7 @@ __device__ __forceinline__ void exp_block(const uint32_t (&s)[N], float sl2, flo
       const uint64_t x =
           f2_fma(f2_pack(__uint_as_float(s[2 * pp]), __uint_as_float(s[2 * pp + 1])), sl2x2, negm2);
       uint64_t pr;
-      if (POLY && (pp & 3) == 3) {
+      if (POLY && (pp & 15) == 15) {
         pr = f2_exp2_poly(x);
         float a0, a1;
         f2_unpack(pr, a0, a1);
