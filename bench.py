@@ -9,6 +9,10 @@ seeded i.i.d. N(0,1) inputs).  FLOPs follow the metric's convention: 4 B H N^2 d
 forward, halved when causal, and 2.5x that for the backward; a local-attention workload
 counts 4 d flop per visible (query, key) pair.
 
+--workload varlen_32k_ragged times fa_fwd_varlen + fa_bwd_varlen over a packed batch of
+ragged sequences (FLOPs of the visible pairs of each sequence); dropout_8k_causal times
+the dropout forward and backward.
+
 Decode workloads (--workload decode_*) time one fa_decode call per step (new query rows
 against a resident key/value cache, split over the cache and merged); their metric is
 the cache-read bandwidth in GB/s against the measured HBM copy peak.
@@ -149,7 +153,11 @@ def _oracle_sample(w, heads: int, seed: int):
     f64 = lambda t: t.float().double().numpy()
     q, k, v, do = f64(q), f64(k), f64(v), f64(do)
     t0 = time.perf_counter()
-    if w.window is not None:
+    if w.dropout_p:
+        oracle.attention_fwd_dropout(q, k, v, w.causal, w.scale, w.dropout_p, w.dropout_seed)
+        if w.backward:
+            oracle.attention_bwd_dropout(q, k, v, do, w.causal, w.scale, w.dropout_p, w.dropout_seed)
+    elif w.window is not None:
         oracle.attention_fwd_window(q, k, v, w.window[0], w.window[1], w.scale)
         if w.backward:
             oracle.attention_bwd_window(q, k, v, do, w.window[0], w.window[1], w.scale)
@@ -219,7 +227,207 @@ def _config(w, world):
                f"{4 * w.B * w.Hq * w.N * w.d * 2 / 1e6:.0f} MB vs 126 MB); no flush"}
     if w.window is not None:
         c["window"] = list(w.window)
+    if w.dropout_p:
+        c["dropout_p"] = w.dropout_p
+        c["dropout_seed"] = w.dropout_seed
     return c
+
+
+def _config_varlen(w, world):
+    lens = w.lens()
+    return {"workload": w.name, "sequences_per_gpu": w.n_seqs, "tokens_per_gpu": sum(lens),
+            "longest": max(lens), "mean_len": w.mean_len, "Hq": w.H, "Hkv": w.H, "head_dim": w.d,
+            "causal": w.causal, "passes": "fwd+bwd", "parallelism": f"dp{world}",
+            "l2": f"inputs exceed L2 (q, k, v, dO = {4 * sum(lens) * w.H * w.d * 2 / 1e6:.0f} MB vs "
+                  "126 MB); no flush"}
+
+
+def _oracle_varlen_sample(w, n_seqs: int):
+    """fp64 oracle fwd+bwd on the n_seqs shortest sequences; returns (seconds, FLOPs)."""
+    import oracle
+    from exact_io_aware_83_b200.inputs import draw_packed
+    lens = sorted(w.lens())[:n_seqs]
+    q, k, v, do, cq, ck = draw_packed(lens, lens, w.H, w.H, w.d, w.seed)
+    f64 = lambda t: t.float().double().numpy()
+    right = 0 if w.causal else -1
+    t0 = time.perf_counter()
+    oracle.attention_fwd_varlen(f64(q), f64(k), f64(v), cq.numpy(), ck.numpy(), -1, right, w.scale)
+    oracle.attention_bwd_varlen(f64(q), f64(k), f64(v), f64(do), cq.numpy(), ck.numpy(), -1, right,
+                                w.scale)
+    dt = time.perf_counter() - t0
+    pairs = sum(L * (L + 1) // 2 if w.causal else L * L for L in lens)
+    return dt, 3.5 * 4.0 * w.H * w.d * pairs
+
+
+def run_reference_varlen(args, w):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    cores = _cores()
+    oracle.set_threads(cores)
+    t1, f1 = _oracle_varlen_sample(w, 1)
+    budget = 120.0 / (args.steps + args.warmup)
+    # Add the next-shortest sequences while the estimated time (proportional to the
+    # visible pairs, i.e. to the FLOPs) stays within the per-step budget.
+    per_flop = t1 / f1
+    lens = sorted(w.lens())
+    n, cost = 0, 0.0
+    for L in lens:
+        f = 3.5 * 4.0 * w.H * w.d * (L * (L + 1) // 2 if w.causal else L * L)
+        if n > 0 and cost + f * per_flop > budget:
+            break
+        n, cost = n + 1, cost + f * per_flop
+    for _ in range(args.warmup):
+        _oracle_varlen_sample(w, n)
+    tt, tf = 0.0, 0.0
+    for _ in range(args.steps):
+        dt, fl = _oracle_varlen_sample(w, n)
+        tt += dt
+        tf += fl
+    value = tf / tt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": _config_varlen(w, args.gpus),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"the {n} shortest sequences of {w.name}, fp64 oracle fwd+bwd, per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours_varlen(args, w):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_83_b200 import fa
+    from exact_io_aware_83_b200.inputs import draw_packed
+    from exact_io_aware_83_b200.shard import max_over_ranks, rank_seed
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    fa.load()
+    lens = w.lens()
+    host = draw_packed(lens, lens, w.H, w.H, w.d, rank_seed(w.seed, rank))
+    q, k, v, do, cq, ck = (t.cuda() for t in host)
+    mx = max(lens)
+    o = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], w.H), dtype=torch.float32, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_varlen_workspace_bytes(w.H, q.shape[0], w.d), dtype=torch.uint8,
+                     device="cuda")
+
+    def step():
+        fa.fwd_varlen(q, k, v, cq, ck, mx, mx, causal=w.causal, scale=w.scale, out=o, lse=lse)
+        fa.bwd_varlen(q, k, v, o, lse, do, cq, ck, mx, mx, causal=w.causal, scale=w.scale,
+                      workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_device_status(None) != fa.FA_OK:
+        raise SystemExit("device status not clean after warm-up")
+    sampler = ClockSampler(local)
+    time.sleep(0.3)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    fa.fa_kernel_timing(True)
+    sampler.start()
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    fa.fa_kernel_timing(False)
+    ms = max_over_ranks(e0.elapsed_time(e1))
+    fwd_ms, nfwd = fa.fa_kernel_time_ms(0)
+    bwd_ms, nbwd = fa.fa_kernel_time_ms(1)
+    if fa.fa_device_status(None) != fa.FA_OK:
+        raise SystemExit("device status not clean after the timed region")
+    clocks = sampler.summary()
+    step_flops = w.fwd_flops() + w.bwd_flops()
+    value = step_flops * args.steps * world / (ms / 1e3) / 1e12
+
+    pin = lambda t: t.pin_memory()
+    qh, kh, vh, doh = (pin(t) for t in host[:4])
+    outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+
+    def e2e_step():
+        q.copy_(qh, non_blocking=True)
+        k.copy_(kh, non_blocking=True)
+        v.copy_(vh, non_blocking=True)
+        do.copy_(doh, non_blocking=True)
+        step()
+        for hst, dev in zip(outs, (o, lse, dq, dk, dv)):
+            hst.copy_(dev, non_blocking=True)
+
+    e2e_steps = max(3, args.steps // 10)
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
+
+    peaks, peak_src = _peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = w.bwd_flops() / (bwd_ms / nbwd / 1e3) / 1e12
+    kernels = {
+        "fa_fwd_kernel": {"ms_per_launch": fwd_ms / nfwd, "tflops": w.fwd_flops() / (fwd_ms / nfwd / 1e3) / 1e12},
+        "fa_bwd_main_kernel": {"ms_per_launch": bwd_ms / nbwd, "tflops": achieved},
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": _config_varlen(w, world),
+        "frac_of_peak": value / world / peak,
+        "roofline": {"bound": "tensor", "kernel": "fa_bwd_main_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": _profile_traffic("fa_bwd_main_kernel", w.name),
+                     "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
+        "kernels": kernels,
+        "e2e": {"value": step_flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
+                "h2d_bytes_per_step": nb(q, k, v, do), "d2h_bytes_per_step": nb(o, lse, dq, dk, dv),
+                "steps": e2e_steps},
+        "gpu_launches": args.steps * 4,
+        "clocks": clocks,
+    }
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        import oracle
+        cores = _cores()
+        oracle.set_threads(cores)
+        dt, fl = _oracle_varlen_sample(w, 2)
+        line["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                "sample": f"the 2 shortest sequences of {w.name}, fp64 oracle fwd+bwd, one pass, {dt:.1f} s wall"}
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
 
 
 def run_ours(args, w):
@@ -253,10 +461,11 @@ def run_ours(args, w):
                      device="cuda")
 
     def step():
-        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, window=w.window)
+        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, window=w.window,
+               dropout_p=w.dropout_p, seed=w.dropout_seed)
         if w.backward:
             fa.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws, dq=dq,
-                   dk=dk, dv=dv, window=w.window)
+                   dk=dk, dv=dv, window=w.window, dropout_p=w.dropout_p, seed=w.dropout_seed)
 
     for _ in range(args.warmup):
         step()
@@ -567,7 +776,12 @@ def main(argv=None):
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    from exact_io_aware_83_b200.inputs import DECODE_WORKLOADS, WORKLOADS
+    from exact_io_aware_83_b200.inputs import DECODE_WORKLOADS, VARLEN_WORKLOADS, WORKLOADS
+    if args.workload in VARLEN_WORKLOADS:
+        w = VARLEN_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            return run_reference_varlen(args, w)
+        return run_ours_varlen(args, w)
     if args.workload in DECODE_WORKLOADS:
         w = DECODE_WORKLOADS[args.workload]
         if args.impl == "reference":

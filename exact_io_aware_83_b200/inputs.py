@@ -20,7 +20,12 @@ window_8k_1k          2   16   16   8192  128  band    fwd+bwd    N(0,1)
 ====================  ==  ===  ===  ====  ===  ======  =========  =====================
 
 window_8k_1k is local attention with the band i - 1023 <= j <= i (1024 keys per row,
-the row's own included).
+the row's own included); dropout_8k_causal is long_8k_causal with attention dropout
+p = 0.1 (Philox4x32-10 mask, seed 8080).
+
+Packed variable-length workload: varlen_32k_ragged, 24 sequences of long-tailed length
+(log-normal around 1500 tokens, clipped to [16, 8192]; 39.7k tokens in all, longest 3867), 16 heads,
+d = 128, causal, forward and backward.
 
 Decode workloads (a few new query rows against a key/value cache; K/V N(0,1)):
 
@@ -52,6 +57,8 @@ class Workload:
     q_std: float
     seed: int
     window: tuple | None = None   # (left, right) key band, -1 = unlimited; None: causal flag
+    dropout_p: float = 0.0        # attention dropout probability (0: none)
+    dropout_seed: int = 0
 
     @property
     def scale(self) -> float:
@@ -87,7 +94,40 @@ WORKLOADS = {
         Workload("gqa_4k_causal_fwd", 4, 32, 8, 4096, 128, True, False, 1.0, 4),
         Workload("d256_4k_stress", 2, 8, 8, 4096, 256, False, True, 4.0, 5),
         Workload("window_8k_1k", 2, 16, 16, 8192, 128, False, True, 1.0, 6, (1023, 0)),
+        Workload("dropout_8k_causal", 2, 16, 16, 8192, 128, True, True, 1.0, 9, None, 0.1, 8080),
     )
+}
+
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    name: str
+    n_seqs: int
+    mean_len: int
+    H: int
+    d: int
+    causal: bool
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
+
+    def lens(self):
+        return packed_lengths(self.n_seqs, self.mean_len, self.seed)
+
+    def fwd_flops(self) -> float:
+        """4 H d per visible (query, key) pair of every sequence."""
+        pairs = sum(L * (L + 1) // 2 if self.causal else L * L for L in self.lens())
+        return 4.0 * self.H * self.d * pairs
+
+    def bwd_flops(self) -> float:
+        return 2.5 * self.fwd_flops()
+
+
+VARLEN_WORKLOADS = {
+    w.name: w
+    for w in (VarlenWorkload("varlen_32k_ragged", 24, 1500, 16, 128, True, 31),)
 }
 
 
