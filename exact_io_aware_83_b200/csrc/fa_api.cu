@@ -711,10 +711,12 @@ int fa_decode_num_splits(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
     (void)cudaGetLastError();
     sms = 148;
   }
-  // One CTA per SM: as many splits as fit into one wave of (b, K/V head) units, but at
-  // least two 128-key blocks per split so each CTA streams a few blocks.
+  // As many splits as fit into one wave of (b, K/V head) units - one CTA per SM, or two
+  // for the variants with up to 16 query rows per K/V head and d = 64 - but at least two 128-key
+  // blocks per split so each CTA streams a few blocks.
+  const int slots = sms * (decode_rows_padded((Hq / Hkv) * Nq) == 16 && d == 64 ? 2 : 1);
   const long long units = static_cast<long long>(B) * Hkv;
-  long long s = units >= sms ? 1 : sms / units;
+  long long s = units >= slots ? 1 : slots / units;
   const long long blocks = (Nk + 127) / 128;
   const long long max_by_len = blocks / 2 > 1 ? blocks / 2 : 1;
   if (s > max_by_len) s = max_by_len;

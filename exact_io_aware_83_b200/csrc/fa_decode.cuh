@@ -78,7 +78,13 @@ struct DecodeLayout {
   static constexpr int kVecBytes = 6 * RP * 4;       // red[4][RP] | mu[RP] | al[RP]
   static constexpr int kNumBarsMax = 8 + 2 * 8;
   static constexpr int kFixed = kQBytes + 2 * kPBytes + kOnesBytes + kPad + kVecBytes + kNumBarsMax * 8 + 16;
-  static constexpr int kSlotsFit = (232448 - 1024 - kFixed) / kKVTile;
+  // Up to 16 query rows and d = 64, two CTAs share an SM (each with half the shared
+  // memory): the softmax of one block is a serial chain (load, max exchange,
+  // exponentials, P store), and a second CTA's chain hides it when a block carries few
+  // bytes (d = 64).
+  static constexpr int kCtasPerSM = (RP == 16 && D == 64) ? 2 : 1;
+  static constexpr int kSmemBudget = (kCtasPerSM == 2) ? 232448 / 2 - 1024 : 232448;
+  static constexpr int kSlotsFit = (kSmemBudget - 1024 - kFixed) / kKVTile;
   static constexpr int kSlots = kSlotsFit > 8 ? 8 : kSlotsFit;
   static constexpr int kOffKV = 0;
   static constexpr int kOffPad = kOffKV + kSlots * kKVTile;
@@ -108,7 +114,7 @@ struct DecodeLayout {
   static_assert((3 + kNH) * RP <= 512, "tensor-memory budget");
   static_assert(kSlots >= 2, "K/V ring");
   static_assert(kNumBars <= kNumBarsMax, "barrier budget");
-  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(kSmemBytes <= kSmemBudget, "shared-memory budget");
 };
 
 // Warp 0: TMA loads; warp 1: TMEM allocation and MMA issue; warps 2-5: softmax (one key
@@ -126,7 +132,7 @@ __device__ __forceinline__ void st_shared_u16(uint32_t addr, uint16_t v) {
 }
 
 template <int D, int RP>
-__global__ void __launch_bounds__(kDecodeThreads, 1)
+__global__ void __launch_bounds__(kDecodeThreads, DecodeLayout<D, RP>::kCtasPerSM)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using L = DecodeLayout<D, RP>;

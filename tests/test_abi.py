@@ -186,11 +186,14 @@ def test_decode_workspace_and_splits():
     assert fa.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, 5) == pad(5 * rows * d * 4) + pad(5 * rows * 4)
     assert fa.fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d, 0) == 0
     assert fa.fa_decode_workspace_bytes(B, Hq, 3, Nq, Nk, d, 2) == 0
-    # Without a device the split choice assumes 148 SMs: 4 units -> 37 splits, capped by
-    # the 8 key blocks (at least two per split) -> 4.
+    # Without a device the split choice assumes 148 SMs (one CTA each): 4 units -> 37
+    # splits, capped by the 8 key blocks (at least two per split) -> 4.
     assert fa.fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d) == 4
     assert fa.fa_decode_num_splits(B, Hq, Hkv, Nq, 1 << 20, d) == 37
     assert fa.fa_decode_num_splits(64, Hq, Hkv, Nq, 1 << 20, d) == 1
+    # d = 64 with up to 16 query rows per K/V head runs two CTAs per SM (296 slots).
+    assert fa.fa_decode_num_splits(B, Hq, Hkv, Nq, 1 << 20, 64) == 74
+    assert fa.fa_decode_num_splits(B, 16, 2, 5, 1 << 20, 64) == 37
     assert fa.fa_decode_num_splits(B, Hq, 3, Nq, Nk, d) == 0
 
 
