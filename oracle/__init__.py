@@ -8,7 +8,7 @@ Every function takes and returns numpy float64 arrays in the ``[B, H, N, d]`` la
 
 Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy example
 of the "Consideration"/FlashAttention article page, finite differences and invariants):
-``oracle_fwd``, ``oracle_bwd``, their key-window, variable-length and dropout forms,
+``oracle_fwd``, ``oracle_bwd``, their key-window, variable-length, block-sparse and dropout forms,
 ``oracle_decode``, ``oracle_merge`` and ``online_softmax_stats`` all have pins; none is
 "parity unpinned".  The dropout generator itself (Philox4x32-10) is pinned by statistics
 (keep rate, uniformity, independence), not by known-answer vectors.
@@ -65,6 +65,12 @@ def _lib():
         lib.oracle_bwd_dropout.argtypes = [dp, dp, dp, dp, dp, dp, dp, ci, ci, ci, ci, ci, ci,
                                            ctypes.c_double, ctypes.c_double, u64]
         lib.oracle_bwd_dropout.restype = ci
+        lib.oracle_fwd_blocksparse.argtypes = [dp, dp, dp, u8p, dp, dp, ci, ci, ci, ci, ci, ci,
+                                               ctypes.c_double]
+        lib.oracle_fwd_blocksparse.restype = ci
+        lib.oracle_bwd_blocksparse.argtypes = [dp, dp, dp, dp, u8p, dp, dp, dp, ci, ci, ci, ci,
+                                               ci, ci, ctypes.c_double]
+        lib.oracle_bwd_blocksparse.restype = ci
         lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
         lib.oracle_online_softmax_stats.restype = ci
         _LIB = lib
@@ -261,6 +267,43 @@ def attention_bwd_dropout(q, k, v, dout, causal: bool, scale: float, p: float, s
                                    float(p), int(seed) & 0xFFFFFFFFFFFFFFFF)
     if rc != 0:
         raise RuntimeError(f"oracle_bwd_dropout failed with {rc}")
+    return dq, dk, dv
+
+
+def _bmask(bmask, B, Hq, N):
+    nb = (N + 127) // 128
+    m = np.ascontiguousarray(np.asarray(bmask, dtype=np.uint8))
+    if m.shape != (B, Hq, nb, nb):
+        raise ValueError(f"block mask must be [B, Hq, {nb}, {nb}]")
+    return m, m.ctypes.data_as(ctypes.POINTER(ctypes.c_ubyte))
+
+
+def attention_fwd_blocksparse(q, k, v, bmask, causal: bool, scale: float):
+    """Attention restricted to the enabled 128 x 128 blocks of bmask [B, Hq, nb, nb]
+    (and to j <= i with causal).  Rows without keys: O = 0, LSE = -inf."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    m, mp = _bmask(bmask, B, Hq, N)
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N), dtype=np.float64)
+    rc = _lib().oracle_fwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), mp, _ptr(o), _ptr(lse), B, Hq,
+                                       Hkv, N, d, int(bool(causal)), float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_fwd_blocksparse failed with {rc}")
+    return o, lse
+
+
+def attention_bwd_blocksparse(q, k, v, dout, bmask, causal: bool, scale: float):
+    """dq, dk, dv of <O, dO> for block-sparse attention."""
+    q, k, v, dout = _as_f64(q), _as_f64(k), _as_f64(v), _as_f64(dout)
+    B, Hq, Hkv, N, d = _shapes(q, k)
+    m, mp = _bmask(bmask, B, Hq, N)
+    dq, dk, dv = np.empty_like(q), np.empty_like(k), np.empty_like(v)
+    rc = _lib().oracle_bwd_blocksparse(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), mp, _ptr(dq),
+                                       _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, int(bool(causal)),
+                                       float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bwd_blocksparse failed with {rc}")
     return dq, dk, dv
 
 

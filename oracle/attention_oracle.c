@@ -749,3 +749,135 @@ int oracle_bwd_dropout(const double *q, const double *k, const double *v, const 
     free(Dv);
     return 0;
 }
+
+/*
+ * Block-sparse attention: the deep-dive page closes by naming block-sparse FlashAttention
+ * without defining it.  The reading here: a 0/1 mask over 128 x 128 blocks of the score
+ * matrix of each query head, bmask[b][h][i / 128][j / 128] (nb = ceil(N / 128) blocks per
+ * side), so key j is visible to query i iff its block is enabled (and, with `causal`,
+ * j <= i).  A row that sees no key gets O = 0 and LSE = -inf.
+ */
+static int block_visible(const unsigned char *bmask, int nb, long long bh, int i, int j, int causal)
+{
+    if (causal && j > i) return 0;
+    return bmask[((size_t)bh * nb + (size_t)(i / 128)) * nb + (size_t)(j / 128)] != 0;
+}
+
+int oracle_fwd_blocksparse(const double *q, const double *k, const double *v,
+                           const unsigned char *bmask, double *o, double *lse, int B, int Hq,
+                           int Hkv, int N, int d, int causal, double scale)
+{
+    if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !bmask || !o || !lse) return -1;
+    const int g = Hq / Hkv, nb = (N + 127) / 128;
+    const long long rows = (long long)B * Hq * N;
+    int fail = 0;
+#pragma omp parallel reduction(|: fail)
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)N);
+        int *idx = (int *)malloc(sizeof(int) * (size_t)N);
+        if (!s || !idx) {
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 16)
+            for (long long r = 0; r < rows; ++r) {
+                const int i = (int)(r % N);
+                const long long bh = r / N;
+                const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+                const double *kh = k + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+                const double *vh = v + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+                double *oi = o + (size_t)r * d;
+                for (int c = 0; c < d; ++c) oi[c] = 0.0;
+                int n = 0;
+                double m = -INFINITY;
+                for (int j = 0; j < N; ++j) {
+                    if (!block_visible(bmask, nb, bh, i, j, causal)) continue;
+                    idx[n] = j;
+                    s[n] = scale * dotd(q + (size_t)r * d, kh + (size_t)j * d, d);
+                    if (s[n] > m) m = s[n];
+                    ++n;
+                }
+                if (n == 0) {
+                    lse[r] = -INFINITY;
+                    continue;
+                }
+                double l = 0.0;
+                for (int t = 0; t < n; ++t) l += exp(s[t] - m);
+                const double L = m + log(l);
+                for (int t = 0; t < n; ++t) {
+                    const double p = exp(s[t] - L);
+                    const double *vj = vh + (size_t)idx[t] * d;
+                    for (int c = 0; c < d; ++c) oi[c] += p * vj[c];
+                }
+                lse[r] = L;
+            }
+        }
+        free(s);
+        free(idx);
+    }
+    return fail ? -2 : 0;
+}
+
+/* Gradient of <O, dO> for block-sparse attention (same mask and causal flag). */
+int oracle_bwd_blocksparse(const double *q, const double *k, const double *v, const double *dout,
+                           const unsigned char *bmask, double *dq, double *dk, double *dv, int B,
+                           int Hq, int Hkv, int N, int d, int causal, double scale)
+{
+    if (check_args(B, Hq, Hkv, N, d) || !q || !k || !v || !dout || !bmask || !dq || !dk || !dv)
+        return -1;
+    const int g = Hq / Hkv, nb = (N + 127) / 128;
+    const long long qrows = (long long)B * Hq * N;
+    double *Lv = (double *)malloc(sizeof(double) * (size_t)qrows);
+    double *Dv = (double *)malloc(sizeof(double) * (size_t)qrows);
+    double *o = (double *)malloc(sizeof(double) * (size_t)qrows * d);
+    if (!Lv || !Dv || !o) { free(Lv); free(Dv); free(o); return -2; }
+    int rc = oracle_fwd_blocksparse(q, k, v, bmask, o, Lv, B, Hq, Hkv, N, d, causal, scale);
+    if (rc) { free(Lv); free(Dv); free(o); return rc; }
+    /* Delta_i = <dO_i, O_i>; rows without keys have O = 0, so Delta = 0. */
+    for (long long r = 0; r < qrows; ++r) Dv[r] = dotd(dout + (size_t)r * d, o + (size_t)r * d, d);
+    free(o);
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long r = 0; r < qrows; ++r) {
+        const int i = (int)(r % N);
+        const long long bh = r / N;
+        const int b = (int)(bh / Hq), h = (int)(bh % Hq);
+        const double *kh = k + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+        const double *vh = v + ((size_t)b * Hkv + h / g) * (size_t)N * d;
+        double *dqi = dq + (size_t)r * d;
+        for (int c = 0; c < d; ++c) dqi[c] = 0.0;
+        for (int j = 0; j < N; ++j) {
+            if (!block_visible(bmask, nb, bh, i, j, causal)) continue;
+            const double P = exp(scale * dotd(q + (size_t)r * d, kh + (size_t)j * d, d) - Lv[r]);
+            const double dS = P * (dotd(dout + (size_t)r * d, vh + (size_t)j * d, d) - Dv[r]);
+            for (int c = 0; c < d; ++c) dqi[c] += dS * kh[(size_t)j * d + c];
+        }
+        for (int c = 0; c < d; ++c) dqi[c] *= scale;
+    }
+    const long long krows = (long long)B * Hkv * N;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (long long r = 0; r < krows; ++r) {
+        const int j = (int)(r % N);
+        const long long bk = r / N;
+        const int kvh = (int)(bk % Hkv), b = (int)(bk / Hkv);
+        const double *kj = k + (size_t)r * d, *vj = v + (size_t)r * d;
+        double *dkj = dk + (size_t)r * d, *dvj = dv + (size_t)r * d;
+        for (int c = 0; c < d; ++c) { dkj[c] = 0.0; dvj[c] = 0.0; }
+        for (int h = kvh * g; h < (kvh + 1) * g; ++h) {
+            const long long bh = (long long)b * Hq + h;
+            for (int i = 0; i < N; ++i) {
+                if (!block_visible(bmask, nb, bh, i, j, causal)) continue;
+                const size_t qr = (size_t)bh * N + i;
+                const double *qi = q + qr * d, *doi = dout + qr * d;
+                const double P = exp(scale * dotd(qi, kj, d) - Lv[qr]);
+                const double dS = P * (dotd(doi, vj, d) - Dv[qr]);
+                for (int c = 0; c < d; ++c) {
+                    dvj[c] += P * doi[c];
+                    dkj[c] += dS * qi[c];
+                }
+            }
+        }
+        for (int c = 0; c < d; ++c) dkj[c] *= scale;
+    }
+    free(Lv);
+    free(Dv);
+    return 0;
+}

@@ -23,6 +23,9 @@ the causal mask on the wrong side, a missing scale) fails at least one test:
 * packed variable-length batches against the dense oracle per sequence (equal lengths),
   the decode oracle per sequence (unequal lengths, bottom-right band), a brute-force
   masked softmax for banded windows, and central finite differences;
+* block-sparse: an all-ones mask is dense attention, a block-diagonal mask is independent
+  chunks, random masks (with an empty block row) equal a brute-force masked softmax, and
+  central finite differences;
 * dropout: p = 0 is plain attention, the forward equals the reweighted masked softmax
   built from the keep mask, it is unbiased over seeds, its gradient matches central
   differences, and the keep mask has the right rate for six p and no visible correlation
@@ -761,3 +764,80 @@ def test_dropout_gradients_match_central_differences():
                 args_m[which][idx] -= eps
                 num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
             np.testing.assert_allclose(g, num, rtol=1e-6, atol=1e-7)
+
+
+# ---------------------------------------------------------------------------- block-sparse
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blocksparse_all_ones_is_dense_attention(causal):
+    r = _rng(103)
+    q, k, v = r.normal(size=(1, 2, 300, 4)), r.normal(size=(1, 1, 300, 4)), r.normal(size=(1, 1, 300, 4))
+    ones = np.ones((1, 2, 3, 3), dtype=np.uint8)
+    o1, l1 = oracle.attention_fwd_blocksparse(q, k, v, ones, causal, 0.5)
+    o2, l2 = oracle.attention_fwd(q, k, v, causal, 0.5)
+    np.testing.assert_allclose(o1, o2, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-13)
+    # Blocks above the diagonal do not matter under the causal mask.
+    tril = np.tril(np.ones((3, 3), dtype=np.uint8))[None, None].repeat(2, axis=1)
+    if causal:
+        o3, l3 = oracle.attention_fwd_blocksparse(q, k, v, tril, True, 0.5)
+        np.testing.assert_array_equal(o3, o1)
+        np.testing.assert_array_equal(l3, l1)
+
+
+def test_blocksparse_block_diagonal_is_independent_chunks():
+    # Only diagonal blocks: each 128-row chunk attends to itself alone.
+    r = _rng(107)
+    q, k, v = r.normal(size=(1, 1, 300, 3)), r.normal(size=(1, 1, 300, 3)), r.normal(size=(1, 1, 300, 3))
+    diag = np.eye(3, dtype=np.uint8)[None, None]
+    o, lse = oracle.attention_fwd_blocksparse(q, k, v, diag, False, 0.7)
+    for c0, c1 in ((0, 128), (128, 256), (256, 300)):
+        o_c, l_c = oracle.attention_fwd(q[:, :, c0:c1], k[:, :, c0:c1], v[:, :, c0:c1], False, 0.7)
+        np.testing.assert_allclose(o[:, :, c0:c1], o_c, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, :, c0:c1], l_c, rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blocksparse_equals_masked_softmax(causal):
+    r = _rng(109 + causal)
+    N = 300
+    q, k, v = r.normal(size=(1, 2, N, 3)), r.normal(size=(1, 1, N, 3)), r.normal(size=(1, 1, N, 3))
+    bm = (r.random(size=(1, 2, 3, 3)) < 0.5).astype(np.uint8)
+    bm[0, 1, 1, :] = 0           # a block row with no keys: rows 128..255 of head 1 see nothing
+    bm[0, 0, :, 0] = 1
+    o, lse = oracle.attention_fwd_blocksparse(q, k, v, bm, causal, 0.6)
+    i = np.arange(N)[:, None]
+    j = np.arange(N)[None, :]
+    for h in range(2):
+        vis = bm[0, h][i // 128, j // 128].astype(bool)
+        if causal:
+            vis &= j <= i
+        s = np.where(vis, 0.6 * q[0, h] @ k[0, 0].T, -np.inf)
+        for t in range(N):
+            if not vis[t].any():
+                assert np.isneginf(lse[0, h, t]) and np.all(o[0, h, t] == 0)
+                continue
+            L = scipy.special.logsumexp(s[t])
+            assert abs(lse[0, h, t] - L) < 1e-12
+            np.testing.assert_allclose(o[0, h, t], np.exp(s[t] - L) @ v[0, 0], rtol=0, atol=1e-12)
+
+
+def test_blocksparse_gradients_match_central_differences():
+    r = _rng(113)
+    N = 140
+    q, k, v, do = (r.normal(size=(1, 1, N, 2)) for _ in range(4))
+    bm = np.array([[[[1, 0], [1, 1]]]], dtype=np.uint8)
+    dq, dk, dv = oracle.attention_bwd_blocksparse(q, k, v, do, bm, False, 0.9)
+    loss = lambda q_, k_, v_: float((oracle.attention_fwd_blocksparse(q_, k_, v_, bm, False, 0.9)[0] * do).sum())
+    eps = 1e-6
+    rng = np.random.default_rng(0)
+    for x, g, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        # a sample of entries from both block rows and both block columns
+        for n in list(rng.integers(0, N, 6)) + [0, 127, 128, N - 1]:
+            for c in range(2):
+                args_p = [q.copy(), k.copy(), v.copy()]
+                args_m = [q.copy(), k.copy(), v.copy()]
+                args_p[which][0, 0, n, c] += eps
+                args_m[which][0, 0, n, c] -= eps
+                num = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+                assert abs(g[0, 0, n, c] - num) <= 1e-6 * max(1.0, abs(num)), (which, n, c)
