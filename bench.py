@@ -11,7 +11,8 @@ counts 4 d flop per visible (query, key) pair.
 
 --workload varlen_32k_ragged times fa_fwd_varlen + fa_bwd_varlen over a packed batch of
 ragged sequences (FLOPs of the visible pairs of each sequence); dropout_8k_causal times
-the dropout forward and backward.
+the dropout forward and backward; blocksparse_8k_causal times the block-sparse forward and
+backward (FLOPs of the pairs of the enabled blocks).
 
 Decode workloads (--workload decode_*) time one fa_decode call per step (new query rows
 against a resident key/value cache, split over the cache and merged); their metric is
@@ -152,8 +153,15 @@ def _oracle_sample(w, heads: int, seed: int):
     q, k, v, do = draw(1, groups * g, groups, w.N, w.d, seed, w.q_std)
     f64 = lambda t: t.float().double().numpy()
     q, k, v, do = f64(q), f64(k), f64(v), f64(do)
+    bm = w.block_mask()
+    if bm is not None:
+        bm = bm[:1, :groups * g].contiguous()
     t0 = time.perf_counter()
-    if w.dropout_p:
+    if bm is not None:
+        oracle.attention_fwd_blocksparse(q, k, v, bm.numpy(), w.causal, w.scale)
+        if w.backward:
+            oracle.attention_bwd_blocksparse(q, k, v, do, bm.numpy(), w.causal, w.scale)
+    elif w.dropout_p:
         oracle.attention_fwd_dropout(q, k, v, w.causal, w.scale, w.dropout_p, w.dropout_seed)
         if w.backward:
             oracle.attention_bwd_dropout(q, k, v, do, w.causal, w.scale, w.dropout_p, w.dropout_seed)
@@ -167,6 +175,9 @@ def _oracle_sample(w, heads: int, seed: int):
             oracle.attention_bwd(q, k, v, do, w.causal, w.scale)
     dt = time.perf_counter() - t0
     flops = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) * (groups * g) / (w.B * w.Hq)
+    if bm is not None:  # the sampled heads' own mask
+        from exact_io_aware_83_b200.inputs import blocksparse_pairs
+        flops = 4.0 * blocksparse_pairs(bm, w.N, w.causal) * w.d * (3.5 if w.backward else 1.0)
     return dt, flops
 
 
@@ -230,6 +241,11 @@ def _config(w, world):
     if w.dropout_p:
         c["dropout_p"] = w.dropout_p
         c["dropout_seed"] = w.dropout_seed
+    if w.block_density:
+        c["block_mask"] = {"block": 128, "density": w.block_density, "diagonal": True,
+                           "mask_seed": w.mask_seed,
+                           "enabled_pairs_share_of_causal": round(
+                               w.fwd_flops() / (2.0 * w.B * w.Hq * w.N * w.N * w.d), 4)}
     return c
 
 
@@ -459,13 +475,16 @@ def run_ours(args, w):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8,
                      device="cuda")
+    bmh = w.block_mask()
+    bmd = None if bmh is None else bmh.cuda()
 
     def step():
         fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, window=w.window,
-               dropout_p=w.dropout_p, seed=w.dropout_seed)
+               dropout_p=w.dropout_p, seed=w.dropout_seed, block_mask=bmd)
         if w.backward:
             fa.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws, dq=dq,
-                   dk=dk, dv=dv, window=w.window, dropout_p=w.dropout_p, seed=w.dropout_seed)
+                   dk=dk, dv=dv, window=w.window, dropout_p=w.dropout_p, seed=w.dropout_seed,
+                   block_mask=bmd)
 
     for _ in range(args.warmup):
         step()
@@ -504,6 +523,7 @@ def run_ours(args, w):
     # ---- end to end through the public API: pinned host inputs in, results back to host
     pin = lambda t: t.pin_memory()
     qh_p, kh_p, vh_p, doh_p = (pin(t) for t in (qh, kh, vh, doh))
+    bmh_p = None if bmh is None else pin(bmh)
     oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     dqh = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
@@ -516,6 +536,8 @@ def run_ours(args, w):
         v.copy_(vh_p, non_blocking=True)
         if w.backward:
             do.copy_(doh_p, non_blocking=True)
+        if bmd is not None:
+            bmd.copy_(bmh_p, non_blocking=True)
         step()
         oh.copy_(o, non_blocking=True)
         lseh.copy_(lse, non_blocking=True)
@@ -538,6 +560,8 @@ def run_ours(args, w):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1))
     nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
     h2d = nbytes(q, k, v, do) if w.backward else nbytes(q, k, v)
+    if bmd is not None:
+        h2d += nbytes(bmd)
     d2h = nbytes(o, lse, dq, dk, dv) if w.backward else nbytes(o, lse)
     e2e_value = step_flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12
 

@@ -111,6 +111,15 @@ bool device_ready() {
     ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnFull>, fa::FwdLayout<128>::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnCausal>, fa::FwdLayout<128>::kSmemBytes);
     ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnGeneral>, fa::FwdLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_kernel<64, fa::kAttnSparse>, fa::FwdLayout<64>::kSmemBytesSparse);
+    ok = ok && set_smem(fa::fa_fwd_kernel<128, fa::kAttnSparse>, fa::FwdLayout<128>::kSmemBytesSparse);
+    ok = ok && set_smem(fa::fa_fwd_d256_kernel<fa::kAttnSparse>, fa::FwdD256Layout::kSmemBytesSparse);
+    ok = ok && set_smem(fa::fa_bwd_main_kernel<64, 64, 64, fa::kAttnSparse>,
+                        fa::BwdLayout<64, 64, 64>::kSmemBytesSparse);
+    ok = ok && set_smem(fa::fa_bwd_main_kernel<128, 128, 64, fa::kAttnSparse>,
+                        fa::BwdLayout<128, 128, 64>::kSmemBytesSparse);
+    ok = ok && set_smem(fa::fa_bwd_main_kernel<256, 128, 32, fa::kAttnSparse>,
+                        fa::BwdLayout<256, 128, 32>::kSmemBytesSparse);
     ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnFull>, fa::kFwdRegsLaunch);
     ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnCausal>, fa::kFwdRegsLaunch);
     ok = ok && regs_at_least(fa::fa_fwd_kernel<64, fa::kAttnGeneral>, fa::kFwdRegsLaunch);
@@ -329,11 +338,15 @@ void launch_merge(const float *o_part, const float *lse_part, void *o, float *ls
 template <int D, int MODE, bool DROP>
 void launch_fwd_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
                   const FwdParams &p, unsigned units, cudaStream_t s) {
+  constexpr bool sparse = MODE == fa::kAttnSparse;
   if constexpr (D == 256)
-    fa::fa_fwd_d256_kernel<MODE, DROP><<<units, fa::kFwdD256Threads, fa::FwdD256Layout::kSmemBytes, s>>>(
-        tq, tk, tv, to, p);
+    fa::fa_fwd_d256_kernel<MODE, DROP><<<units, fa::kFwdD256Threads,
+                                         sparse ? fa::FwdD256Layout::kSmemBytesSparse : fa::FwdD256Layout::kSmemBytes,
+                                         s>>>(tq, tk, tv, to, p);
   else
-    fa::fa_fwd_kernel<D, MODE, DROP><<<units, fa::kFwdThreads, fa::FwdLayout<D>::kSmemBytes, s>>>(tq, tk, tv, to, p);
+    fa::fa_fwd_kernel<D, MODE, DROP><<<units, fa::kFwdThreads,
+                                       sparse ? fa::FwdLayout<D>::kSmemBytesSparse : fa::FwdLayout<D>::kSmemBytes,
+                                       s>>>(tq, tk, tv, to, p);
 }
 
 template <int D>
@@ -342,6 +355,7 @@ void launch_fwd_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtenso
   if (drop && mode == fa::kAttnCausal) launch_fwd_d<D, fa::kAttnCausal, true>(tq, tk, tv, to, p, units, s);
   else if (drop) launch_fwd_d<D, fa::kAttnFull, true>(tq, tk, tv, to, p, units, s);
   else if (mode == fa::kAttnGeneral) launch_fwd_d<D, fa::kAttnGeneral, false>(tq, tk, tv, to, p, units, s);
+  else if (mode == fa::kAttnSparse) launch_fwd_d<D, fa::kAttnSparse, false>(tq, tk, tv, to, p, units, s);
   else if (mode == fa::kAttnCausal) launch_fwd_d<D, fa::kAttnCausal, false>(tq, tk, tv, to, p, units, s);
   else launch_fwd_d<D, fa::kAttnFull, false>(tq, tk, tv, to, p, units, s);
 }
@@ -352,6 +366,7 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
                FwdParams &p, int d, int mode, cudaStream_t s, const fa::DropCfg *drop = nullptr) {
   const int g = p.Hq / p.Hkv;
   p.drop = drop ? *drop : fa::DropCfg{};
+  if (mode != fa::kAttnSparse) p.bmask = nullptr;
   const int tslot = timer_start(0, s);
   if (d == 256) {
     p.pair_heads = 0;
@@ -407,11 +422,25 @@ bool normalise_window_varlen(int w, int max_q, int max_k, int *out) {
   return true;
 }
 
+// Block-sparse limits: the forward keeps each CTA's key-block list in shared memory (at most
+// 4096 blocks of 128 keys), the backward a bitmap of g x ceil(nb / 32) words.
+int check_blocksparse(const unsigned char *mask, int Hq, int Hkv, int N, int d, int causal) {
+  if (!mask || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  const long long nb = (N + 127) / 128;
+  if (nb > fa::kMaxSparseBlocks) return FA_ERR_UNSUPPORTED;
+  const long long words = static_cast<long long>(Hq / Hkv) * ((nb + 31) / 32);
+  const int cap = d == 64 ? fa::BwdLayout<64, 64, 64>::kSparseBitmapBytes
+                  : d == 128 ? fa::BwdLayout<128, 128, 64>::kSparseBitmapBytes
+                             : fa::BwdLayout<256, 128, 32>::kSparseBitmapBytes;
+  if (words * 4 > cap) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
 }  // namespace
 
 extern "C" {
 
-int fa_version(void) { return 101; }
+int fa_version(void) { return 102; }
 
 const char *fa_status_string(int code) {
   switch (code) {
@@ -652,6 +681,59 @@ int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, c
   // N = 1 with causal is full attention (normalise_window's rule); the mask is the same.
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
                         static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop, nullptr, &drop);
+}
+
+int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                       const unsigned char *block_mask, int B, int Hq, int Hkv, int N, int d, int causal,
+                       float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  rc = check_blocksparse(block_mask, Hq, Hkv, N, d, causal);
+  if (rc != FA_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  const int kv_rows = d == 256 ? 64 : 128;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_map_bf16(&tq, q, d, N, static_cast<long long>(B) * Hq, 128) ||
+      !make_map_bf16(&tk, k, d, N, static_cast<long long>(B) * Hkv, kv_rows) ||
+      !make_map_bf16(&tv, v, d, N, static_cast<long long>(B) * Hkv, kv_rows) ||
+      !make_map_bf16(&to, o, d, N, static_cast<long long>(B) * Hq, 128))
+    return FA_ERR_CUDA;
+  FwdParams p;
+  p.lse = lse;
+  p.o = static_cast<__nv_bfloat16 *>(o);
+  p.cu_q = p.cu_k = nullptr;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.total_q = p.total_k = 0;
+  p.nqb = (N + 127) / 128;
+  p.left = -1;
+  p.right = causal ? 0 : -1;  // the kernel reads causality from right == 0
+  p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.bmask = block_mask;
+  return launch_fwd(tq, tk, tv, to, p, d, fa::kAttnSparse, static_cast<cudaStream_t>(stream));
+}
+
+int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                       const void *dout, void *dq, void *dk, void *dv, void *workspace, size_t workspace_bytes,
+                       const unsigned char *block_mask, int B, int Hq, int Hkv, int N, int d, int causal,
+                       float scale, void *stream) {
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  int rc = check_sizes(B, Hq, Hkv, N, d, scale);
+  if (rc != FA_OK) return rc;
+  rc = check_blocksparse(block_mask, Hq, Hkv, N, d, causal);
+  if (rc != FA_OK) return rc;
+  if (!workspace || workspace_bytes < fa::bwd_workspace_bytes(B, Hq, N, d)) return FA_ERR_WORKSPACE;
+  const void *ptrs[] = {q, k, v, o, lse, dout, dq, dk, dv, workspace};
+  for (const void *ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_ALIGN;
+  if (!device_ready()) return FA_ERR_CUDA;
+  return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
+                        static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop, nullptr, nullptr,
+                        block_mask);
 }
 
 int fa_kernel_timing(int enable) {

@@ -106,6 +106,7 @@ struct BwdParams {
   float sl2;              // scale * log2(e)
   float scale;
   DropCfg drop;           // dropout (kernels instantiated with DROP only)
+  const uint8_t *bmask;   // block-sparse: [B, Hq, nkb, nkb] 0/1 over 128 x 128 blocks
 };
 
 // D: head dimension (contraction of S^T and dP^T); DH: output columns owned by a CTA
@@ -149,6 +150,13 @@ struct BwdLayout {
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // Block-sparse variant only: after misc, a 16-byte header (steps counted by each of the
+  // four warps that build it) and a bitmap per query head of the group: bit qb of head hh
+  // is set when 128-row query block qb of that head sees this key block.
+  static constexpr int kOffList = kOffMisc + 16;
+  static constexpr int kSparseBitmapBytes =
+      (232448 - (kOffList + 16 + 1024)) / 4 * 4 < 8192 ? (232448 - (kOffList + 16 + 1024)) / 4 * 4 : 8192;
+  static constexpr int kSmemBytesSparse = kOffList + 16 + kSparseBitmapBytes + 1024;
   // tensor memory: dV | dK | S^T | dP^T | dQ^T
   static constexpr uint32_t kTmDV = 0;
   static constexpr uint32_t kTmDK = DH;
@@ -166,15 +174,60 @@ struct BwdLayout {
     return static_cast<uint32_t>((kk / kKStepsPerHalf) * kHC + (kk % kKStepsPerHalf) * 8);
   }
   static_assert(kTmDQ + BQ <= 512, "tensor-memory budget");
-  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(kSmemBytesSparse <= 232448 && kSparseBitmapBytes >= 256, "shared-memory budget");
   static_assert(BQ == 32 || BQ == 64, "query block");
 };
 
 // Warps 0-7: two elementwise warpgroups; 8-11: dQ drain; 12: MMA; 13: loader.
 constexpr int kBwdThreads = 448;
 
-// Kernel variants (kAttnFull, kAttnCausal, kAttnGeneral, see fa_common.cuh): dense full and
-// dense causal attention, and the general form (packed sequences and/or a key band).
+// Block-sparse backward: the steps of a key-block CTA are (query head hh of the group,
+// BQ-row query block) for every 128-row query block whose bit is set in head hh's bitmap,
+// heads in order, blocks in order, the 128 / BQ sub-blocks of each block in order (the last
+// block of the sequence has only those that start before N).  Each role walks the same
+// sequence with its own cursor.
+struct SparseSteps {
+  const uint32_t *bits;  // [g][W] words
+  int W, g, nqb, nsub, nsub_last;
+  int hh, qb, sub;
+  __device__ __forceinline__ void init(const uint32_t *bits_, int W_, int g_, int nqb_, int nsub_, int nsub_last_) {
+    bits = bits_;
+    W = W_;
+    g = g_;
+    nqb = nqb_;
+    nsub = nsub_;
+    nsub_last = nsub_last_;
+    hh = 0;
+    qb = -1;
+    sub = 0;
+  }
+  // First set bit >= from in head hh's bitmap, or -1.
+  __device__ __forceinline__ int find(int from) const {
+    for (int w = from >> 5; w < W; ++w) {
+      uint32_t u = bits[hh * W + w];
+      if (w == (from >> 5)) u &= ~0u << (from & 31);
+      if (u) return w * 32 + __ffs(u) - 1;
+    }
+    return -1;
+  }
+  // Moves to the next step (the first one on the first call); bounded by the bitmap.
+  __device__ __forceinline__ void next() {
+    if (qb >= 0 && ++sub < (qb == nqb - 1 ? nsub_last : nsub)) return;
+    sub = 0;
+    while (hh < g) {
+      qb = find(qb + 1);
+      if (qb >= 0) return;
+      ++hh;
+      qb = -1;
+    }
+  }
+  template <int BQ>
+  __device__ __forceinline__ int q0() const { return qb * 128 + sub * BQ; }
+};
+
+// Kernel variants (kAttnFull, kAttnCausal, kAttnGeneral, kAttnSparse, see fa_common.cuh):
+// dense full and dense causal attention, the general form (packed sequences and/or a key
+// band), and a 0/1 mask over 128 x 128 blocks (optionally with the causal mask).
 template <int D, int DH, int BQ, int MODE, bool DROP = false>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     fa_bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -229,7 +282,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     q_first = MODE == kAttnCausal ? kv0 / BQ : 0;
     nq = (p.N + BQ - 1) / BQ - q_first;
   }
-  const int T = g * nq;  // steps: (query head of the group, query block)
+  constexpr bool SPARSE = MODE == kAttnSparse;
+  constexpr bool GENLIKE = GEN || SPARSE;  // a key block may see no query at all
+  int T = g * nq;  // steps: (query head of the group, query block); block-sparse: counted below
+  const int spW = (p.nkb + 31) / 32;
+  constexpr int kSub = 128 / BQ;
+  const int spSubLast = (p.N - (p.nkb - 1) * 128 + BQ - 1) / BQ;
+  uint32_t *spbits = reinterpret_cast<uint32_t *>(smem + L::kOffList + 16);
   const int dcol0 = half * DH;  // first output column owned by this CTA
   // TMA coordinates (dimensions 1 and 2): dense maps are [B*H][N][cols], packed [total][H][cols].
   auto q_coords = [&](int hh, int row, int &c1, int &c2) {
@@ -258,13 +317,53 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(smem_u32(misc), L::kTmemCols);
     tmem_relinquish_alloc_permit();
   }
+  if constexpr (SPARSE) {
+    // Warps 8-11 (idle until the first dQ) read this key block's column of the mask for
+    // every head of the group, sixteen independent loads per lane in flight, and write the
+    // bitmaps and their step counts.
+    if (warp >= 8 && warp < 12) {
+      const int wq = warp - 8, nw = g * spW;
+      const int qlo = p.right == 0 ? kb : 0;  // causal: query blocks at or after the diagonal
+      const size_t col0 = static_cast<size_t>(b * p.Hq + kvh * g) * p.nkb * p.nkb + kb;
+      int steps = 0;
+      for (int f0 = wq; f0 < nw; f0 += 4 * 16) {
+        bool v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int fw = f0 + 4 * k;
+          const int hh = fw / spW, qb = (fw - hh * spW) * 32 + lane;
+          v[k] = fw < nw && qb >= qlo && qb < p.nkb &&
+                 p.bmask[col0 + (static_cast<size_t>(hh) * p.nkb + qb) * p.nkb] != 0;
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int fw = f0 + 4 * k;
+          const uint32_t u = __ballot_sync(0xffffffffu, v[k]);
+          if (fw < nw && lane == 0) {
+            spbits[fw] = u;
+            steps += __popc(u) * kSub;
+            // the sequence's last query block has only the sub-blocks that start before N
+            if (fw % spW == spW - 1 && ((u >> ((p.nkb - 1) & 31)) & 1u)) steps -= kSub - spSubLast;
+          }
+        }
+      }
+      if (lane == 0) reinterpret_cast<int *>(smem + L::kOffList)[wq] = steps;
+    }
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = misc[0];
+  if constexpr (SPARSE) {
+    const int *hdr = reinterpret_cast<const int *>(smem + L::kOffList);
+    T = hdr[0] + hdr[1] + hdr[2] + hdr[3];
+  }
 
   auto step_head = [&](int i) { return kvh * g + i / nq; };
   auto step_q0 = [&](int i) { return (q_first + i % nq) * BQ; };
+  // Block-sparse: each role's cursor, moved once per step before (h, q0) are used.
+  SparseSteps cur;
+  if constexpr (SPARSE) cur.init(spbits, spW, g, p.nkb, kSub, spSubLast);
 
   if (warp == 13) {
     // ================================================================ loader
@@ -287,7 +386,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       ok = warp_wait_bounded(bar(L::kBarQEmpty + st), (use & 1) ^ 1, abort_flag,
                              wait_site(3, L::kBarQEmpty + st, i));
       if (!ok) break;
-      const int h = step_head(i), q0 = step_q0(i);
+      if constexpr (SPARSE) cur.next();
+      const int h = SPARSE ? kvh * g + cur.hh : step_head(i), q0 = SPARSE ? cur.q0<BQ>() : step_q0(i);
       if (lane == 0) {
         int c1, c2;
         q_coords(h, q0, c1, c2);
@@ -337,8 +437,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
       };
       bool ok = wait_bounded(bar(L::kBarKV), 0, abort_flag, wait_site(3, L::kBarKV, 0));
-      if (ok && (!GEN || T > 0)) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
-      if (ok && (!GEN || T > 0)) {
+      if (ok && (!GENLIKE || T > 0)) ok = wait_bounded(bar(L::kBarQFull), 0, abort_flag, wait_site(3, L::kBarQFull, 0));
+      if (ok && (!GENLIKE || T > 0)) {
         tc_fence_after_sync();
         issue_st(L::kTmS, sK, sQ);
         tc_commit(bar(L::kBarS));
@@ -412,7 +512,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = true;
     for (int i = 0; ok && i < T; ++i) {
       const int st = i % QS;
-      const int q0 = step_q0(i) + c0;  // first query column of this warpgroup
+      if constexpr (SPARSE) cur.next();
+      const int q0 = (SPARSE ? cur.q0<BQ>() : step_q0(i)) + c0;  // first query column of this warpgroup
       if (!(ok = warp_wait_bounded(bar(L::kBarQFull + st), (i / QS) & 1, abort_flag,
                                    wait_site(3, L::kBarQFull + st, i))))
         break;
@@ -446,7 +547,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           for (int c = 0; c < HC; ++c)
             if (c < c_lo || c > c_hi) pr[c] = 0.f;
         }
-      } else if (MODE == kAttnCausal && q0 < kv) {
+      } else if ((MODE == kAttnCausal || (SPARSE && p.right == 0)) && q0 < kv) {
 #pragma unroll
         for (int c = 0; c < HC; ++c)
           if (q0 + c < kv) pr[c] = 0.f;
@@ -459,7 +560,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if constexpr (DROP) {
         keep = 0u;
         const int m = lane & 7;  // == kv & 7
-        const uint32_t bh = static_cast<uint32_t>(b * p.Hq + step_head(i));
+        const uint32_t bh = static_cast<uint32_t>(b * p.Hq + (SPARSE ? kvh * g + cur.hh : step_head(i)));
 #pragma unroll
         for (int t = 0; t < HC / 8; ++t) {
           uint32_t w[4];
@@ -543,7 +644,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < DH / 32; ++cc) {
         uint32_t o[32];
-        if (!GEN || T > 0) {
+        if (!GENLIKE || T > 0) {
           tmem_ld_x32(tacc + cc * 32, o);
         } else {
 #pragma unroll
@@ -605,7 +706,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kBarDQEmpty));
-      const int h = step_head(i), q0 = step_q0(i);
+      if constexpr (SPARSE) cur.next();
+      const int h = SPARSE ? kvh * g + cur.hh : step_head(i), q0 = SPARSE ? cur.q0<BQ>() : step_q0(i);
 #pragma unroll
       for (int hp = 0; hp < L::kDQHalves; ++hp) {
         // The previous reduce must have finished reading the staging buffer.
@@ -692,8 +794,10 @@ template <int D, int DH, int BQ, int MODE, bool DROP = false>
 inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
                             const CUtensorMap &tdo, const CUtensorMap &tdk, const CUtensorMap &tdv,
                             const CUtensorMap &tdq, const BwdParams &p, unsigned grid, cudaStream_t s) {
-  fa_bwd_main_kernel<D, DH, BQ, MODE, DROP><<<grid, kBwdThreads, BwdLayout<D, DH, BQ>::kSmemBytes, s>>>(
-      tq, tk, tv, tdo, tdk, tdv, tdq, p);
+  using L = BwdLayout<D, DH, BQ>;
+  fa_bwd_main_kernel<D, DH, BQ, MODE, DROP>
+      <<<grid, kBwdThreads, MODE == kAttnSparse ? L::kSmemBytesSparse : L::kSmemBytes, s>>>(tq, tk, tv, tdo, tdk,
+                                                                                           tdv, tdq, p);
 }
 
 typedef int (*TimerStartFn)(int, cudaStream_t);
@@ -703,7 +807,8 @@ template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                         int Hkv, int N, int left, int right, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
-                        TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk, const DropCfg *drop) {
+                        TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk, const DropCfg *drop,
+                        const uint8_t *bmask) {
   const long long rows = pk ? static_cast<long long>(pk->total_q) * Hq : static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
   float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
@@ -749,12 +854,15 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.scale = scale;
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.drop = drop ? *drop : DropCfg{};
+  p.bmask = bmask;
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
   if (grid > 0) {
     // Dense full and causal attention have their own variants; packed sequences and other
     // bands take the general one.
-    if (drop && right == 0)  // dropout: dense attention only (the host checks)
+    if (bmask)  // block-sparse: dense layout, causal or not (right = 0 or -1)
+      bwd_launch_main<D, DH, BQ, kAttnSparse>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
+    else if (drop && right == 0)  // dropout: dense attention only (the host checks)
       bwd_launch_main<D, DH, BQ, kAttnCausal, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
     else if (drop)
       bwd_launch_main<D, DH, BQ, kAttnFull, true>(tq, tk, tv, tdo, tdk, tdv, tdq, p, grid, s);
@@ -778,16 +886,16 @@ inline int bwd_launch(const void *q, const void *k, const void *v, const void *o
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                       int Hkv, int N, int d, int left, int right, float scale, cudaStream_t s, Enc enc,
                       TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk = nullptr,
-                      const DropCfg *drop = nullptr) {
+                      const DropCfg *drop = nullptr, const uint8_t *bmask = nullptr) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
     return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk, drop);
+                                    scale, s, e, tstart, tstop, pk, drop, bmask);
   if (d == 128)
     return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                      scale, s, e, tstart, tstop, pk, drop);
+                                      scale, s, e, tstart, tstop, pk, drop, bmask);
   return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk, drop);
+                                    scale, s, e, tstart, tstop, pk, drop, bmask);
 }
 
 }  // namespace fa

@@ -107,7 +107,9 @@ struct DropCfg {
 // Kernel variants: dense attention over every key, dense causal attention, and the general
 // form (packed variable-length sequences and/or a key band), whose extra bookkeeping the
 // two common dense cases do not pay for.
-constexpr int kAttnFull = 0, kAttnCausal = 1, kAttnGeneral = 2;
+// kAttnSparse: dense layout with a 0/1 mask over 128 x 128 blocks (and optionally the
+// causal mask); only enabled blocks are visited.
+constexpr int kAttnFull = 0, kAttnCausal = 1, kAttnGeneral = 2, kAttnSparse = 3;
 
 // The sequence a CTA works on.  Dense: Lq = Lk = N.  Packed: the lengths of sequence b and
 // its first rows in the packed tensors.  The keys are aligned to the END of the queries:

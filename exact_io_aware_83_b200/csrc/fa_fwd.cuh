@@ -50,6 +50,7 @@ struct FwdParams {
   int left, right;        // key band around the diagonal: [c - left, c + right]; -1 = unlimited
   float sl2;              // scale * log2(e)
   DropCfg drop;           // dropout (kernels instantiated with DROP only)
+  const uint8_t *bmask;   // block-sparse: [B, Hq, nqb, nqb] 0/1 over 128 x 128 blocks
 };
 
 // Blocks of KB keys [lo, hi] that some row q0 .. min(q0 + 127, Lq - 1) of a query tile can
@@ -94,6 +95,9 @@ __device__ __forceinline__ void mask_scores(uint32_t (&s)[NC], int left, int rig
 }
 
 constexpr float kLn2 = 0.693147180559945309f;
+// Longest block-sparse sequence, in 128-key blocks (the per-CTA block list lives in shared
+// memory).
+constexpr int kMaxSparseBlocks = 4096;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units
 
 template <int D>
@@ -117,11 +121,15 @@ struct FwdLayout {
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-B alignment
+  // Block-sparse variant only: after misc, a 16-byte header {steps, blocks of tile 0, blocks
+  // of tile 1} and the CTA's key-block list (uint16: block | tile-0 bit 14 | tile-1 bit 15).
+  static constexpr int kOffList = kOffMisc + 16;
+  static constexpr int kSmemBytesSparse = kOffList + 16 + 2 * kMaxSparseBlocks + 1024;
   static constexpr uint32_t kTmemCols = 512;
   __host__ __device__ static constexpr uint32_t tm_s(int t) { return static_cast<uint32_t>(t) * 128u; }
   __host__ __device__ static constexpr uint32_t tm_o(int t) { return 256u + static_cast<uint32_t>(t * D); }
   static_assert(256 + 2 * D <= 512, "tensor-memory budget");
-  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(kSmemBytesSparse <= 232448, "shared-memory budget");
 };
 
 // Warps 0-7: softmax warpgroups of the two tiles; warp 8: MMA; warp 9: TMA; warps 10-11
@@ -311,6 +319,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   }
   const int kvh = h[0] / g;
   constexpr bool GEN = MODE == kAttnGeneral;
+  constexpr bool SPARSE = MODE == kAttnSparse;
+  constexpr bool GENLIKE = GEN || SPARSE;  // rows may see no key at all
   const bool packed = GEN && p.cu_q != nullptr;
   SeqGeom sg{p.N, p.N, 0, 0, 0};
   // Key blocks: the CTA walks the union [ulo, ulo + nu) of its tiles' ranges (contiguous:
@@ -334,11 +344,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     nblk[0] = has0 ? hi0 - lo0 + 1 : 0;
     a[1] = has1 ? lo1 - ulo : 0;
     nblk[1] = has1 ? hi1 - lo1 + 1 : 0;
-  } else {
+  } else if constexpr (!SPARSE) {
 #pragma unroll
     for (int t = 0; t < 2; ++t) nblk[t] = !valid[t] ? 0 : (MODE == kAttnCausal ? qb[t] + 1 : p.nqb);
     nu = nblk[0] > nblk[1] ? nblk[0] : nblk[1];
   }
+  // Block-sparse: tile t visits the enabled key blocks of its mask row (those up to the
+  // diagonal when causal), in order; the CTA walks the union of the two tiles' lists, which
+  // an idle warp writes to shared memory before the roles start.
+  const uint16_t *blist = reinterpret_cast<const uint16_t *>(smem + L::kOffList + 16);
   // TMA coordinates (dimensions 1 and 2) of a 128-row tile: dense maps are [B*H][N][d],
   // packed maps [total][H][d].
   auto q_coords = [&](int hh, int row, int &c1, int &c2) {
@@ -361,10 +375,49 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tmem_alloc(smem_u32(misc), L::kTmemCols);
     tmem_relinquish_alloc_permit();
   }
+  if constexpr (SPARSE) {
+    if (warp == 10) {
+      const bool causal = p.right == 0;
+      const uint8_t *row[2];
+      int hi[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        row[t] = p.bmask + (static_cast<size_t>(b * p.Hq + h[t]) * p.nqb + qb[t]) * p.nqb;
+        hi[t] = !valid[t] ? -1 : (causal ? qb[t] : p.nqb - 1);
+      }
+      uint16_t *list = reinterpret_cast<uint16_t *>(smem + L::kOffList + 16);
+      int n = 0, c0 = 0, c1 = 0;
+      const int hmax = hi[0] > hi[1] ? hi[0] : hi[1];
+      for (int base0 = 0; base0 <= hmax; base0 += 32) {
+        const int kb = base0 + lane;
+        const bool m0 = kb <= hi[0] && row[0][kb] != 0;
+        const bool m1 = kb <= hi[1] && row[1][kb] != 0;
+        const uint32_t u = __ballot_sync(0xffffffffu, m0 || m1);
+        if (m0 || m1)
+          list[n + __popc(u & ((1u << lane) - 1u))] =
+              static_cast<uint16_t>(kb | (m0 ? 1 << 14 : 0) | (m1 ? 1 << 15 : 0));
+        n += __popc(u);
+        c0 += __popc(__ballot_sync(0xffffffffu, m0));
+        c1 += __popc(__ballot_sync(0xffffffffu, m1));
+      }
+      if (lane == 0) {
+        int *hdr = reinterpret_cast<int *>(smem + L::kOffList);
+        hdr[0] = n;
+        hdr[1] = c0;
+        hdr[2] = c1;
+      }
+    }
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = misc[0];
+  if constexpr (SPARSE) {
+    const int *hdr = reinterpret_cast<const int *>(smem + L::kOffList);
+    nu = hdr[0];
+    nblk[0] = hdr[1];
+    nblk[1] = hdr[2];
+  }
 
   if (warp >= 8) {
   // ================================================================ producer warpgroup
@@ -402,7 +455,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kTileBytes);
           const CUtensorMap *m = kind ? &tm_v : &tm_k;
           int c1, c2;
-          kv_coords((ulo + j) * 128, c1, c2);
+          kv_coords((SPARSE ? (blist[j] & 0x3FFF) : ulo + j) * 128, c1, c2);
 #pragma unroll
           for (int c = 0; c < L::kChunks; ++c)
             tma_load_3d(sKV + slot * L::kTileBytes + c * L::kChunkBytes, m, bar(L::kBarKVFull + slot),
@@ -448,6 +501,74 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                  sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (!first || kk > 0));
       };
 
+      if constexpr (SPARSE) {
+        // Union step j loads key block blist[j]; tile t takes part in the steps whose entry
+        // carries its bit.  Its S for its next block is issued one step ahead, right after
+        // its P V of the current block (or at the start, for a first block at step 0).
+        int cnt[2] = {0, 0};  // P V products issued per tile
+        bool ok = nu > 0;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (ok && nblk[t] > 0) ok = wait_bounded(bar(L::kBarQ + t), 0, abort_flag, wait_site(1, L::kBarQ + t, 0));
+        if (ok) ok = wait_bounded(bar(L::kBarKVFull + kslot(0)), kpar(0), abort_flag,
+                                  wait_site(1, L::kBarKVFull + kslot(0), 0));
+        uint32_t e = ok ? blist[0] : 0u;
+        if (ok) {
+          tc_fence_after_sync();
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!(e & (1u << (14 + t)))) continue;
+            issue_qk(t, 0);
+            tc_commit(bar(L::kBarS + t));
+          }
+          tc_commit(bar(L::kBarKVEmpty + kslot(0)));
+        }
+        for (int j = 0; ok && j < nu; ++j) {
+          const uint32_t en = j + 1 < nu ? blist[j + 1] : 0u;
+          if (!wait_bounded(bar(L::kBarKVFull + vslot(j)), vpar(j), abort_flag,
+                            wait_site(1, L::kBarKVFull + vslot(j), j))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          bool knext = false;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const bool in_j = e & (1u << (14 + t)), in_n = en & (1u << (14 + t));
+            if (!ok || (!in_j && !in_n)) continue;
+            if (in_j) {
+              if (!wait_bounded(bar(L::kBarP + t), cnt[t] & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
+                ok = false;
+                continue;
+              }
+              tc_fence_after_sync();
+              issue_pv(t, j, cnt[t] == 0);
+              ++cnt[t];
+            }
+            if (in_n) {
+              if (!knext) {
+                if (!wait_bounded(bar(L::kBarKVFull + kslot(j + 1)), kpar(j + 1), abort_flag,
+                                  wait_site(1, L::kBarKVFull + kslot(j + 1), j + 1))) {
+                  ok = false;
+                  continue;
+                }
+                tc_fence_after_sync();
+                knext = true;
+              }
+              issue_qk(t, j + 1);
+              tc_commit(bar(L::kBarS + t));
+            } else if (cnt[t] == nblk[t]) {
+              tc_commit(bar(L::kBarO + t));  // the tile's last block
+            }
+          }
+          if (!ok) break;
+          tc_commit(bar(L::kBarKVEmpty + vslot(j)));
+          if (knext) tc_commit(bar(L::kBarKVEmpty + kslot(j + 1)));  // every step has a member
+          e = en;
+        }
+        tc_commit(bar(L::kBarDrain));
+        wait_drain(bar(L::kBarDrain), 0, 100000000ull);
+      } else {
       // Local block range of each tile (an empty tile gets an empty range; in the dense
       // variants every tile starts at block 0).
       const int first[2] = {!GEN ? 0 : (nblk[0] > 0 ? a[0] : 1 << 30), !GEN ? 0 : (nblk[1] > 0 ? a[1] : 1 << 30)};
@@ -512,6 +633,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // Nothing issued by this thread may still run when tensor memory is released.
       tc_commit(bar(L::kBarDrain));
       wait_drain(bar(L::kBarDrain), 0, 100000000ull);
+      }
     }
     __syncwarp();
   }
@@ -538,7 +660,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // O / r_run is a properly normalised average.
     float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float sl2 = p.sl2;
+    int cur = -1;  // block-sparse: this tile's current entry of the block list
     for (int j = 0; ok && j < my_n; ++j) {
+      if constexpr (SPARSE) {
+        do ++cur;
+        while (cur < nu - 1 && !(blist[cur] & (1u << (14 + t))));
+      }
       if (!warp_wait_bounded(bar(L::kBarS + t), j & 1, abort_flag, wait_site(1, L::kBarS + t, j))) {
         ok = false;
         break;
@@ -554,15 +681,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_ld_x64_nowait(tS + 64, s1);
         tmem_wait_ld_2x64(s0, s1);
       }
-      const int kv0 = (my_j0 + j) * 128;
+      const int kv0 = (SPARSE ? (blist[cur] & 0x3FFF) : my_j0 + j) * 128;
       bool masked;
       if constexpr (GEN) {
         masked = block_needs_mask<128>(p.left, p.right, sg.Lk, my_qb * 128 + sg.dlt, kv0);
         if (masked) mask_scores<128>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
       } else {
-        masked = (MODE == kAttnCausal && j == my_qb) || kv0 + 128 > p.N;
+        const bool causal = MODE == kAttnCausal || (SPARSE && p.right == 0);
+        masked = (causal && kv0 == my_qb * 128) || kv0 + 128 > p.N;
         if (masked) {
-          const int lim = MODE == kAttnCausal ? min(qrow + 1, p.N) : p.N;  // keys kv < lim are visible
+          const int lim = causal ? min(qrow + 1, p.N) : p.N;  // keys kv < lim are visible
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
@@ -611,11 +739,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // cases take a separate path: a packed tile that ends past its sequence stores its
     // rows directly, and a tile that sees no key writes O = 0 (no MMA touched it).
     if (my_valid) {
-      bool okw = ok && ((GEN && my_n == 0) ||
+      bool okw = ok && ((GENLIKE && my_n == 0) ||
                         warp_wait_bounded(bar(L::kBarO + t), 0, abort_flag, wait_site(1, L::kBarO + t, 0)));
       okw = named_bar_and(1 + t, 128, okw && *abort_flag == 0);
       const bool direct = packed && my_qb * 128 + 128 > sg.Lq;
-      if (okw && (!GEN || (!direct && my_n > 0))) {
+      if (okw && (!GENLIKE || (!direct && my_n > 0))) {
         tc_fence_after_sync();
         // rows without keys: O = 0; dropout scales the kept probabilities by 1 / (1 - p)
         const float inv_l = (!GEN || r_run > 0.f) ? (DROP ? p.drop.inv_keep : 1.f) / r_run : 0.f;
@@ -646,7 +774,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           bulk_commit_group();
           bulk_wait_group_read0();
         }
-      } else if (GEN && okw) {
+      } else if (GENLIKE && okw) {
         fwd_epilogue_rows<D>(tO, my_n > 0, r_run, qrow < sg.Lq, direct, sQ + t * L::kTileBytes, r,
                              p.o + (static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h) * D);
         if (!direct) {
@@ -664,7 +792,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       if (okw && qrow < sg.Lq) {
-        const float lse = (!GEN || l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        const float lse = (!GENLIKE || l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         if (packed)
           p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + my_h] = lse;
         else

@@ -48,15 +48,19 @@ struct FwdD256Layout {
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  // Block-sparse variant only: after misc, a 16-byte header {blocks} and the list of the
+  // 64-key blocks to visit (uint16), two per enabled 128-key mask block.
+  static constexpr int kOffList = kOffMisc + 16;
+  static constexpr int kSmemBytesSparse = kOffList + 16 + 2 * (2 * kMaxSparseBlocks) + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kTmS0 = 0;     // S_a: columns 0..63, S_b: 64..127
   static constexpr uint32_t kTmO = 128;    // O: columns 128..383
-  static_assert(kSmemBytes <= 232448, "shared-memory budget");
+  static_assert(kSmemBytesSparse <= 232448, "shared-memory budget");
 };
 
 constexpr int kFwdD256Threads = 192;  // warps 0-3 softmax, 4 MMA, 5 TMA
 
-template <int MODE, bool DROP = false>  // MODE: kAttnFull, kAttnCausal or kAttnGeneral (fa_common.cuh)
+template <int MODE, bool DROP = false>  // MODE: kAttnFull, kAttnCausal, kAttnGeneral or kAttnSparse
 __global__ void __launch_bounds__(kFwdD256Threads, 1)
     fa_fwd_d256_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -84,7 +88,13 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
   const int b = u / p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
   constexpr bool GEN = MODE == kAttnGeneral;
+  constexpr bool SPARSE = MODE == kAttnSparse;
+  constexpr bool GENLIKE = GEN || SPARSE;  // rows may see no key at all
   const bool packed = GEN && p.cu_q != nullptr;
+  // Block-sparse: the 64-key blocks of the enabled 128-key mask blocks of this query block
+  // (up to the diagonal when causal), in order; written to shared memory by the TMA warp
+  // before the roles start.
+  const uint16_t *blist = reinterpret_cast<const uint16_t *>(smem + L::kOffList + 16);
   SeqGeom sg{p.N, p.N, 0, 0, 0};
   // 64-key blocks [jlo, jlo + nblk) that some row of the query block can see; the loop
   // index j below counts from jlo.  nblk = 0: no row sees a key (O = 0, LSE = -inf).
@@ -95,7 +105,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
     int jhi = -1;
     key_block_range<64>(p.left, p.right, sg, qb * 128, jlo, jhi);
     nblk = jhi - jlo + 1;
-  } else {
+  } else if constexpr (!SPARSE) {
     const int nkb_all = (p.N + 63) / 64;
     nblk = MODE == kAttnCausal ? min(2 * qb + 2, nkb_all) : nkb_all;
   }
@@ -116,10 +126,32 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
     tmem_alloc(smem_u32(misc), L::kTmemCols);
     tmem_relinquish_alloc_permit();
   }
+  if constexpr (SPARSE) {
+    if (warp == 5) {
+      const uint8_t *row = p.bmask + (static_cast<size_t>(b * p.Hq + h) * p.nqb + qb) * p.nqb;
+      const int hi = p.right == 0 ? qb : p.nqb - 1;
+      const int nkb64 = (p.N + 63) / 64;
+      uint16_t *list = reinterpret_cast<uint16_t *>(smem + L::kOffList + 16);
+      int n = 0;
+      for (int base0 = 0; base0 <= hi; base0 += 32) {
+        const int kb = base0 + lane;
+        const bool m = kb <= hi && row[kb] != 0;
+        const bool two = m && 2 * kb + 1 < nkb64;  // the second half exists
+        const uint32_t u1 = __ballot_sync(0xffffffffu, m), u2 = __ballot_sync(0xffffffffu, two);
+        const uint32_t below = (1u << lane) - 1u;
+        const int at = n + __popc(u1 & below) + __popc(u2 & below);
+        if (m) list[at] = static_cast<uint16_t>(2 * kb);
+        if (two) list[at + 1] = static_cast<uint16_t>(2 * kb + 1);
+        n += __popc(u1) + __popc(u2);
+      }
+      if (lane == 0) *reinterpret_cast<int *>(smem + L::kOffList) = n;
+    }
+  }
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = misc[0];
+  if constexpr (SPARSE) nblk = *reinterpret_cast<const int *>(smem + L::kOffList);
 
   // Load/consume order of the K/V ring: K_0, K_1, then V_j followed by K_{j+2}.
   // Item index -> (is_v, block).  Both the TMA warp and the MMA warp walk this order.
@@ -148,7 +180,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
         mbar_arrive_expect_tx(bar(L::kBarKVFull + slot), L::kKVBytes);
         const CUtensorMap *m = is_v ? &tm_v : &tm_k;
         int c1, c2;
-        kv_coords((jlo + j) * 64, c1, c2);
+        kv_coords((SPARSE ? blist[j] : jlo + j) * 64, c1, c2);
 #pragma unroll
         for (int c = 0; c < L::kChunks; ++c)
           tma_load_3d(sKV + slot * L::kKVBytes + c * L::kKChunkBytes, m, bar(L::kBarKVFull + slot), c * 64,
@@ -246,15 +278,18 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       tc_fence_after_sync();
       uint32_t s[64];
       tmem_ld_x64(tS, s);
-      const int kv0 = (jlo + j) * 64;
+      const int kv0 = (SPARSE ? blist[j] : jlo + j) * 64;
       bool masked;
       if constexpr (GEN) {
         masked = block_needs_mask<64>(p.left, p.right, sg.Lk, qb * 128 + sg.dlt, kv0);
         if (masked) mask_scores<64>(s, p.left, p.right, sg.Lk, qrow + sg.dlt, kv0);
       } else {
-        masked = (MODE == kAttnCausal && kv0 + 63 > qb * 128) || kv0 + 64 > p.N;
+        // (block-sparse: a row's first block always holds a visible key, the diagonal
+        // block's first half coming before its second)
+        const bool causal = MODE == kAttnCausal || (SPARSE && p.right == 0);
+        masked = (causal && kv0 + 63 > qb * 128) || kv0 + 64 > p.N;
         if (masked) {
-          const int lim = MODE == kAttnCausal ? min(qrow + 1, p.N) : p.N;  // keys kv < lim are visible
+          const int lim = causal ? min(qrow + 1, p.N) : p.N;  // keys kv < lim are visible
 #pragma unroll
           for (int c = 0; c < 64; ++c)
             if (kv0 + c >= lim) s[c] = __float_as_uint(-INFINITY);
@@ -303,12 +338,12 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
       if (lane == 0) mbar_arrive(bar(L::kBarP + (j & 1)));  // one arrival per warp
     }
 
-    bool okw = ok && ((GEN && nblk == 0) || warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0)));
+    bool okw = ok && ((GENLIKE && nblk == 0) || warp_wait_bounded(bar(L::kBarO), 0, abort_flag, wait_site(2, L::kBarO, 0)));
     okw = named_bar_and(1, 128, okw && *abort_flag == 0);
     if (okw) {
       tc_fence_after_sync();
       // rows without keys: O = 0; dropout scales the kept probabilities by 1 / (1 - p)
-      const float inv_l = (!GEN || r_run > 0.f) ? (DROP ? p.drop.inv_keep : 1.f) / r_run : 0.f;
+      const float inv_l = (!GENLIKE || r_run > 0.f) ? (DROP ? p.drop.inv_keep : 1.f) / r_run : 0.f;
       // A packed block that ends past its sequence stores its rows directly.
       const bool direct = packed && qb * 128 + 128 > sg.Lq;
       const bool row_ok = qrow < sg.Lq;
@@ -316,7 +351,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc) {
         uint32_t o[32];
-        if (!GEN || nblk > 0) {
+        if (!GENLIKE || nblk > 0) {
           tmem_ld_x32(tO + cc * 32, o);
         } else {
 #pragma unroll
@@ -348,7 +383,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
         }
       }
       if (row_ok) {
-        const float lse = (!GEN || l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        const float lse = (!GENLIKE || l_run > 0.f) ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         if (packed)
           p.lse[static_cast<size_t>(sg.q_base + qrow) * p.Hq + h] = lse;
         else

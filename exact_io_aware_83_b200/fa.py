@@ -91,6 +91,11 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_bwd_dropout.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
                                        ci, ci, ci, ci, ci, ci, cf, u64, cf, vp]
         lib.fa_bwd_dropout.restype = ci
+        lib.fa_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, vp]
+        lib.fa_fwd_blocksparse.restype = ci
+        lib.fa_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp,
+                                           ci, ci, ci, ci, ci, ci, cf, vp]
+        lib.fa_bwd_blocksparse.restype = ci
         lib.fa_decode_num_splits.argtypes = [ci, ci, ci, ci, ci, ci]
         lib.fa_decode_num_splits.restype = ci
         lib.fa_decode_workspace_bytes.argtypes = [ci, ci, ci, ci, ci, ci, ci]
@@ -203,6 +208,21 @@ def fa_bwd_dropout(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes
            "fa_bwd_dropout")
 
 
+def fa_fwd_blocksparse(q, k, v, o, lse, block_mask, B, Hq, Hkv, N, d, causal, scale,
+                       stream) -> None:
+    _check(load().fa_fwd_blocksparse(q, k, v, o, lse, block_mask, B, Hq, Hkv, N, d, int(causal),
+                                     float(scale), stream),
+           "fa_fwd_blocksparse")
+
+
+def fa_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, block_mask,
+                       B, Hq, Hkv, N, d, causal, scale, stream) -> None:
+    _check(load().fa_bwd_blocksparse(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                                     block_mask, B, Hq, Hkv, N, d, int(causal), float(scale),
+                                     stream),
+           "fa_bwd_blocksparse")
+
+
 def fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d) -> int:
     return int(load().fa_decode_num_splits(B, Hq, Hkv, Nq, Nk, d))
 
@@ -280,12 +300,27 @@ def _window(causal, window):
     return left, right
 
 
+def _block_mask(block_mask, B, Hq, N, win, dropout_p):
+    import torch
+    if block_mask is None:
+        return None
+    nb = (N + 127) // 128
+    if (not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous()
+            or tuple(block_mask.shape) != (B, Hq, nb, nb)):
+        raise ValueError(f"block_mask must be a contiguous uint8 CUDA tensor [{B}, {Hq}, {nb}, {nb}]")
+    if win is not None or dropout_p:
+        raise ValueError("block_mask combines with causal only (no window, no dropout)")
+    return block_mask
+
+
 def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-        window=None, dropout_p: float = 0.0, seed: int = 0):
+        window=None, dropout_p: float = 0.0, seed: int = 0, block_mask=None):
     """O, LSE = attention(q, k, v); q [B,Hq,N,d], k/v [B,Hkv,N,d] bf16 on one GPU.
     ``window=(left, right)``: local attention, key j visible to query i iff
     i - left <= j <= i + right (-1 = unlimited on that side).  ``dropout_p`` > 0: attention
-    dropout with the Philox4x32-10 mask of ``seed`` (full or causal attention)."""
+    dropout with the Philox4x32-10 mask of ``seed`` (full or causal attention).
+    ``block_mask``: block-sparse attention, uint8 [B, Hq, ceil(N/128), ceil(N/128)] on the
+    GPU, nonzero = the 128 x 128 block is computed (with or without ``causal``)."""
     import torch
     win = _window(causal, window)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -296,7 +331,11 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     scale = default_scale(d) if scale is None else scale
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    if dropout_p:
+    bm = _block_mask(block_mask, B, Hq, N, win, dropout_p)
+    if bm is not None:
+        fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                           bm.data_ptr(), B, Hq, Hkv, N, d, causal, scale, _stream_handle(q))
+    elif dropout_p:
         if win is not None:
             raise ValueError("dropout is supported with full or causal attention only")
         fa_fwd_dropout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
@@ -312,8 +351,9 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
 
 def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
         workspace=None, dq=None, dk=None, dv=None, window=None, dropout_p: float = 0.0,
-        seed: int = 0):
-    """dQ, dK, dV of <O, dO> given the forward's O and LSE (same causal / window)."""
+        seed: int = 0, block_mask=None):
+    """dQ, dK, dV of <O, dO> given the forward's O and LSE (same causal / window /
+    dropout / block_mask)."""
     import torch
     win = _window(causal, window)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
@@ -329,7 +369,10 @@ def bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
     ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
             dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
             workspace.numel() * workspace.element_size(), B, Hq, Hkv, N, d)
-    if dropout_p:
+    bm = _block_mask(block_mask, B, Hq, N, win, dropout_p)
+    if bm is not None:
+        fa_bwd_blocksparse(*ptrs[:11], bm.data_ptr(), *ptrs[11:], causal, scale, _stream_handle(q))
+    elif dropout_p:
         if win is not None:
             raise ValueError("dropout is supported with full or causal attention only")
         fa_bwd_dropout(*ptrs, causal, dropout_p, seed, scale, _stream_handle(q))

@@ -17,11 +17,15 @@ long_8k_causal        2   16   16   8192  128  yes     fwd+bwd    N(0,1)
 gqa_4k_causal_fwd     4   32   8    4096  128  yes     fwd        N(0,1)
 d256_4k_stress        2   8    8    4096  256  no      fwd+bwd    N(0,4^2)
 window_8k_1k          2   16   16   8192  128  band    fwd+bwd    N(0,1)
+dropout_8k_causal     2   16   16   8192  128  yes     fwd+bwd    N(0,1)
+blocksparse_8k_causal 2   16   16   8192  128  yes     fwd+bwd    N(0,1)
 ====================  ==  ===  ===  ====  ===  ======  =========  =====================
 
 window_8k_1k is local attention with the band i - 1023 <= j <= i (1024 keys per row,
 the row's own included); dropout_8k_causal is long_8k_causal with attention dropout
-p = 0.1 (Philox4x32-10 mask, seed 8080).
+p = 0.1 (Philox4x32-10 mask, seed 8080); blocksparse_8k_causal is long_8k_causal with a
+block mask enabling each 128 x 128 block with probability 1/4 and every diagonal block
+(mask seed 1010), causal on top.
 
 Packed variable-length workload: varlen_32k_ragged, 24 sequences of long-tailed length
 (log-normal around 1500 tokens, clipped to [16, 8192]; 39.7k tokens in all, longest 3867), 16 heads,
@@ -59,6 +63,15 @@ class Workload:
     window: tuple | None = None   # (left, right) key band, -1 = unlimited; None: causal flag
     dropout_p: float = 0.0        # attention dropout probability (0: none)
     dropout_seed: int = 0
+    block_density: float = 0.0    # block-sparse: share of enabled 128 x 128 blocks (0: dense)
+    mask_seed: int = 0
+
+    def block_mask(self):
+        """The block-sparse workload's mask (None for dense workloads)."""
+        if not self.block_density:
+            return None
+        return draw_block_mask(self.B, self.Hq, self.N, self.block_density, self.mask_seed,
+                               diagonal=True)
 
     @property
     def scale(self) -> float:
@@ -67,8 +80,10 @@ class Workload:
         return float(torch.tensor(1.0 / math.sqrt(self.d), dtype=torch.float32).item())
 
     def fwd_flops(self) -> float:
-        """4 B Hq N^2 d, halved when causal (the metric's convention); with a key band,
-        4 B Hq d times the number of visible (query, key) pairs."""
+        """4 B Hq N^2 d, halved when causal (the metric's convention); with a key band or
+        a block mask, 4 d times the number of visible (query, key) pairs."""
+        if self.block_density:
+            return 4.0 * blocksparse_pairs(self.block_mask(), self.N, self.causal) * self.d
         if self.window is not None:
             left, right = self.window
             pairs = 0
@@ -95,6 +110,8 @@ WORKLOADS = {
         Workload("d256_4k_stress", 2, 8, 8, 4096, 256, False, True, 4.0, 5),
         Workload("window_8k_1k", 2, 16, 16, 8192, 128, False, True, 1.0, 6, (1023, 0)),
         Workload("dropout_8k_causal", 2, 16, 16, 8192, 128, True, True, 1.0, 9, None, 0.1, 8080),
+        Workload("blocksparse_8k_causal", 2, 16, 16, 8192, 128, True, True, 1.0, 10,
+                 block_density=0.25, mask_seed=1010),
     )
 }
 
@@ -231,3 +248,28 @@ def packed_lengths(n: int, mean: int, seed: int, lo: int = 16, hi: int = 8192):
     x = torch.randn(n, generator=g, dtype=torch.float64) * 0.8
     lens = (torch.exp(x) * mean / math.exp(0.32)).round().clamp(lo, hi).to(torch.int64)
     return [int(v) for v in lens]
+
+
+def draw_block_mask(B: int, Hq: int, N: int, density: float, seed: int, diagonal: bool = False):
+    """uint8 CPU tensor [B, Hq, nb, nb], nb = ceil(N / 128): each 128 x 128 block enabled
+    independently with probability `density` (the diagonal blocks always, with
+    `diagonal`)."""
+    nb = (N + 127) // 128
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    m = (torch.rand((B, Hq, nb, nb), generator=g, dtype=torch.float64) < density).to(torch.uint8)
+    if diagonal:
+        m[:, :, range(nb), range(nb)] = 1
+    return m
+
+
+def blocksparse_pairs(mask, N: int, causal: bool) -> int:
+    """Visible (query, key) pairs of a block mask [B, Hq, nb, nb]: a counting helper for
+    FLOP totals (every pair of an enabled block, j <= i only with causal)."""
+    nb = mask.shape[-1]
+    rows = torch.tensor([min(128, N - 128 * b) for b in range(nb)], dtype=torch.float64)
+    full = rows[:, None] * rows[None, :]                  # pairs of block (qb, kb)
+    if causal:
+        full = torch.tril(full, -1)
+        full += torch.diag(rows * (rows + 1) / 2)
+    return int((mask.to(torch.float64) * full).sum().item())

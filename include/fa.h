@@ -25,9 +25,12 @@
  *    visible to query i when j <= i;
  *  - local (sliding-window) attention: the "FlashAttention1" Q&A, question on scaling to
  *    very long sequences, item 4, proposes combining the method with local attention;
- *    the deep-dive page's closing paragraph names block-sparse FlashAttention.  Neither
- *    defines the window; this library's reading is the band i - left <= j <= i + right,
- *    and key blocks outside every row's band are skipped rather than masked.
+ *    neither page defines the window; this library's reading is the band
+ *    i - left <= j <= i + right, and key blocks outside every row's band are skipped
+ *    rather than masked;
+ *  - block-sparse attention: the deep-dive page's closing paragraph names block-sparse
+ *    FlashAttention; this library's reading is a per-head 0/1 mask over 128 x 128 blocks
+ *    (see fa_fwd_blocksparse).
  *
  * Conventions shared by every entry point
  *  - Layout: Q, dQ, O, dO are [B, Hq, N, d]; K, V, dK, dV are [B, Hkv, N, d]; all
@@ -197,6 +200,40 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, co
                   const void *dout, void *dq, void *dk, void *dv, void *workspace,
                   size_t workspace_bytes, int B, int Hq, int Hkv, int N, int d, int window_left,
                   int window_right, float scale, void *stream);
+
+/*
+ * Block-sparse attention: the deep-dive page's closing paragraph names block-sparse
+ * FlashAttention without defining it.  The library's reading: a 0/1 mask over the
+ * 128 x 128 blocks of each query head's score matrix; key j is visible to query i iff
+ * block_mask[b][h][i / 128][j / 128] != 0 (and, with causal = 1, j <= i).  Only enabled
+ * blocks are loaded and multiplied; the others cost nothing.
+ *   q, k, v, o, lse, B, Hq, Hkv, N, d, scale, stream: as fa_fwd (dense [B, H, N, d]).
+ *   block_mask: DEVICE uint8 [B, Hq, nb, nb], nb = ceil(N / 128), row-major; any nonzero
+ *        byte enables its block.  Read, never written; the caller keeps it alive until
+ *        the call's kernels have run.  With causal = 1, blocks above the diagonal are
+ *        ignored whatever their byte.
+ * A row whose blocks are all disabled gets O = 0 and LSE = -inf.  Limits: nb <= 4096, and
+ * (Hq / Hkv) * ceil(nb / 32) * 4 bytes of per-key-block bitmap for the backward within
+ * its shared-memory budget (8192 bytes for d = 64 and 128, about 1.3 KB for d = 256);
+ * larger sizes return FA_ERR_UNSUPPORTED (checked by both calls, so a forward that runs
+ * always has a backward).  A NULL mask or a causal flag other than 0/1 is
+ * FA_ERR_INVALID_ARG.
+ */
+int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
+                       const unsigned char *block_mask, int B, int Hq, int Hkv, int N, int d,
+                       int causal, float scale, void *stream);
+
+/*
+ * Backward pass of fa_fwd_blocksparse (same mask and causal flag; O and LSE from it):
+ * arguments as fa_bwd plus block_mask.  A key block is visited only by the query blocks
+ * of the query heads that enable it; a key that no query sees gets dK = dV = 0, a query
+ * that sees no key dQ = 0.
+ */
+int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *o,
+                       const float *lse, const void *dout, void *dq, void *dk, void *dv,
+                       void *workspace, size_t workspace_bytes, const unsigned char *block_mask,
+                       int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                       void *stream);
 
 /*
  * Backward pass for callers that cannot allocate device memory.

@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
                      "fa_fwd_varlen", "fa_bwd_varlen", "fa_fwd_dropout", "fa_bwd_dropout",
                      "fa_decode_num_splits", "fa_decode_workspace_bytes", "fa_merge",
                      "fa_bwd_workspace_bytes", "fa_device_status", "fa_status_string",
-                     "fa_version"):
+                     "fa_version", "fa_fwd_blocksparse", "fa_bwd_blocksparse"):
         assert required in names
 
 
@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_version():
-    assert fa.load().fa_version() == 101
+    assert fa.load().fa_version() == 102
     for code in range(8):
         assert fa.fa_status_string(code) not in ("", "unknown status")
     assert fa.fa_status_string(99) == "unknown status"
@@ -221,6 +221,34 @@ def test_dropout_argument_errors(p_drop, causal, code):
                               0.125, None) == code
     assert lib.fa_bwd_dropout(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30,
                               1, 2, 1, 16, 128, causal, p_drop, 7, 0.125, None) == code
+
+
+def _sparse(mask, Hq, Hkv, N, d, causal):
+    lib = fa.load()
+    rf = lib.fa_fwd_blocksparse(FAKE, FAKE, FAKE, FAKE, FAKE, mask, 1, Hq, Hkv, N, d, causal, 0.125,
+                                None)
+    rb = lib.fa_bwd_blocksparse(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 40,
+                                mask, 1, Hq, Hkv, N, d, causal, 0.125, None)
+    return rf, rb
+
+
+@pytest.mark.parametrize("mask,Hq,Hkv,N,d,causal,code", [
+    (None, 2, 1, 16, 128, 0, fa.FA_ERR_INVALID_ARG),              # no mask
+    (FAKE, 2, 1, 16, 128, 2, fa.FA_ERR_INVALID_ARG),              # causal not 0/1
+    (FAKE, 2, 1, 4096 * 128 + 1, 64, 0, fa.FA_ERR_UNSUPPORTED),   # more than 4096 blocks a side
+    (FAKE, 64, 1, 32768, 256, 1, fa.FA_ERR_UNSUPPORTED),          # d = 256 bitmap: 64 x 8 words
+    (FAKE, 2, 3, 16, 128, 0, fa.FA_ERR_GQA),
+])
+def test_blocksparse_argument_errors(mask, Hq, Hkv, N, d, causal, code):
+    assert _sparse(mask, Hq, Hkv, N, d, causal) == (code, code)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="valid-argument path needs no GPU")
+def test_blocksparse_limits_that_fit_reach_the_device_check():
+    # 64 query heads per K/V head over 256 blocks: 2 KB of bitmap fits for d = 128, and a
+    # 4096-block side is the longest sequence taken.
+    assert _sparse(FAKE, 64, 1, 32768, 128, 1) == (fa.FA_ERR_CUDA, fa.FA_ERR_CUDA)
+    assert _sparse(FAKE, 2, 1, 4096 * 128, 64, 0) == (fa.FA_ERR_CUDA, fa.FA_ERR_CUDA)
 
 
 def test_workspace_size():
