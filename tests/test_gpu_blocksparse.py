@@ -4,8 +4,8 @@ Key j is visible to query i iff block (i // 128, j // 128) of the query head's 0
 enabled (and j <= i with causal); the deep-dive page's closing paragraph names block-sparse
 FlashAttention.  Tolerances as for the dense tests: |O - O_ref| <= max(1e-2, one bf16
 spacing of O_ref), |LSE - LSE_ref| <= 1e-3, relative Frobenius error <= 2e-2 for dQ, dK,
-dV, guard bands intact, no NaN/Inf.  Exact checks: an all-ones mask reproduces fa_fwd /
-fa_bwd bit for bit (same blocks in the same order), an all-zeros mask gives O = 0,
+dV, guard bands intact, no NaN/Inf.  Exact checks: an all-ones mask reproduces fa_fwd and
+fa_bwd's dK, dV bit for bit (same blocks in the same order), an all-zeros mask gives O = 0,
 LSE = -inf and zero gradients, and rows or keys whose blocks are all disabled give zeros.
 """
 import math
@@ -142,8 +142,10 @@ def test_all_ones_mask_equals_dense_calls_bitwise(d):
         g1 = fa.bwd(qd, kd, vd, o1, l1, dod, causal=causal)
         g2 = fa.bwd(qd, kd, vd, o1, l1, dod, causal=causal, block_mask=ones)
         torch.cuda.synchronize()
-        for a, b in zip(g1, g2):
-            assert torch.equal(a, b)
+        assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+        # dQ sums the key blocks' fp32 partials with reduce-adds in whatever order the
+        # CTAs finish, so two runs of the same kernel agree only up to rounding.
+        assert _rel_fro(_f64(g1[0]), _f64(g2[0])) < 1e-3
 
 
 @pytest.mark.parametrize("d", [64, 128, 256])
