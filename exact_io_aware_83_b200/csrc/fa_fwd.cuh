@@ -117,7 +117,9 @@ struct FwdLayout {
   static constexpr int kBarS = kBarKVEmpty + kStages;
   static constexpr int kBarP = kBarS + 2;
   static constexpr int kBarO = kBarP + 2;
-  static constexpr int kBarDrain = kBarO + 2;
+  static constexpr int kBarPV = kBarO + 2;    // block-sparse: P V of tile t completed
+  static constexpr int kBarSX = kBarPV + 2;   // block-sparse: S buffer b holds a tile-1 block
+  static constexpr int kBarDrain = kBarSX + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // [0] TMEM base, [1] abort flag
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-B alignment
@@ -481,90 +483,104 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       auto vslot = [](int j) { return (2 * j + 1) % S; };
       auto vpar = [](int j) { return static_cast<uint32_t>(((2 * j + 1) / S) & 1); };
       // S_t = Q_t K_j^T : M = 128 query rows, N = 128 keys, K = D (16 per instruction).
-      auto issue_qk = [&](int t, int j) {
+      // (buf: the S buffer; the dense variants use buffer t for tile t)
+      auto issue_qk = [&](int t, int j, int buf) {
         const uint32_t a0 = sQ + t * L::kTileBytes;
         const uint32_t b0 = sKV + kslot(j) * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * L::kChunkBytes + (kk % 4) * 32;
-          mma_ss(tmem + L::tm_s(t), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
+          mma_ss(tmem + L::tm_s(buf), sdesc_sw128(a0 + off, 16, 1024), sdesc_sw128(b0 + off, 16, 1024),
                  idesc_qk, kk > 0);
         }
       };
       // O_t += P_t V_j : M = 128 query rows, N = D, K = 128 keys; P (bf16) in TMEM,
       // V MN-major in shared memory (16 key rows = 2048 bytes per instruction).
-      auto issue_pv = [&](int t, int j, bool first) {
+      auto issue_pv = [&](int t, int j, bool first, int buf) {
         const uint32_t b0 = sKV + vslot(j) * L::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + L::tm_o(t), tmem + L::tm_s(t) + kk * 8,
+          mma_ts(tmem + L::tm_o(t), tmem + L::tm_s(buf) + kk * 8,
                  sdesc_sw128(b0 + kk * 2048, L::kChunkBytes, 1024), idesc_pv, (!first || kk > 0));
       };
 
       if constexpr (SPARSE) {
         // Union step j loads key block blist[j]; tile t takes part in the steps whose entry
-        // carries its bit.  Its S for its next block is issued one step ahead, right after
-        // its P V of the current block (or at the start, for a first block at step 0).
-        int cnt[2] = {0, 0};  // P V products issued per tile
+        // carries its bit.  Score tiles are numbered n = 0, 1, ... in list order (tile 0
+        // before tile 1 within a step) and use the two S buffers alternately (n & 1), so a
+        // tile whose blocks come in a run can have its next Q K^T computed while its
+        // softmax works on the current one.  Score tile n + 2 is issued right after P V of
+        // score tile n, which frees its buffer.  Every barrier has one waiter that takes
+        // its phases in order and can never fall two phases behind or ahead: "S ready" per
+        // (buffer, tile) (kBarS + b for tile 0, kBarSX + b for tile 1), "P written" per
+        // buffer (the MMA consumes score tiles in order, and a buffer's next occupant is
+        // issued only after its P was consumed), "P V done" per tile for the softmax's rare
+        // rescale of O.
+        const int total = nblk[0] + nblk[1];
+        auto first_pos = [&](int &j, int &t) {
+          j = 0;
+          t = (blist[0] & (1u << 14)) ? 0 : 1;
+        };
+        auto advance = [&](int &j, int &t) {
+          if (t == 0 && (blist[j] & (1u << 15))) {
+            t = 1;
+            return;
+          }
+          ++j;
+          if (j < nu) t = (blist[j] & (1u << 14)) ? 0 : 1;
+        };
+        auto last_of_step = [&](int j, int t) { return t == 1 || !(blist[j] & (1u << 15)); };
         bool ok = nu > 0;
 #pragma unroll
         for (int t = 0; t < 2; ++t)
           if (ok && nblk[t] > 0) ok = wait_bounded(bar(L::kBarQ + t), 0, abort_flag, wait_site(1, L::kBarQ + t, 0));
-        if (ok) ok = wait_bounded(bar(L::kBarKVFull + kslot(0)), kpar(0), abort_flag,
-                                  wait_site(1, L::kBarKVFull + kslot(0), 0));
-        uint32_t e = ok ? blist[0] : 0u;
-        if (ok) {
-          tc_fence_after_sync();
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!(e & (1u << (14 + t)))) continue;
-            issue_qk(t, 0);
-            tc_commit(bar(L::kBarS + t));
+        int qj = 0, qt = 0, nq = 0, k_ready = -1;
+        auto issue_next_qk = [&]() {
+          if (qj != k_ready) {
+            if (!wait_bounded(bar(L::kBarKVFull + kslot(qj)), kpar(qj), abort_flag,
+                              wait_site(1, L::kBarKVFull + kslot(qj), qj))) {
+              ok = false;
+              return;
+            }
+            tc_fence_after_sync();
+            k_ready = qj;
           }
-          tc_commit(bar(L::kBarKVEmpty + kslot(0)));
+          issue_qk(qt, qj, nq & 1);
+          tc_commit(bar((qt ? L::kBarSX : L::kBarS) + (nq & 1)));
+          if (last_of_step(qj, qt)) tc_commit(bar(L::kBarKVEmpty + kslot(qj)));
+          ++nq;
+          advance(qj, qt);
+        };
+        if (ok) {
+          first_pos(qj, qt);
+          issue_next_qk();
+          if (ok && total > 1) issue_next_qk();
         }
-        for (int j = 0; ok && j < nu; ++j) {
-          const uint32_t en = j + 1 < nu ? blist[j + 1] : 0u;
-          if (!wait_bounded(bar(L::kBarKVFull + vslot(j)), vpar(j), abort_flag,
-                            wait_site(1, L::kBarKVFull + vslot(j), j))) {
+        int cnt[2] = {0, 0};  // P V products issued per tile
+        int pj = 0, pt = 0, v_ready = -1;
+        if (ok) first_pos(pj, pt);
+        for (int n = 0; ok && n < total; ++n) {
+          if (pj != v_ready) {
+            if (!wait_bounded(bar(L::kBarKVFull + vslot(pj)), vpar(pj), abort_flag,
+                              wait_site(1, L::kBarKVFull + vslot(pj), pj))) {
+              ok = false;
+              break;
+            }
+            v_ready = pj;
+          }
+          if (!wait_bounded(bar(L::kBarP + (n & 1)), (n >> 1) & 1, abort_flag,
+                            wait_site(1, L::kBarP + (n & 1), n))) {
             ok = false;
             break;
           }
           tc_fence_after_sync();
-          bool knext = false;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            const bool in_j = e & (1u << (14 + t)), in_n = en & (1u << (14 + t));
-            if (!ok || (!in_j && !in_n)) continue;
-            if (in_j) {
-              if (!wait_bounded(bar(L::kBarP + t), cnt[t] & 1, abort_flag, wait_site(1, L::kBarP + t, j))) {
-                ok = false;
-                continue;
-              }
-              tc_fence_after_sync();
-              issue_pv(t, j, cnt[t] == 0);
-              ++cnt[t];
-            }
-            if (in_n) {
-              if (!knext) {
-                if (!wait_bounded(bar(L::kBarKVFull + kslot(j + 1)), kpar(j + 1), abort_flag,
-                                  wait_site(1, L::kBarKVFull + kslot(j + 1), j + 1))) {
-                  ok = false;
-                  continue;
-                }
-                tc_fence_after_sync();
-                knext = true;
-              }
-              issue_qk(t, j + 1);
-              tc_commit(bar(L::kBarS + t));
-            } else if (cnt[t] == nblk[t]) {
-              tc_commit(bar(L::kBarO + t));  // the tile's last block
-            }
-          }
-          if (!ok) break;
-          tc_commit(bar(L::kBarKVEmpty + vslot(j)));
-          if (knext) tc_commit(bar(L::kBarKVEmpty + kslot(j + 1)));  // every step has a member
-          e = en;
+          issue_pv(pt, pj, cnt[pt] == 0, n & 1);
+          ++cnt[pt];
+          tc_commit(bar(L::kBarPV + pt));
+          if (cnt[pt] == nblk[pt]) tc_commit(bar(L::kBarO + pt));  // the tile's last block
+          if (last_of_step(pj, pt)) tc_commit(bar(L::kBarKVEmpty + vslot(pj)));
+          if (n + 2 < total) issue_next_qk();
+          advance(pj, pt);
         }
         tc_commit(bar(L::kBarDrain));
         wait_drain(bar(L::kBarDrain), 0, 100000000ull);
@@ -584,7 +600,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (nblk[t] == 0 || a[t] != 0) continue;
-          issue_qk(t, 0);
+          issue_qk(t, 0, t);
           tc_commit(bar(L::kBarS + t));
         }
         tc_commit(bar(L::kBarKVEmpty + kslot(0)));
@@ -608,7 +624,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               continue;
             }
             tc_fence_after_sync();
-            issue_pv(t, j, j == first[t]);
+            issue_pv(t, j, j == first[t], t);
           }
           if (j < last[t]) {
             if (!knext) {
@@ -620,7 +636,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               tc_fence_after_sync();
               knext = true;
             }
-            issue_qk(t, j + 1);
+            issue_qk(t, j + 1, t);
             tc_commit(bar(L::kBarS + t));
           } else {
             tc_commit(bar(L::kBarO + t));  // jt is this tile's last block
@@ -644,7 +660,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const int wq = warp % 4;          // TMEM lane quadrant of this warp
     const int r = wq * 32 + lane;     // row of the tile = TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + L::tm_s(t) + lane_off;
+    uint32_t tS = tmem + L::tm_s(t) + lane_off;  // block-sparse: the block's S buffer
     const uint32_t tO = tmem + L::tm_o(t) + lane_off;
     // This warpgroup's tile (selects instead of runtime-indexed arrays keep them in registers).
     const int my_qb = t ? qb[1] : qb[0];
@@ -660,13 +676,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // O / r_run is a properly normalised average.
     float m_run = -INFINITY, l_run = 0.f, r_run = 0.f;
     const float sl2 = p.sl2;
-    int cur = -1;  // block-sparse: this tile's current entry of the block list
+    // Block-sparse: this tile's current entry of the block list, and the number of score
+    // tiles (both tiles) listed before it, which gives the block's S buffer and phase.
+    int cur = -1, nbase = 0, prev_bits = 0, uses0 = 0, uses1 = 0;  // uses: own blocks per buffer
     for (int j = 0; ok && j < my_n; ++j) {
+      int sb = L::kBarS + t, sp = j & 1, pb = L::kBarP + t;
       if constexpr (SPARSE) {
-        do ++cur;
-        while (cur < nu - 1 && !(blist[cur] & (1u << (14 + t))));
+        do {
+          nbase += prev_bits;
+          ++cur;
+          prev_bits = __popc(static_cast<uint32_t>(blist[cur]) >> 14);
+        } while (cur < nu - 1 && !(blist[cur] & (1u << (14 + t))));
+        const int n = nbase + ((t == 1 && (blist[cur] & (1u << 14))) ? 1 : 0);
+        const int bsel = n & 1;
+        sb = (t ? L::kBarSX : L::kBarS) + bsel;
+        sp = (bsel ? uses1 : uses0) & 1;
+        if (bsel) ++uses1; else ++uses0;
+        pb = L::kBarP + bsel;
+        tS = tmem + L::tm_s(bsel) + lane_off;
       }
-      if (!warp_wait_bounded(bar(L::kBarS + t), j & 1, abort_flag, wait_site(1, L::kBarS + t, j))) {
+      if (!warp_wait_bounded(bar(sb), sp, abort_flag, wait_site(1, sb, j))) {
         ok = false;
         break;
       }
@@ -713,7 +742,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       r_run = r_run * alpha + (lsum + pmax_rounding(smax, sl2, m_use, ppmax));
       m_run = m_new;
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O was last written by P V of block j-1, which completed before S_j was ready.
+        // O was last written by P V of block j-1.  Dense: it completed before S_j was
+        // ready.  Block-sparse: S_j may have been computed ahead of it, so wait for it.
+        if constexpr (SPARSE) {
+          if (!warp_wait_bounded(bar(L::kBarPV + t), (j - 1) & 1, abort_flag, wait_site(1, L::kBarPV + t, j))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+        }
         const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -732,7 +769,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(L::kBarP + t));  // one arrival per warp
+      if (lane == 0) mbar_arrive(bar(pb));  // one arrival per warp
     }
 
     // ---- epilogue: O / l -> bf16 -> shared memory (this tile's Q slot) -> TMA store.  Two
