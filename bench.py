@@ -18,6 +18,10 @@ Decode workloads (--workload decode_*) time one fa_decode call per step (new que
 against a resident key/value cache, split over the cache and merged); their metric is
 the cache-read bandwidth in GB/s against the measured HBM copy peak.
 
+The `e2e` leg runs the same steps through the public binding with each step's inputs copied
+from pinned host memory and its results copied back, overlapped across neighbouring steps
+on three streams (input copy, kernels, result copy) with two device buffer sets.
+
 Rank 0 prints one JSON line.  Under torchrun each rank (one GPU each) processes its own
 shard of a global batch of N x B sequences with the unchanged kernels (no collective on
 the data path); the timed region is bracketed by barriers and the slowest rank's time is
@@ -45,6 +49,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd+bwd TFLOP/s at 1 B200 and % of dense-BF16 tensor peak"
+E2E_OVERLAP = ("each step's inputs host->device, its kernels and its results device->host on three "
+               "streams, overlapping neighbouring steps, with two device buffer sets")
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
@@ -179,6 +185,59 @@ def _oracle_sample(w, heads: int, seed: int):
         from exact_io_aware_83_b200.inputs import blocksparse_pairs
         flops = 4.0 * blocksparse_pairs(bm, w.N, w.causal) * w.d * (3.5 if w.backward else 1.0)
     return dt, flops
+
+
+def _e2e_pipelined(host_in, dev_in, dev_out, host_out, compute, n_steps, n_warm, barrier):
+    """End-to-end time (ms) of `n_steps` steps through the public API, every step copying its
+    inputs from pinned host memory to the device and its results back.  Two sets of device
+    buffers alternate, and three streams overlap step i's input copy, step i-1's kernels and
+    step i-2's result copy (as a training loop prefetches its next batch); events order the
+    reuse of each buffer set.  host_in: pinned inputs (one set, re-sent every step);
+    dev_in / dev_out / host_out: two sets each; compute(slot) launches one step's kernels on
+    the current stream over set `slot`."""
+    import torch
+    h2d, comp, d2h = (torch.cuda.Stream() for _ in range(3))
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_done = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def one(i):
+        sl = i % 2
+        if i >= 2:
+            h2d.wait_event(ev_done[sl])        # step i-2's kernels have read this input set
+        with torch.cuda.stream(h2d):
+            for dev, hst in zip(dev_in[sl], host_in):
+                dev.copy_(hst, non_blocking=True)
+            ev_in[sl].record(h2d)
+        comp.wait_event(ev_in[sl])
+        if i >= 2:
+            comp.wait_event(ev_out[sl])        # step i-2's results have left this output set
+        with torch.cuda.stream(comp):
+            compute(sl)
+            ev_done[sl].record(comp)
+        d2h.wait_event(ev_done[sl])
+        with torch.cuda.stream(d2h):
+            for hst, dev in zip(host_out[sl], dev_out[sl]):
+                hst.copy_(dev, non_blocking=True)
+            ev_out[sl].record(d2h)
+
+    for i in range(n_warm):
+        one(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(h2d)
+    for i in range(n_steps):
+        one(i)
+    # the last result copy ends the region; wait for every stream
+    d2h.wait_stream(h2d)
+    d2h.wait_stream(comp)
+    e1.record(d2h)
+    torch.cuda.synchronize()
+    barrier()
+    return e0.elapsed_time(e1)
 
 
 def _cores():
@@ -382,30 +441,22 @@ def run_ours_varlen(args, w):
     value = step_flops * args.steps * world / (ms / 1e3) / 1e12
 
     pin = lambda t: t.pin_memory()
-    qh, kh, vh, doh = (pin(t) for t in host[:4])
-    outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (o, lse, dq, dk, dv)]
+    host_in = [pin(t) for t in host[:4]]
+    outs = [o, lse, dq, dk, dv]
+    dev_in = [[q, k, v, do], [torch.empty_like(t) for t in (q, k, v, do)]]
+    dev_out = [outs, [torch.empty_like(t) for t in outs]]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs] for _ in range(2)]
 
-    def e2e_step():
-        q.copy_(qh, non_blocking=True)
-        k.copy_(kh, non_blocking=True)
-        v.copy_(vh, non_blocking=True)
-        do.copy_(doh, non_blocking=True)
-        step()
-        for hst, dev in zip(outs, (o, lse, dq, dk, dv)):
-            hst.copy_(dev, non_blocking=True)
+    def compute(sl):
+        qq, kk, vv, dd = dev_in[sl]
+        oo, ll, gq, gk, gv = dev_out[sl]
+        fa.fwd_varlen(qq, kk, vv, cq, ck, mx, mx, causal=w.causal, scale=w.scale, out=oo, lse=ll)
+        fa.bwd_varlen(qq, kk, vv, oo, ll, dd, cq, ck, mx, mx, causal=w.causal, scale=w.scale,
+                      workspace=ws, dq=gq, dk=gk, dv=gv)
 
-    e2e_steps = max(3, args.steps // 10)
-    for _ in range(2):
-        e2e_step()
-    barrier()
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_steps = max(8, args.steps // 10)
+    e2e_ms = max_over_ranks(_e2e_pipelined(host_in, dev_in, dev_out, host_out, compute, e2e_steps, 2,
+                                           barrier))
     nb = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
 
     peaks, peak_src = _peaks()
@@ -428,7 +479,7 @@ def run_ours_varlen(args, w):
         "kernels": kernels,
         "e2e": {"value": step_flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12, "unit": UNIT,
                 "h2d_bytes_per_step": nb(q, k, v, do), "d2h_bytes_per_step": nb(o, lse, dq, dk, dv),
-                "steps": e2e_steps},
+                "steps": e2e_steps, "overlap": E2E_OVERLAP},
         "gpu_launches": args.steps * 4,
         "clocks": clocks,
     }
@@ -478,13 +529,16 @@ def run_ours(args, w):
     bmh = w.block_mask()
     bmd = None if bmh is None else bmh.cuda()
 
-    def step():
+    def run(q, k, v, do, o, lse, dq, dk, dv, bm):
         fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, window=w.window,
-               dropout_p=w.dropout_p, seed=w.dropout_seed, block_mask=bmd)
+               dropout_p=w.dropout_p, seed=w.dropout_seed, block_mask=bm)
         if w.backward:
             fa.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws, dq=dq,
                    dk=dk, dv=dv, window=w.window, dropout_p=w.dropout_p, seed=w.dropout_seed,
-                   block_mask=bmd)
+                   block_mask=bm)
+
+    def step():
+        run(q, k, v, do, o, lse, dq, dk, dv, bmd)
 
     for _ in range(args.warmup):
         step()
@@ -522,47 +576,30 @@ def run_ours(args, w):
 
     # ---- end to end through the public API: pinned host inputs in, results back to host
     pin = lambda t: t.pin_memory()
-    qh_p, kh_p, vh_p, doh_p = (pin(t) for t in (qh, kh, vh, doh))
-    bmh_p = None if bmh is None else pin(bmh)
-    oh = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    lseh = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    dqh = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
-    dkh = torch.empty(dk.shape, dtype=dk.dtype).pin_memory()
-    dvh = torch.empty(dv.shape, dtype=dv.dtype).pin_memory()
+    ins = [qh, kh, vh] + ([doh] if w.backward else []) + ([] if bmh is None else [bmh])
+    host_in = [pin(t) for t in ins]
+    outs = [o, lse] + ([dq, dk, dv] if w.backward else [])
+    dev_in = [[q, k, v] + ([do] if w.backward else []) + ([] if bmd is None else [bmd]),
+              [torch.empty_like(t, device="cuda") for t in ins]]
+    dev_out = [outs, [torch.empty_like(t) for t in outs]]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs] for _ in range(2)]
 
-    def e2e_step():
-        q.copy_(qh_p, non_blocking=True)
-        k.copy_(kh_p, non_blocking=True)
-        v.copy_(vh_p, non_blocking=True)
+    def compute(sl):
+        di, do_ = dev_in[sl], dev_out[sl]
+        qq, kk, vv = di[0], di[1], di[2]
+        dd = di[3] if w.backward else None
+        bm = di[-1] if bmd is not None else None
         if w.backward:
-            do.copy_(doh_p, non_blocking=True)
-        if bmd is not None:
-            bmd.copy_(bmh_p, non_blocking=True)
-        step()
-        oh.copy_(o, non_blocking=True)
-        lseh.copy_(lse, non_blocking=True)
-        if w.backward:
-            dqh.copy_(dq, non_blocking=True)
-            dkh.copy_(dk, non_blocking=True)
-            dvh.copy_(dv, non_blocking=True)
+            run(qq, kk, vv, dd, do_[0], do_[1], do_[2], do_[3], do_[4], bm)
+        else:
+            run(qq, kk, vv, None, do_[0], do_[1], None, None, None, bm)
 
-    e2e_steps = max(3, args.steps // 10)
-    for _ in range(2):
-        e2e_step()
-    barrier()
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_steps = max(8, args.steps // 10)
+    e2e_ms = max_over_ranks(_e2e_pipelined(host_in, dev_in, dev_out, host_out, compute, e2e_steps, 2,
+                                           barrier))
     nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
-    h2d = nbytes(q, k, v, do) if w.backward else nbytes(q, k, v)
-    if bmd is not None:
-        h2d += nbytes(bmd)
-    d2h = nbytes(o, lse, dq, dk, dv) if w.backward else nbytes(o, lse)
+    h2d = nbytes(*dev_in[0])
+    d2h = nbytes(*outs)
     e2e_value = step_flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_src = _peaks()
@@ -596,7 +633,7 @@ def run_ours(args, w):
                      "peak_source": f"{peak_src} bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps, "overlap": E2E_OVERLAP},
         "gpu_launches": args.steps * (1 + (3 if w.backward else 0)),
         "clocks": clocks,
     }
