@@ -52,6 +52,7 @@ METRIC = "attention fwd+bwd TFLOP/s at 1 B200 and % of dense-BF16 tensor peak"
 E2E_OVERLAP = ("each step's inputs host->device, its kernels and its results device->host on three "
                "streams, overlapping neighbouring steps, with two device buffer sets")
 UNIT = "TFLOP/s"
+NOMINAL_BF16_TFLOPS = 2250.0  # NVIDIA's dense bf16 figure for one B200, for context only
 FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
 
 
@@ -621,6 +622,7 @@ def run_ours(args, w):
     for kname, kd in kernels.items():
         kd["frac_of_burst_peak"] = kd["tflops"] / peak
         kd["frac_of_sustained_peak"] = kd["tflops"] / float(peaks["bf16_tflops_sustained"])
+        kd["frac_of_nominal_peak"] = kd["tflops"] / NOMINAL_BF16_TFLOPS
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
