@@ -368,12 +368,23 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   p.drop = drop ? *drop : fa::DropCfg{};
   if (mode != fa::kAttnSparse) p.bmask = nullptr;
   const int tslot = timer_start(0, s);
+  // Unit order (unit_order): dense causal attention runs its heavy units first - every unit
+  // alone once a head has at most 16 query blocks, two tiers beyond that (where one head's
+  // K/V no longer fits many times over in L2); other variants, whose units are alike or
+  // ragged per sequence, stay head-major.  Measured on B200 (forward, TFLOP/s): gpt_2k
+  // 660 -> 724, 8k causal 984 -> 1040, GQA 4k 983 -> 1006.
+  auto order = [&](int levels) {
+    if (mode != fa::kAttnCausal) return levels;
+    return p.nqb <= 16 ? 1 : (levels + 1) / 2;
+  };
   if (d == 256) {
     p.pair_heads = 0;
+    p.tsz = order(p.nqb);
     const unsigned units = static_cast<unsigned>(p.B) * p.Hq * p.nqb;
     launch_fwd_mode<256>(tq, tk, tv, to, p, units, mode, drop != nullptr, s);
   } else {
     p.pair_heads = (g % 2 == 0) ? 1 : 0;
+    p.tsz = order(p.pair_heads ? p.nqb : (p.nqb + 1) / 2);
     const unsigned units = p.pair_heads ? static_cast<unsigned>(p.B) * (p.Hq / 2) * p.nqb
                                         : static_cast<unsigned>(p.B) * p.Hq * ((p.nqb + 1) / 2);
     if (d == 64)

@@ -111,6 +111,21 @@ struct DropCfg {
 // causal mask); only enabled blocks are visited.
 constexpr int kAttnFull = 0, kAttnCausal = 1, kAttnGeneral = 2, kAttnSparse = 3;
 
+// Order of the work units of a grid: `heads` rows of `levels` units each, level 0 the
+// heaviest (the most key blocks under a causal mask).  Levels are cut into tiers of `tsz`
+// levels; the tiers run heaviest first, and inside a tier one head's units are consecutive,
+// so the CTAs that run together share that head's K/V (or Q/dO) in L2.  tsz = levels is
+// head-major order, tsz = 1 pure heaviest-first.  The hardware starts CTAs in index order,
+// so heavy units never start last and leave a long tail.
+__device__ __forceinline__ void unit_order(int u, int heads, int levels, int tsz, int &head, int &level) {
+  const int per_tier = heads * tsz;
+  const int t = u / per_tier;
+  const int v = u - t * per_tier;
+  const int cnt = min(tsz, levels - t * tsz);
+  head = v / cnt;
+  level = t * tsz + v % cnt;
+}
+
 // The sequence a CTA works on.  Dense: Lq = Lk = N.  Packed: the lengths of sequence b and
 // its first rows in the packed tensors.  The keys are aligned to the END of the queries:
 // query i sits at key position c = i + dlt, dlt = Lk - Lq (0 for self-attention), and sees

@@ -51,6 +51,7 @@ struct FwdParams {
   float sl2;              // scale * log2(e)
   DropCfg drop;           // dropout (kernels instantiated with DROP only)
   const uint8_t *bmask;   // block-sparse: [B, Hq, nqb, nqb] 0/1 over 128 x 128 blocks
+  int tsz;                // unit order: levels per tier (see unit_order)
 };
 
 // Blocks of KB keys [lo, hi] that some row q0 .. min(q0 + 127, Lq - 1) of a query tile can
@@ -296,23 +297,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   int b, h[2], qb[2];
   bool valid[2];
   {
-    int u = blockIdx.x;
+    const int u = blockIdx.x;
+    int head, level;
     if (p.pair_heads) {
       const int hp_count = p.Hq / 2;
-      const int q = p.nqb - 1 - (u % p.nqb);
-      u /= p.nqb;
-      const int hp = u % hp_count;
-      b = u / hp_count;
+      unit_order(u, p.B * hp_count, p.nqb, p.tsz, head, level);
+      const int q = p.nqb - 1 - level;
+      const int hp = head % hp_count;
+      b = head / hp_count;
       h[0] = 2 * hp;
       h[1] = 2 * hp + 1;
       qb[0] = qb[1] = q;
       valid[0] = valid[1] = true;
     } else {
       const int npairs = (p.nqb + 1) / 2;
-      const int pi = npairs - 1 - (u % npairs);
-      u /= npairs;
-      h[0] = h[1] = u % p.Hq;
-      b = u / p.Hq;
+      unit_order(u, p.B * p.Hq, npairs, p.tsz, head, level);
+      const int pi = npairs - 1 - level;
+      h[0] = h[1] = head % p.Hq;
+      b = head / p.Hq;
       qb[0] = 2 * pi;
       qb[1] = 2 * pi + 1;
       valid[0] = true;

@@ -80,12 +80,13 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
 
-  // ---- unit = (b, h, query block), last query blocks (longest under a causal mask) first
-  int u = blockIdx.x;
-  const int qb = p.nqb - 1 - (u % p.nqb);
-  u /= p.nqb;
-  const int h = u % p.Hq;
-  const int b = u / p.Hq;
+  // ---- unit = (b, h, query block), ordered by unit_order (last query blocks, the longest
+  // under a causal mask, are level 0)
+  int head, level;
+  unit_order(blockIdx.x, p.B * p.Hq, p.nqb, p.tsz, head, level);
+  const int qb = p.nqb - 1 - level;
+  const int h = head % p.Hq;
+  const int b = head / p.Hq;
   const int kvh = h / (p.Hq / p.Hkv);
   constexpr bool GEN = MODE == kAttnGeneral;
   constexpr bool SPARSE = MODE == kAttnSparse;
