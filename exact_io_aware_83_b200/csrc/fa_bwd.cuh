@@ -854,12 +854,11 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.drop = drop ? *drop : DropCfg{};
   p.bmask = bmask;
-  // Unit order (unit_order): dense causal attention over at most 16 key blocks runs in three
-  // tiers, heavy key blocks first (gpt_2k backward call 537 -> 557 TFLOP/s on B200); longer
-  // sequences and the other variants stay head-major, which keeps the Q / dO / dQ rows a
-  // head's CTAs share in L2 (three tiers cost 2% at 8k).
-  const bool causal_dense = !pk && !bmask && left < 0 && right == 0;
-  p.tsz = (causal_dense && p.nkb <= 16) ? (p.nkb + 2) / 3 : p.nkb;
+  // Unit order (unit_order): head-major, so the CTAs of one head, which stream the same Q,
+  // dO and dQ rows, run together and share them in L2.  Heavy-first tiers were measured on
+  // B200: at gpt_2k three tiers made the backward 2% faster but raised its DRAM traffic from
+  // 630 to 977 MB per launch (each tier re-reads every head's rows); at 8k they were slower.
+  p.tsz = p.nkb;
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
   if (grid > 0) {
