@@ -807,7 +807,7 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                         int Hkv, int N, int left, int right, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
                         TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk, const DropCfg *drop,
-                        const uint8_t *bmask) {
+                        const uint8_t *bmask, int tiers) {
   const long long rows = pk ? static_cast<long long>(pk->total_q) * Hq : static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
   float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
@@ -854,11 +854,8 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.drop = drop ? *drop : DropCfg{};
   p.bmask = bmask;
-  // Unit order (unit_order): head-major, so the CTAs of one head, which stream the same Q,
-  // dO and dQ rows, run together and share them in L2.  Heavy-first tiers were measured on
-  // B200: at gpt_2k three tiers made the backward 2% faster but raised its DRAM traffic from
-  // 630 to 977 MB per launch (each tier re-reads every head's rows); at 8k they were slower.
-  p.tsz = p.nkb;
+  // Unit order (unit_order): `tiers` tiers of key-block levels (1: head-major).
+  p.tsz = (p.nkb + tiers - 1) / tiers;
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
   if (grid > 0) {
@@ -890,16 +887,16 @@ inline int bwd_launch(const void *q, const void *k, const void *v, const void *o
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                       int Hkv, int N, int d, int left, int right, float scale, cudaStream_t s, Enc enc,
                       TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk = nullptr,
-                      const DropCfg *drop = nullptr, const uint8_t *bmask = nullptr) {
+                      const DropCfg *drop = nullptr, const uint8_t *bmask = nullptr, int tiers = 1) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
     return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk, drop, bmask);
+                                    scale, s, e, tstart, tstop, pk, drop, bmask, tiers < 1 ? 1 : tiers);
   if (d == 128)
     return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                      scale, s, e, tstart, tstop, pk, drop, bmask);
+                                      scale, s, e, tstart, tstop, pk, drop, bmask, tiers < 1 ? 1 : tiers);
   return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk, drop, bmask);
+                                    scale, s, e, tstart, tstop, pk, drop, bmask, tiers < 1 ? 1 : tiers);
 }
 
 }  // namespace fa
