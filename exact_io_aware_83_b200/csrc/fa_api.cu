@@ -368,14 +368,16 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   p.drop = drop ? *drop : fa::DropCfg{};
   if (mode != fa::kAttnSparse) p.bmask = nullptr;
   const int tslot = timer_start(0, s);
-  // Unit order (unit_order): dense causal attention runs its heavy units first - every unit
-  // alone once a head has at most 16 query blocks, two tiers beyond that (where one head's
-  // K/V no longer fits many times over in L2); other variants, whose units are alike or
-  // ragged per sequence, stay head-major.  Measured on B200 (forward, TFLOP/s): gpt_2k
-  // 660 -> 724, 8k causal 984 -> 1040, GQA 4k 983 -> 1006.
+  // Unit order (unit_order), chosen from B200 measurements (forward TFLOP/s): dense causal
+  // attention runs its heavy units first - every level alone up to 16 query blocks, two
+  // tiers beyond (gpt_2k 660 -> 724, 8k causal 984 -> 1040, GQA 4k 983 -> 1006); a band or a
+  // block mask goes level by level (window_8k_1k 578 -> 611, blocksparse_8k 560 -> 614);
+  // full attention and packed sequences stay head-major (packed: 680 head-major, 669-679
+  // tiered).
   auto order = [&](int levels) {
-    if (mode != fa::kAttnCausal) return levels;
-    return p.nqb <= 16 ? 1 : (levels + 1) / 2;
+    if (mode == fa::kAttnCausal) return p.nqb <= 16 ? 1 : (levels + 1) / 2;
+    if (mode == fa::kAttnSparse || (mode == fa::kAttnGeneral && p.cu_q == nullptr)) return 1;
+    return levels;
   };
   if (d == 256) {
     p.pair_heads = 0;
@@ -433,13 +435,17 @@ bool normalise_window_varlen(int w, int max_q, int max_k, int *out) {
   return true;
 }
 
-// Backward unit order for dense causal attention: over at most 16 key blocks the work runs
-// in three tiers of key blocks, heavy first, so no heavy unit starts last.  Measured on
-// B200 at gpt_2k: main kernel 615 -> 649 TFLOP/s, at the price of DRAM traffic 628 -> 977 MB
-// per launch (each tier streams every head's Q / dO / dQ rows again); at 8k the tiers were
-// 2% slower, so longer sequences stay head-major (one head's CTAs together in L2).
+// Backward unit order (tiers of key-block levels for unit_order), from B200 measurements.
+// Dense causal attention over at most 16 key blocks runs in three tiers, heavy first, so
+// no heavy unit starts last: gpt_2k main kernel 615 -> 649 TFLOP/s, at the price of DRAM
+// traffic 628 -> 977 MB per launch (each tier streams every head's Q / dO / dQ rows
+// again); at 8k the tiers were 2% slower, so longer sequences stay head-major (one head's
+// CTAs together in L2).  A band goes level by level (window_8k_1k backward call 518 -> 541);
+// full attention and (in the callers) block masks and packed sequences stay head-major.
 int bwd_tiers(int N, int left, int right) {
-  return (left < 0 && right == 0 && (N + 127) / 128 <= 16) ? 3 : 1;
+  if (left < 0 && right < 0) return 1;
+  if (left < 0 && right == 0) return (N + 127) / 128 <= 16 ? 3 : 1;
+  return 1 << 20;
 }
 
 // Block-sparse limits: the forward keeps each CTA's key-block list in shared memory (at most
