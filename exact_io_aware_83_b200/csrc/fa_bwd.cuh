@@ -10,13 +10,15 @@
 //   dS_ij  = P_ij (dP_ij - Delta_i)
 //   dV_j   = sum_i P_ij do_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
 // (dK, dV summed over the query heads that share a K/V head), with P_ij = 0 for keys
-// outside query i's window i - left <= j <= i + right (causal: left unlimited, right 0).
+// outside query i's window i - left <= j <= i + right (causal: left unlimited, right 0)
+// or, block-sparse, outside the enabled 128 x 128 blocks of the query head's mask.
 //
 // Three kernels on one stream:
 //  1. fa_bwd_pre:  Delta_i = <dO_i, O_i> (fp32) and a zeroed fp32 dQ accumulator.
 //  2. fa_bwd_main: one CTA per (b, K/V head, 128-key block).  It keeps K_j and V_j in
 //     shared memory and dK_j, dV_j in tensor memory, and walks every (query head of the
-//     group, 64-row query block) that can see the key block (a window skips the others):
+//     group, 64-row query block) that can see the key block (a window or a block mask
+//     skips the others):
 //        S^T  = K Q_i^T        (tcgen05, TMEM)      P^T = exp2(S^T scale log2e - LSE2_i)
 //        dP^T = V dO_i^T       (tcgen05, TMEM)      dS^T = P^T (dP^T - Delta_i)
 //        dV  += P^T dO_i       (P^T read from TMEM as the A operand)

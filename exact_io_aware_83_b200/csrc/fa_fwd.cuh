@@ -4,9 +4,10 @@
 //   O_i = sum_j softmax_j(scale * q_i . k_j) v_j,  LSE_i = ln sum_j exp(scale * q_i . k_j)
 // where J(i) is every key, or the local window i - left <= j <= i + right (causal
 // attention is left unlimited, right = 0; the "FlashAttention1" Q&A's scaling question,
-// item 4, pairs the method with local attention).  Key blocks no row of a tile can see
-// are skipped, not masked.
-// with the score matrix processed one 128 x 128 tile at a time and the online-softmax
+// item 4, pairs the method with local attention), or the keys of the enabled 128 x 128
+// blocks of a block mask (block-sparse attention, named in the deep-dive page's closing
+// paragraph).  Key blocks no row of a tile can see are skipped, not masked.  The score
+// matrix is processed one 128 x 128 tile at a time with the online-softmax
 // recurrence of the "FlashAttention1" Q&A page (question on computing the softmax,
 // items 1-3): a running row maximum m, a running sum l, and a rescale of the partial
 // output by exp(m_old - m_new) when a new key block raises the maximum (the deep-dive
@@ -17,7 +18,8 @@
 //  * One CTA owns two 128-row query tiles that share every K/V block: either two query
 //    blocks of one head, or - for grouped-query attention with an even group - the same
 //    query block of two heads that share a K/V head, so each K/V tile is loaded once for
-//    both.  Work units are ordered so the longest causal units start first.
+//    both.  Work units are ordered by unit_order (fa_common.cuh), heavy units first
+//    where that shortens the tail.
 //  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and tile 1
 //    (one query row per thread, the row's TMEM lane); warp 8 allocates tensor memory and
 //    issues every tcgen05.mma from one lane; warp 9 issues the TMA loads from one lane;
@@ -28,7 +30,8 @@
 //  * K and V blocks stream through a ring of shared-memory slots filled by TMA in the
 //    order K_0, V_0, K_1, V_1, ...; 128-byte swizzled tiles feed the tensor core directly.
 //  * The two tiles ping-pong: while the softmax warps of one tile work, the tensor core
-//    runs the other tile's P V and next Q K^T.
+//    runs the other tile's P V and next Q K^T.  (Block-sparse: the two tiles' masks differ,
+//    so the two S buffers are shared and a tile can also run a block ahead on its own.)
 //  * exp is evaluated as exp2 with scale*log2(e) folded into one FMA.  The running max
 //    used as the exponent offset is only moved when a row's max rises by more than 2^8
 //    (the recurrence is exact for any offset; keeping it avoids rescaling O for most
