@@ -13,11 +13,16 @@ Entry points mirror the C ABI names:
 * :func:`fa_fwd_varlen` / :func:`fa_bwd_varlen` - packed variable-length sequences
   ([total, H, d] rows, [B+1] offsets; query and key lengths may differ, the band being
   aligned to the end of each sequence);
+* :func:`fa_fwd_dropout` / :func:`fa_bwd_dropout` - attention dropout with a
+  Philox4x32-10 keep mask regenerated in the backward;
+* :func:`fa_fwd_blocksparse` / :func:`fa_bwd_blocksparse` - block-sparse attention over a
+  per-head 0/1 mask of 128 x 128 blocks (with or without the causal mask);
 * :func:`fa_decode` / :func:`fa_merge` - a few new query rows against a long key/value
   cache, split over the cache, and the merge of partial results;
 * :func:`fwd` / :func:`bwd` / :func:`fwd_varlen` / :func:`bwd_varlen` / :func:`decode` /
-  :func:`merge` - tensor conveniences that
-  allocate outputs with torch (``window=(left, right)`` selects local attention);
+  :func:`merge` - tensor conveniences that allocate outputs with torch
+  (``window=(left, right)`` selects local attention, ``dropout_p`` / ``seed`` dropout,
+  ``block_mask`` block-sparse attention);
 * :func:`fa_bwd_workspace_bytes`, :func:`fa_device_status`, :func:`fa_status_string`.
 """
 from __future__ import annotations
