@@ -134,8 +134,26 @@ def check_bwd(dq, dk, dv, q, k, v, do, causal, scale):
             assert errs[name] <= O_TOL, f"{name} should vanish, max |x| = {errs[name]}"
             continue
         errs[name] = _rel_fro(x, ref)
-        assert errs[name] <= GRAD_TOL, f"{name} relative Frobenius error {errs[name]}"
+        worst = _worst_head(x, ref)
+        errs[name + " worst (b, h)"] = worst
+        assert errs[name] <= GRAD_TOL, (f"{name} relative Frobenius error {errs[name]}; worst "
+                                        f"(b, h) = {worst[1]} at {worst[0]:.3e}")
+    print(" ".join(f"{k}={v}" for k, v in errs.items()))
     return errs
+
+
+def _worst_head(x, ref):
+    """(relative Frobenius error, (b, h)) of the worst [b, h] slice whose reference is not
+    zero: reported beside the whole-tensor error."""
+    worst = (0.0, None)
+    for b in range(ref.shape[0]):
+        for h in range(ref.shape[1]):
+            nr = np.linalg.norm(ref[b, h])
+            if nr > 1e-12:
+                e = float(np.linalg.norm(x[b, h] - ref[b, h]) / nr)
+                if e > worst[0]:
+                    worst = (e, (b, h))
+    return worst
 
 
 # ----------------------------------------------------------------------------- small cases
