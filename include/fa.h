@@ -214,7 +214,7 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, co
  *        ignored whatever their byte.
  * A row whose blocks are all disabled gets O = 0 and LSE = -inf.  Limits: nb <= 4096, and
  * (Hq / Hkv) * ceil(nb / 32) * 4 bytes of per-key-block bitmap for the backward within
- * its shared-memory budget (8192 bytes for d = 64 and 128, about 1.3 KB for d = 256);
+ * its shared-memory budget (8192 bytes for d = 64 and 128, 1392 bytes for d = 256);
  * larger sizes return FA_ERR_UNSUPPORTED (checked by both calls, so a forward that runs
  * always has a backward).  A NULL mask or a causal flag other than 0/1 is
  * FA_ERR_INVALID_ARG.
