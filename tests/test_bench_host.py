@@ -1,0 +1,82 @@
+"""Host logic of bench.py that needs no GPU: the DRAM-traffic lookup (an entry is used
+only while its kernel sources are unchanged), the clock-sample summary (only samples
+inside the timed region count; throttle reasons are collected), and the workload config
+that the JSON line carries."""
+import datetime as dt
+import hashlib
+import json
+import os
+
+import bench
+from exact_io_aware_83_b200.inputs import DECODE_WORKLOADS, WORKLOADS
+
+
+def _write_traffic(root, source_text, recorded_text):
+    os.makedirs(os.path.join(root, "profiles"))
+    os.makedirs(os.path.join(root, "src"))
+    with open(os.path.join(root, "src", "k.cuh"), "w") as f:
+        f.write(source_text)
+    entry = {"kernel": "k", "workload": "w", "dram_bytes_per_launch": 1234,
+             "sources": ["src/k.cuh"],
+             "sources_sha256": [hashlib.sha256(recorded_text.encode()).hexdigest()]}
+    with open(os.path.join(root, "profiles", "dram_traffic.json"), "w") as f:
+        json.dump({"entries": [entry]}, f)
+
+
+def test_traffic_used_while_the_source_is_unchanged(tmp_path, monkeypatch):
+    _write_traffic(str(tmp_path), "kernel v1", "kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._profile_traffic("k", "w") == 1234
+    assert bench._profile_traffic("k", "other") is None
+    assert bench._profile_traffic("other", "w") is None
+
+
+def test_traffic_dropped_once_the_source_changes(tmp_path, monkeypatch):
+    _write_traffic(str(tmp_path), "kernel v2", "kernel v1")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench._profile_traffic("k", "w") is None
+
+
+def test_committed_traffic_entries_name_existing_sources():
+    with open(os.path.join(bench.ROOT, "profiles", "dram_traffic.json")) as f:
+        entries = json.load(f)["entries"]
+    assert entries
+    for e in entries:
+        assert e["dram_bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
+        for src in e["sources"]:
+            assert os.path.exists(os.path.join(bench.ROOT, src)), src
+
+
+def test_clock_summary_keeps_the_timed_region_only(tmp_path):
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.file = open(tmp_path / "c.csv", "w+")
+    s.proc = object()  # stands for the nvidia-smi process
+    t0 = dt.datetime(2026, 1, 1, 12, 0, 0)
+    s.t0, s.t1 = t0, t0 + dt.timedelta(seconds=1)
+    rows = [
+        (-0.5, 900, "Not Active", "Not Active"),     # before the region: ignored
+        (0.1, 1900, "Not Active", "Active"),         # sw_power_cap active
+        (0.3, 1950, "Not Active", "Not Active"),
+        (0.6, 1930, "Not Active", "Not Active"),
+        (1.5, 300, "Active", "Not Active"),          # after the region: ignored
+    ]
+    for off, mhz, hw, cap in rows:
+        ts = (t0 + dt.timedelta(seconds=off)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        s.file.write(f"{ts}, {mhz}, 1965, 900.0, 0x0, {hw}, Not Active, Not Active, {cap}\n")
+    out = s.summary()
+    assert out["samples"] == 3
+    assert out["sm_mhz"] == 1930
+    assert out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["sw_power_cap"]
+
+
+def test_config_names_the_workload():
+    c = bench._config(WORKLOADS["gpt_2k_causal"], 1)
+    assert c["workload"] == "gpt_2k_causal" and c["global_batch"] == 8 and c["causal"]
+    c = bench._config(WORKLOADS["blocksparse_8k_causal"], 2)
+    assert c["global_batch"] == 4 and c["parallelism"] == "dp2"
+    assert c["block_mask"]["density"] == 0.25 and 0.2 < c["block_mask"]["enabled_pairs_share_of_causal"] < 0.35
+    c = bench._config(WORKLOADS["window_8k_1k"], 1)
+    assert c["window"] == [1023, 0]
+    c = bench._config(DECODE_WORKLOADS["decode_64k_gqa"], 1)
+    assert c["cache_len"] == 65536 and c["passes"] == "decode"
