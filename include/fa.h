@@ -325,7 +325,8 @@ int fa_device_status(void *stream);
 
 /*
  * Kernel timing for benchmarks.  fa_kernel_timing(1) resets the counters and makes every
- * later fa_fwd / fa_bwd / fa_decode call (and their window forms) in this process record
+ * later fa_fwd / fa_bwd / fa_decode call (and their window, varlen, dropout and
+ * block-sparse forms, and fa_bwd_noalloc) in this process record
  * a pair of CUDA events (created by the
  * library, no device memory) around its main attention kernel, on the call's stream;
  * fa_kernel_timing(0) stops recording.  fa_kernel_time_ms(which, &ms, &launches)
