@@ -310,6 +310,8 @@ def _block_mask(block_mask, B, Hq, N, win, dropout_p):
     if block_mask is None:
         return None
     nb = (N + 127) // 128
+    if block_mask.dtype == torch.bool:
+        block_mask = block_mask.view(torch.uint8)  # one byte, 0 or 1, per block
     if (not block_mask.is_cuda or block_mask.dtype != torch.uint8 or not block_mask.is_contiguous()
             or tuple(block_mask.shape) != (B, Hq, nb, nb)):
         raise ValueError(f"block_mask must be a contiguous uint8 CUDA tensor [{B}, {Hq}, {nb}, {nb}]")
@@ -324,8 +326,8 @@ def fwd(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse
     ``window=(left, right)``: local attention, key j visible to query i iff
     i - left <= j <= i + right (-1 = unlimited on that side).  ``dropout_p`` > 0: attention
     dropout with the Philox4x32-10 mask of ``seed`` (full or causal attention).
-    ``block_mask``: block-sparse attention, uint8 [B, Hq, ceil(N/128), ceil(N/128)] on the
-    GPU, nonzero = the 128 x 128 block is computed (with or without ``causal``)."""
+    ``block_mask``: block-sparse attention, uint8 (or bool) [B, Hq, ceil(N/128), ceil(N/128)]
+    on the GPU, nonzero = the 128 x 128 block is computed (with or without ``causal``)."""
     import torch
     win = _window(causal, window)
     for t, n in ((q, "q"), (k, "k"), (v, "v")):

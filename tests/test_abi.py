@@ -271,6 +271,17 @@ def test_valid_arguments_without_a_device_report_cuda_error():
     assert fa.load().fa_merge(FAKE, FAKE, FAKE, FAKE, 2, 4, 64, None) == fa.FA_ERR_CUDA
 
 
+def test_binding_checks_the_block_mask():
+    m = torch.zeros(1, 2, 3, 3, dtype=torch.uint8)
+    with pytest.raises(ValueError):      # not on the GPU
+        fa._block_mask(m, 1, 2, 300, None, 0.0)
+    with pytest.raises(ValueError):      # wrong dtype
+        fa._block_mask(m.float(), 1, 2, 300, None, 0.0)
+    with pytest.raises(ValueError):      # wrong shape (nb = 3 for N = 300)
+        fa._block_mask(torch.zeros(1, 2, 2, 2, dtype=torch.uint8), 1, 2, 300, None, 0.0)
+    assert fa._block_mask(None, 1, 2, 300, None, 0.0) is None
+
+
 def test_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
