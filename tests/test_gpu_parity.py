@@ -1,18 +1,30 @@
 """GPU parity of the CUDA library (through the C ABI) against the fp64 oracle.
 
 Tolerances, on the same seeded bf16 inputs:
-  |O - O_ref| <= max(1e-2, ulp_bf16(O_ref)) element-wise (after the GPU's bf16 store),
+  |O - O_ref| <= 1e-2 element-wise (after the GPU's bf16 store) wherever |O_ref| < 4,
+  and above that half a bf16 spacing plus the derived pre-rounding allowance below;
   max|LSE - LSE_ref| <= 1e-3,
   ||X - X_ref||_F / ||X_ref||_F <= 2e-2 for X in {dQ, dK, dV};
 no NaN/Inf anywhere, and guard bands of sentinel values around every output buffer left
 untouched (an out-of-bounds write shows up there).
 
-Reading of the O bound: the stated 1e-2 is an absolute bound on a bf16 output, but bf16
-spaces its values 2^(e-7) apart (0.0156 in [2, 4), 0.031 in [4, 8)), so no bf16 result
-can meet 1e-2 for every |O| >= 2 -- rounding alone can cost up to half that spacing, and
-the bf16 probabilities fed to the P V product add up to about as much again.  The test
-keeps 1e-2 wherever the format can resolve it and one bf16 spacing of the reference value
-elsewhere.
+Reading of the O bound.  The stated bound is an absolute 1e-2 on a bf16 output.  bf16
+keeps 8 significant bits, so rounding the exact value to bf16 costs up to half a spacing,
+2^(e-8) for |O| in [2^e, 2^(e+1)): at most 0.0078 below 4, so 1e-2 is attainable there
+and is kept as is.  For |O| >= 4 half a spacing alone is 0.0156 or more, above 1e-2, and
+the bound becomes half a spacing plus an allowance for the error of the fp32 value before
+that rounding.  That error comes from the probabilities as the P V product sees them:
+each one is rounded to bf16 (relative error <= 2^-9) after an exp2 whose error is below
+2^-13 (the MUFU unit, or the FMA-pipe polynomial: 7.5e-5 measured over its whole reduced
+range), and O is divided by the fp32 sum of the unrounded probabilities corrected by the
+rounding of each key block's largest one.  With P_j the exact probabilities of the row,
+delta_j their relative errors (|delta_j| <= eps = 2^-9 + 2^-13) and M the corrected keys,
+    O_pre - O = [sum_j P_j delta_j (v_j - O) + sum_{j not in M} P_j delta_j O] / (1 + ...)
+so, to first order,
+    |O_pre - O| <= eps (1 + 2 eps) [sum_j P_j |v_j - O| + (1 - P_max + 2^-10) |O|] + 1e-5,
+where P_max is the row's largest probability (the corrected keys carry at least
+(1 - 2^-10) P_max between them) and 1e-5 covers the fp32 accumulation.  The tests compute
+this allowance from the oracle's probabilities for every element with |O_ref| >= 4.
 
 Small cases run the oracle on everything; the five full-size workloads are compared on
 sampled (batch, K/V-head group) slices, which the oracle computes exactly because
@@ -102,17 +114,72 @@ def bf16_spacing(x):
     return np.exp2(np.floor(np.log2(ax)) - 7)
 
 
-def o_tolerance(o_ref):
-    return np.maximum(O_TOL, bf16_spacing(o_ref))
+O_FLAT = 4.0                     # below this |O_ref|, half a bf16 spacing is <= 2^-7 < 1e-2
+P_EPS = 2.0 ** -9 + 2.0 ** -13   # relative error of one probability as P V sees it
+O_ACC = 1e-5                     # fp32 accumulation of O and the division by the sum
+
+
+def o_tolerance(o_ref, allowance=None):
+    """Element-wise bound on |O - O_ref|: 1e-2 where |O_ref| < 4, else half a bf16
+    spacing plus the pre-rounding allowance (see the module docstring).  `allowance`
+    maps the index tuple of the elements with |O_ref| >= 4 to their allowances; without
+    it (callers whose outputs never reach 4 in practice) the allowance is taken as 0,
+    which only makes the bound stricter."""
+    a = np.abs(o_ref)
+    tol = np.full(o_ref.shape, O_TOL)
+    hi = np.nonzero(a >= O_FLAT)
+    if len(hi[0]):
+        extra = np.zeros(len(hi[0])) if allowance is None else allowance(hi)
+        tol[hi] = 0.5 * bf16_spacing(a[hi] + extra) + extra + O_ACC
+    return tol
+
+
+def p_allowance(q64, k64, v64, o_ref, lse_ref, causal, scale):
+    """Allowance function for o_tolerance on dense (optionally causal) attention: for each
+    flagged element (b, h, i, c), eps (1 + 2 eps) [sum_j P_ij |v_jc - O_ic| +
+    (1 - max_j P_ij + 2^-10) |O_ic|], with P_ij = exp(scale q_i.k_j - LSE_ref_i)."""
+    g = q64.shape[1] // k64.shape[1]
+
+    def fn(idx):
+        out = np.empty(len(idx[0]))
+        rows = {}
+        for n, (b, h, i, c) in enumerate(zip(*idx)):
+            key = (b, h, i)
+            if key not in rows:
+                s = scale * (k64[b, h // g] @ q64[b, h, i])
+                if causal:
+                    s[i + 1:] = -np.inf
+                rows[key] = np.exp(s - lse_ref[b, h, i])
+            p = rows[key]
+            o = o_ref[b, h, i, c]
+            spread = float(p @ np.abs(v64[b, h // g, :, c] - o))
+            out[n] = P_EPS * (1 + 2 * P_EPS) * (spread + (1.0 - p.max() + 2.0 ** -10) * abs(o))
+        return out
+
+    return fn
+
+
+def o_error_bins(o, o_ref):
+    """Largest |O - O_ref| among elements with |O_ref| in [0, 2), [2, 4) and >= 4."""
+    diff = np.abs(o - o_ref)
+    a = np.abs(o_ref)
+    bins = {}
+    for name, m in (("[0,2)", a < 2), ("[2,4)", (a >= 2) & (a < 4)), (">=4", a >= 4)):
+        bins[name] = (float(diff[m].max()) if m.any() else None, int(m.sum()))
+    return bins
 
 
 def check_fwd(o, lse, q, k, v, causal, scale):
-    o_ref, lse_ref = oracle.attention_fwd(_f64(q), _f64(k), _f64(v), causal, scale)
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    o_ref, lse_ref = oracle.attention_fwd(q64, k64, v64, causal, scale)
     _finite(o, lse)
-    diff = np.abs(_f64(o) - o_ref)
-    excess = float(np.max(diff - o_tolerance(o_ref)))
+    o64 = _f64(o)
+    diff = np.abs(o64 - o_ref)
+    tol = o_tolerance(o_ref, p_allowance(q64, k64, v64, o_ref, lse_ref, causal, scale))
+    excess = float(np.max(diff - tol))
     err_o = float(np.max(diff))
     err_l = float(np.max(np.abs(lse.double().numpy() - lse_ref)))
+    print(f"O error by |O_ref| bin (max, count): {o_error_bins(o64, o_ref)}")
     assert excess <= 0.0, f"|O-O_ref| above tolerance by {excess} (max |O-O_ref| = {err_o})"
     assert err_l <= LSE_TOL, f"max|LSE-LSE_ref| = {err_l}"
     return err_o, err_l
@@ -259,6 +326,9 @@ def _slice_group(t, b, h0, h1):
 
 @pytest.mark.parametrize("name", list(WORKLOADS))
 def test_full_size_workloads(name):
+    """The workloads at their full sizes, in the launch configuration the benchmark times.
+    The forward is compared with the oracle on three (b, K/V head) groups, the backward on
+    two; the gradient invariants are checked on the whole tensors."""
     w = WORKLOADS[name]
     inputs = draw_workload(w)
     q, k, v = inputs[:3]
@@ -266,11 +336,13 @@ def test_full_size_workloads(name):
     _finite(o, lse)
     g = w.Hq // w.Hkv
     rng = np.random.default_rng(w.seed)
-    # Sampled (b, K/V head) groups: compare every row of the group with the oracle.
-    groups = {(0, 0), (w.B - 1, w.Hkv - 1), (int(rng.integers(w.B)), int(rng.integers(w.Hkv)))}
-    if w.N >= 8192:
-        groups = {(w.B - 1, w.Hkv - 1)}
-    for b, kh in sorted(groups):
+    # Sampled (b, K/V head) groups: the first, the last and a random one (distinct where
+    # the workload has three); every row of a sampled group is compared with the oracle.
+    cand = [(0, 0), (w.B - 1, w.Hkv - 1)]
+    while len(set(cand)) < min(3, w.B * w.Hkv):
+        cand.append((int(rng.integers(w.B)), int(rng.integers(w.Hkv))))
+    groups = list(dict.fromkeys(cand))
+    for b, kh in groups:
         hs = slice(kh * g, (kh + 1) * g)
         qs = _slice_group(q, b, hs.start, hs.stop)
         ks = _slice_group(k, b, kh, kh + 1)
@@ -281,15 +353,17 @@ def test_full_size_workloads(name):
     do = inputs[3]
     dq, dk, dv = run_bwd(q, k, v, o, lse, do, w.causal, w.scale)
     _finite(dq, dk, dv)
-    # Invariants at full size: sum_j dK_j = 0 and sum_j dV_j = sum over the group's rows of dO.
+    # Invariants at full size, per (b, K/V head, column): sum_j dK_j = 0 and sum_j dV_j =
+    # the sum of dO over the group's query rows (the probabilities of a row sum to 1).
+    # Each sum is bounded relative to the sum of the magnitudes of its terms: the bf16
+    # outputs and the bf16 probabilities each carry a relative error of at most 2^-9.
     dk64, dv64 = _f64(dk), _f64(dv)
     do_sum = _f64(do).reshape(w.B, w.Hkv, g, w.N, w.d).sum(axis=(2, 3))
-    scale_dk = np.abs(dk64).sum(axis=2).max()
-    assert np.abs(dk64.sum(axis=2)).max() <= 2e-2 * scale_dk
-    assert np.abs(dv64.sum(axis=2) - do_sum).max() <= 2e-2 * np.abs(do_sum).max() + 1.0
-    b, kh = sorted(groups)[-1]
-    hs = slice(kh * g, (kh + 1) * g)
-    check_bwd(dq[b:b + 1, hs], dk[b:b + 1, kh:kh + 1], dv[b:b + 1, kh:kh + 1],
-              _slice_group(q, b, hs.start, hs.stop), _slice_group(k, b, kh, kh + 1),
-              _slice_group(v, b, kh, kh + 1), _slice_group(do, b, hs.start, hs.stop),
-              w.causal, w.scale)
+    assert np.all(np.abs(dk64.sum(axis=2)) <= 1e-2 * np.abs(dk64).sum(axis=2))
+    assert np.all(np.abs(dv64.sum(axis=2) - do_sum) <= 1e-2 * np.abs(dv64).sum(axis=2))
+    for b, kh in groups[:2]:
+        hs = slice(kh * g, (kh + 1) * g)
+        check_bwd(dq[b:b + 1, hs], dk[b:b + 1, kh:kh + 1], dv[b:b + 1, kh:kh + 1],
+                  _slice_group(q, b, hs.start, hs.stop), _slice_group(k, b, kh, kh + 1),
+                  _slice_group(v, b, kh, kh + 1), _slice_group(do, b, hs.start, hs.stop),
+                  w.causal, w.scale)
