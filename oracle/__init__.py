@@ -10,8 +10,9 @@ Pins (checked by ``tests/test_oracle_pins.py`` against closed forms, the toy exa
 of the "Consideration"/FlashAttention article page, finite differences and invariants):
 ``oracle_fwd``, ``oracle_bwd``, their key-window, variable-length, block-sparse and dropout forms,
 ``oracle_decode``, ``oracle_merge`` and ``online_softmax_stats`` all have pins; none is
-"parity unpinned".  The dropout generator itself (Philox4x32-10) is pinned by statistics
-(keep rate, uniformity, independence), not by known-answer vectors.
+"parity unpinned".  The dropout generator itself (Philox4x32-10) is pinned word for word
+against an independent implementation (PyTorch's ATen Philox engine, compiled from its
+header by the test) and by statistics (keep rate, uniformity, independence).
 """
 from __future__ import annotations
 
@@ -23,12 +24,29 @@ import numpy as np
 from . import build as _build
 
 _LIB = None
+_VARIANT = "portable"
+
+
+def use_build(variant: str) -> None:
+    """Select the shared object the functions below call: "portable" (-O2, the one the
+    tests pin) or "native" (-O3 -march=native for this host, used to time the oracle as
+    a CPU baseline; it computes bit-identical results)."""
+    global _LIB, _VARIANT
+    if variant not in ("portable", "native"):
+        raise ValueError(variant)
+    if variant != _VARIANT:
+        _LIB, _VARIANT = None, variant
+
+
+def build_flags() -> str:
+    """Compiler flags of the build currently selected."""
+    return " ".join(_build.NATIVE_FLAGS if _VARIANT == "native" else ["-O2", "-ffp-contract=off", "-fopenmp"])
 
 
 def _lib():
     global _LIB
     if _LIB is None:
-        path = _build.build()
+        path = _build.build_native() if _VARIANT == "native" else _build.build()
         lib = ctypes.CDLL(path)
         dp = ctypes.POINTER(ctypes.c_double)
         ci = ctypes.c_int
@@ -71,6 +89,9 @@ def _lib():
         lib.oracle_bwd_blocksparse.argtypes = [dp, dp, dp, dp, u8p, dp, dp, dp, ci, ci, ci, ci,
                                                ci, ci, ctypes.c_double]
         lib.oracle_bwd_blocksparse.restype = ci
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        lib.oracle_philox4x32_10.argtypes = [u32p, u32p, u32p]
+        lib.oracle_philox4x32_10.restype = ci
         lib.oracle_online_softmax_stats.argtypes = [dp, ci, ci, dp, dp]
         lib.oracle_online_softmax_stats.restype = ci
         _LIB = lib
@@ -231,6 +252,20 @@ def attention_bwd_varlen(q, k, v, dout, cu_q, cu_k, left: int, right: int, scale
     if rc != 0:
         raise RuntimeError(f"oracle_bwd_varlen failed with {rc}")
     return dq, dk, dv
+
+
+def philox4x32_10(ctr, key):
+    """The oracle's Philox4x32-10: four uint32 output words for counter ``ctr`` (4 words)
+    and key ``key`` (2 words)."""
+    c = np.ascontiguousarray(np.asarray(ctr, dtype=np.uint32).reshape(4))
+    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint32).reshape(2))
+    out = np.empty(4, dtype=np.uint32)
+    u32p = ctypes.POINTER(ctypes.c_uint32)
+    rc = _lib().oracle_philox4x32_10(c.ctypes.data_as(u32p), k.ctypes.data_as(u32p),
+                                     out.ctypes.data_as(u32p))
+    if rc != 0:
+        raise RuntimeError(f"oracle_philox4x32_10 failed with {rc}")
+    return out
 
 
 def dropout_keep_mask(BH: int, N: int, p: float, seed: int):

@@ -590,6 +590,15 @@ static void philox4x32_10(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3, ui
     out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
+/* The generator itself, exported so that tests can compare it word for word with an
+ * independent implementation: out = Philox4x32-10(counter ctr[0..3], key key[0..1]). */
+int oracle_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    if (!ctr || !key || !out) return -1;
+    philox4x32_10(ctr[0], ctr[1], ctr[2], ctr[3], key[0], key[1], out);
+    return 0;
+}
+
 static uint32_t drop_threshold(double p)
 {
     const double t = floor(p * 65536.0);

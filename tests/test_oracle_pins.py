@@ -29,7 +29,11 @@ the causal mask on the wrong side, a missing scale) fails at least one test:
 * dropout: p = 0 is plain attention, the forward equals the reweighted masked softmax
   built from the keep mask, it is unbiased over seeds, its gradient matches central
   differences, and the keep mask has the right rate for six p and no visible correlation
-  between neighbouring keys, rows, heads or seeds.
+  between neighbouring keys, rows, heads or seeds;
+* the dropout generator: the oracle's Philox4x32-10 equals, word for word, PyTorch's
+  ATen Philox engine (an independent implementation of the same published generator,
+  compiled here from its C++ header), and the keep mask is exactly the stated selection
+  of 16-bit halves of that engine's output.
 """
 import math
 import os
@@ -715,6 +719,83 @@ def test_dropout_mask_has_no_visible_correlation():
     np.testing.assert_array_equal(keep, again)
 
 
+_ATEN_PHILOX_SRC = r"""
+#include <cstdint>
+#include <ATen/core/PhiloxRNGEngine.h>
+// n generator calls: counter ctr[4 i .. 4 i + 3], key key[2 i .. 2 i + 1] -> out[4 i ..].
+// The engine's state is (key = seed, counter = (offset lo, offset hi, subsequence lo,
+// subsequence hi)); its first four outputs are the four words of one block.
+extern "C" void aten_philox4x32_10(int n, const uint32_t *ctr, const uint32_t *key, uint32_t *out) {
+  for (int i = 0; i < n; ++i) {
+    const uint32_t *c = ctr + 4 * i, *k = key + 2 * i;
+    at::Philox4_32 eng(k[0] | (static_cast<uint64_t>(k[1]) << 32),
+                       c[2] | (static_cast<uint64_t>(c[3]) << 32),
+                       c[0] | (static_cast<uint64_t>(c[1]) << 32));
+    for (int w = 0; w < 4; ++w) out[4 * i + w] = eng();
+  }
+}
+"""
+
+
+@pytest.fixture(scope="module")
+def aten_philox(tmp_path_factory):
+    """PyTorch's header-only ATen Philox4x32-10 engine compiled into a tiny shared object:
+    an implementation of the generator that shares nothing with the oracle."""
+    import ctypes
+    import subprocess
+    import torch
+    inc = os.path.join(os.path.dirname(torch.__file__), "include")
+    d = tmp_path_factory.mktemp("aten_philox")
+    src, lib = d / "aten_philox.cpp", d / "libaten_philox.so"
+    src.write_text(_ATEN_PHILOX_SRC)
+    cuda_inc = os.environ.get("CUDA_HOME", "/usr/local/cuda") + "/include"
+    subprocess.run(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", f"-I{inc}", f"-I{cuda_inc}",
+                    str(src), "-o", str(lib)], check=True)
+    so = ctypes.CDLL(str(lib))
+    u32p = ctypes.POINTER(ctypes.c_uint32)
+
+    def run(ctr, key):
+        ctr = np.ascontiguousarray(ctr, dtype=np.uint32).reshape(-1, 4)
+        key = np.ascontiguousarray(key, dtype=np.uint32).reshape(-1, 2)
+        out = np.empty_like(ctr)
+        so.aten_philox4x32_10(ctypes.c_int(len(ctr)), ctr.ctypes.data_as(u32p),
+                              key.ctypes.data_as(u32p), out.ctypes.data_as(u32p))
+        return out
+
+    return run
+
+
+def test_philox_equals_the_aten_engine_word_for_word(aten_philox):
+    # Seeded random counters and keys over the whole 32-bit range, plus the extremes.
+    r = _rng(2011)
+    ctr = r.integers(0, 2 ** 32, size=(2000, 4), dtype=np.uint64).astype(np.uint32)
+    key = r.integers(0, 2 ** 32, size=(2000, 2), dtype=np.uint64).astype(np.uint32)
+    ctr[0], key[0] = 0, 0
+    ctr[1], key[1] = 0xFFFFFFFF, 0xFFFFFFFF
+    ctr[2] = [7, 0, 0, 0]          # small counters as the dropout mask uses them
+    ctr[3] = [0, 5, 3, 0]
+    want = aten_philox(ctr, key)
+    got = np.stack([oracle.philox4x32_10(c, k) for c, k in zip(ctr, key)])
+    np.testing.assert_array_equal(got, want)
+    # and the generator is not trivially the identity or constant
+    assert len({tuple(w) for w in got}) == len(got)
+
+
+def test_dropout_mask_is_the_stated_halves_of_the_generator(aten_philox):
+    # keep(bh, i, j) iff the 16-bit value j % 8 of Philox(counter (j / 8, i, bh, 0), key
+    # (seed low, seed high)) - the low half of word (j % 8) / 2 for even j, the high half
+    # for odd j - is >= floor(p 2^16); here the values come from the ATen engine.
+    BH, N, p, seed = 3, 41, 0.3, 0x1234ABCD9876F00D
+    thr = math.floor(p * 65536)
+    bh, i, j8 = np.meshgrid(np.arange(BH), np.arange(N), np.arange((N + 7) // 8), indexing="ij")
+    ctr = np.stack([j8.ravel(), i.ravel(), bh.ravel(), np.zeros(bh.size, dtype=np.int64)], axis=1)
+    key = np.tile([seed & 0xFFFFFFFF, seed >> 32], (len(ctr), 1))
+    words = aten_philox(ctr, key).reshape(BH, N, (N + 7) // 8, 4).astype(np.int64)
+    halves = np.stack([words & 0xFFFF, words >> 16], axis=-1).reshape(BH, N, -1)  # value m = 2w + half
+    want = (halves[:, :, :N] >= thr).astype(np.uint8)
+    np.testing.assert_array_equal(oracle.dropout_keep_mask(BH, N, p, seed), want)
+
+
 def test_dropout_forward_is_the_masked_reweighted_softmax():
     # Brute force from the keep mask: O = (softmax(S) * Z / (1 - p)) V, LSE unchanged.
     r = _rng(89)
@@ -841,3 +922,21 @@ def test_blocksparse_gradients_match_central_differences():
                 args_m[which][0, 0, n, c] -= eps
                 num = (loss(*args_p) - loss(*args_m)) / (2 * eps)
                 assert abs(g[0, 0, n, c] - num) <= 1e-6 * max(1.0, abs(num)), (which, n, c)
+
+
+# ---------------------------------------------------------------------------- timing build
+
+def test_native_timing_build_computes_the_same_bits():
+    # The -O3 -march=native build that times the oracle as a CPU baseline must be the
+    # same computation: no contraction into FMAs and no reassociation, so equal bits.
+    r = _rng(404)
+    q, k, v, do = (r.normal(size=(1, 4, 70, 16)) for _ in range(4))
+    k, v = k[:, :2], v[:, :2]
+    want = oracle.attention_fwd(q, k, v, True, 0.3) + oracle.attention_bwd(q, k, v, do, True, 0.3)
+    oracle.use_build("native")
+    try:
+        got = oracle.attention_fwd(q, k, v, True, 0.3) + oracle.attention_bwd(q, k, v, do, True, 0.3)
+    finally:
+        oracle.use_build("portable")
+    for a, b in zip(want, got):
+        np.testing.assert_array_equal(a, b)
