@@ -265,22 +265,28 @@ bool normalise_window(int w, int N, int *out) {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
 struct NoallocState {
-  std::once_flag once;
-  void *ptr = nullptr;
+  std::mutex mu;
+  void *ptr = nullptr;  // set only once a lookup has succeeded
 };
 NoallocState g_noalloc[kMaxDevices];
 
 // Device address of the static scratch on the current device (nullptr on failure).
-// Looked up once per device, on the first fa_bwd_noalloc call made with it current.
+// Looked up on the first fa_bwd_noalloc call made with the device current; a failed
+// lookup (for instance one attempted inside a stream capture) is not remembered, so a
+// later call retries it, and its error is cleared from the runtime so that it cannot
+// surface as the status of a later, unrelated launch.
 void *noalloc_scratch() {
   int dev = 0;
   if (!cuda_ok(cudaGetDevice(&dev), "cudaGetDevice") || dev < 0 || dev >= kMaxDevices) return nullptr;
   NoallocState &st = g_noalloc[dev];
-  std::call_once(st.once, [&] {
+  std::lock_guard<std::mutex> lock(st.mu);
+  if (!st.ptr) {
     void *p = nullptr;
     if (cuda_ok(cudaGetSymbolAddress(&p, g_noalloc_scratch), "cudaGetSymbolAddress(no-alloc scratch)"))
       st.ptr = p;
-  });
+    else
+      (void)cudaGetLastError();
+  }
   return st.ptr;
 }
 

@@ -253,7 +253,9 @@ int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *
  * return FA_ERR_SCRATCH_LIMIT before anything is launched.  No call allocates memory.
  *
  * The first call on a device (with that device current) looks up the buffer's device
- * address once; make that first call before any stream capture.  Every call on a device
+ * address; make that first call before any stream capture.  A lookup that fails returns
+ * FA_ERR_CUDA, leaves no error pending in the CUDA runtime and is retried by the next
+ * call; once it has succeeded it is not repeated.  Every call on a device
  * shares the same buffer, which keeps the previous call's contents (the kernels
  * re-initialise what they need), so calls whose kernels overlap on the GPU - on different
  * streams without ordering between them - race on it: order them on one stream or with
