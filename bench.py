@@ -2,12 +2,16 @@
 """Throughput of exact attention (forward + backward) on B200 through libfa_sm100.so.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--scaling weak|strong]
 
 A step is one forward (fa_fwd) and one backward (fa_bwd) pass over one batch of the
-workload (default: GPT-style 2K causal self-attention, B=8, H=16, N=2048, d=128, bf16,
-seeded i.i.d. N(0,1) inputs).  FLOPs follow the metric's convention: 4 B H N^2 d for the
-forward, halved when causal, and 2.5x that for the backward; a local-attention workload
-counts 4 d flop per visible (query, key) pair.
+workload (default: long-context causal self-attention, B=2, H=16, N=8192, d=128, bf16,
+seeded i.i.d. N(0,1) inputs - the largest single-GPU workload, the pages' 8K-context
+rows).  FLOPs follow the metric's convention: 4 B H N^2 d for the forward, halved when
+causal, and 2.5x that for the backward; a local-attention workload counts 4 d flop per
+visible (query, key) pair.  Each kernel is also reported against its two bounds: the
+tensor-core time of its FLOPs at the measured bf16 peak, and the MUFU time of its
+exponentials (one per visible score and pass) at 16 per clock per SM.
 
 --workload varlen_32k_ragged times fa_fwd_varlen + fa_bwd_varlen over a packed batch of
 ragged sequences (FLOPs of the visible pairs of each sequence); dropout_8k_causal times
@@ -22,13 +26,18 @@ The `e2e` leg runs the same steps through the public binding with each step's in
 from pinned host memory and its results copied back, overlapped across neighbouring steps
 on three streams (input copy, kernels, result copy) with two device buffer sets.
 
-Rank 0 prints one JSON line.  Under torchrun each rank (one GPU each) processes its own
-shard of a global batch of N x B sequences with the unchanged kernels (no collective on
-the data path); the timed region is bracketed by barriers and the slowest rank's time is
-used, so `value` is the whole job's TFLOP/s ("scaling": "weak").
+Rank 0 prints one JSON line.  Under torchrun each rank (one GPU each) runs the unchanged
+kernels on its own share with no collective on the data path; the timed region is
+bracketed by barriers and the slowest rank's time is used, so `value` is the whole job's
+TFLOP/s.  --scaling weak (default): each rank processes its own batch of the workload's
+shape, a global batch of N x B sequences.  --scaling strong: the workload itself is split
+by (batch row, K/V head) groups, so B = 2 at 8K context still spreads over 32 ranks.
 
-`--impl reference` times the fp64 CPU oracle (the parity reference) on a bounded sample of
-the same workload on this host's cores, on rank 0 only.
+The CPU baseline times the fp64 oracle (the parity reference, built -O3 -march=native for
+the host) on whole K/V-head groups of the workload, one oracle call per group, for about
+--cpu-budget seconds, and extrapolates the full workload's time from it.
+`--impl reference` times the same oracle on a per-step sample of the same workload, on
+rank 0 only.
 """
 from __future__ import annotations
 
@@ -88,6 +97,93 @@ def _profile_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
+    """SM clock, power and clock-event (throttle) reasons sampled DURING the timed region.
+
+    A thread polls NVML (read-only queries) every `period_s` between start() and stop(),
+    so even a timed region of a few tens of milliseconds gets samples; where NVML is
+    unavailable it falls back to `nvidia-smi -lms 20`, whose samples are kept only when
+    their timestamps fall inside the region."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, gpu_index: int, period_s: float = 0.002):
+        import threading
+        self.period = period_s
+        self.samples = []          # (sm_mhz, max_mhz, power_w, reason bits)
+        self.source = "nvml"
+        self.nvml = None
+        self.handle = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(gpu_index)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId_v2(bus.encode())
+            except Exception:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(gpu_index)
+            self.nvml = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+            self.source = "nvidia-smi"
+        self._smi = None if self.nvml is not None else _SmiSampler(gpu_index)
+
+    def _poll(self):
+        nv, h = self.nvml, self.handle
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                              getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+        while not self._stop.is_set():
+            try:
+                sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                bits = int(get_reasons(h)) if get_reasons else 0
+                self.samples.append((sm, self.max_mhz, pw, bits))
+            except Exception:
+                pass
+            self._stop.wait(self.period)
+
+    def start(self):
+        if self.nvml is None:
+            self._smi.start()
+            return
+        import threading
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+
+    def stop(self):
+        if self.nvml is None:
+            self._smi.stop()
+            return
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self):
+        if self.nvml is None:
+            return self._smi.summary()
+        sm = [x[0] for x in self.samples]
+        reasons = set()
+        for _, _, _, bits in self.samples:
+            for name, const in self.REASONS:
+                if bits & int(getattr(self.nvml, const, 0)):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(sm) if sm else None,
+                "power_w_max": max(x[2] for x in self.samples) if self.samples else None,
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "source": f"NVML every {self.period * 1e3:.0f} ms during the timed region"}
+
+
+class _SmiSampler:
     """nvidia-smi clock / throttle-reason samples, kept only inside [t0, t1]."""
 
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -99,10 +195,11 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.file, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        time.sleep(0.3)  # let nvidia-smi start sampling
         self.t0 = self.t1 = None
 
     def start(self):
@@ -110,7 +207,7 @@ class ClockSampler:
 
     def stop(self):
         self.t1 = _dt.datetime.now()
-        time.sleep(0.12)
+        time.sleep(0.05)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -145,47 +242,69 @@ class ClockSampler:
         os.unlink(self.file.name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": n}
+                "reasons": sorted(reasons), "samples": n,
+                "source": "nvidia-smi -lms 20 during the timed region"}
 
 
-def _oracle_sample(w, heads: int, seed: int):
-    """fp64 oracle fwd+bwd on the first `heads` query heads (whole K/V groups) of batch
-    row 0 of the workload's inputs; returns (seconds, metric FLOPs of the sample)."""
-    import numpy as np
-    import torch
+def _oracle_groups(w, n_groups: int, seed: int, budget_s: float | None = None):
+    """Time the fp64 oracle (fwd, plus bwd when the workload has one) on whole K/V-head
+    groups of batch row 0 of the workload's shapes, one oracle call per group, so the
+    working set and the per-flop rate do not depend on how many groups are sampled.
+    Stops after `n_groups` groups, or earlier once `budget_s` seconds of oracle time have
+    been spent (at least one group).  Returns (seconds, metric FLOPs, groups timed)."""
     import oracle
     from exact_io_aware_83_b200.inputs import draw
     g = w.Hq // w.Hkv
-    groups = max(1, heads // g)
-    q, k, v, do = draw(1, groups * g, groups, w.N, w.d, seed, w.q_std)
+    n_groups = max(1, min(n_groups, w.Hkv))
+    q, k, v, do = draw(1, n_groups * g, n_groups, w.N, w.d, seed, w.q_std)
     f64 = lambda t: t.float().double().numpy()
-    q, k, v, do = f64(q), f64(k), f64(v), f64(do)
     bm = w.block_mask()
-    if bm is not None:
-        bm = bm[:1, :groups * g].contiguous()
-    t0 = time.perf_counter()
-    if bm is not None:
-        oracle.attention_fwd_blocksparse(q, k, v, bm.numpy(), w.causal, w.scale)
-        if w.backward:
-            oracle.attention_bwd_blocksparse(q, k, v, do, bm.numpy(), w.causal, w.scale)
-    elif w.dropout_p:
-        oracle.attention_fwd_dropout(q, k, v, w.causal, w.scale, w.dropout_p, w.dropout_seed)
-        if w.backward:
-            oracle.attention_bwd_dropout(q, k, v, do, w.causal, w.scale, w.dropout_p, w.dropout_seed)
-    elif w.window is not None:
-        oracle.attention_fwd_window(q, k, v, w.window[0], w.window[1], w.scale)
-        if w.backward:
-            oracle.attention_bwd_window(q, k, v, do, w.window[0], w.window[1], w.scale)
-    else:
-        oracle.attention_fwd(q, k, v, w.causal, w.scale)
-        if w.backward:
-            oracle.attention_bwd(q, k, v, do, w.causal, w.scale)
-    dt = time.perf_counter() - t0
-    flops = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) * (groups * g) / (w.B * w.Hq)
+    total_t, groups = 0.0, 0
+    for kv in range(n_groups):
+        qs, ks, vs, ds = (f64(t[:, kv * g:(kv + 1) * g] if t.shape[1] == n_groups * g else t[:, kv:kv + 1])
+                          for t in (q, k, v, do))
+        t0 = time.perf_counter()
+        if bm is not None:
+            m = bm[:1, kv * g:(kv + 1) * g].contiguous().numpy()
+            oracle.attention_fwd_blocksparse(qs, ks, vs, m, w.causal, w.scale)
+            if w.backward:
+                oracle.attention_bwd_blocksparse(qs, ks, vs, ds, m, w.causal, w.scale)
+        elif w.dropout_p:
+            oracle.attention_fwd_dropout(qs, ks, vs, w.causal, w.scale, w.dropout_p, w.dropout_seed)
+            if w.backward:
+                oracle.attention_bwd_dropout(qs, ks, vs, ds, w.causal, w.scale, w.dropout_p, w.dropout_seed)
+        elif w.window is not None:
+            oracle.attention_fwd_window(qs, ks, vs, w.window[0], w.window[1], w.scale)
+            if w.backward:
+                oracle.attention_bwd_window(qs, ks, vs, ds, w.window[0], w.window[1], w.scale)
+        else:
+            oracle.attention_fwd(qs, ks, vs, w.causal, w.scale)
+            if w.backward:
+                oracle.attention_bwd(qs, ks, vs, ds, w.causal, w.scale)
+        total_t += time.perf_counter() - t0
+        groups += 1
+        if budget_s is not None and total_t >= budget_s:
+            break
+    per_group = (w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)) / (w.B * w.Hkv)
+    flops = per_group * groups
     if bm is not None:  # the sampled heads' own mask
         from exact_io_aware_83_b200.inputs import blocksparse_pairs
-        flops = 4.0 * blocksparse_pairs(bm, w.N, w.causal) * w.d * (3.5 if w.backward else 1.0)
-    return dt, flops
+        flops = 4.0 * blocksparse_pairs(bm[:1, :groups * g].contiguous(), w.N, w.causal) * w.d * (
+            3.5 if w.backward else 1.0)
+    return total_t, flops, groups
+
+
+def _cpu_baseline_line(w, seconds, flops, groups, cores, note):
+    """The cpu_baseline object: the oracle's rate on the sample, what the sample was, and
+    the full workload's time extrapolated from it (per group; groups are independent)."""
+    import oracle
+    from oracle import build as oracle_build
+    return {"value": flops / seconds / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "cpu_model": oracle_build.cpu_model(), "build": oracle.build_flags(),
+            "sample": (f"K/V-head groups 0..{groups - 1} of batch row 0 of {w.name} ({groups * (w.Hq // w.Hkv)} "
+                       f"query heads), fp64 oracle fwd{'+bwd' if w.backward else ''}, one oracle call per "
+                       f"group, {seconds:.1f} s {note}"),
+            "full_size_s_extrapolated": seconds / groups * w.B * w.Hkv}
 
 
 def _e2e_pipelined(host_in, dev_in, dev_out, host_out, compute, n_steps, n_warm, barrier):
@@ -253,32 +372,31 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     import oracle
+    oracle.use_build("native")
     cores = _cores()
     oracle.set_threads(cores)
-    # Size the per-step sample so the whole run stays near a two-minute budget: whole
-    # K/V-head groups of batch row 0, at least one.
-    g = w.Hq // w.Hkv
-    t_group, _ = _oracle_sample(w, g, w.seed)
-    budget = 120.0 / (args.steps + args.warmup)
-    heads = g * max(1, min(w.Hkv, int(budget // max(t_group, 1e-6))))
+    # Size the per-step sample so the whole run stays near a two-and-a-half-minute budget:
+    # whole K/V-head groups of batch row 0, at least one.
+    t_group, _, _ = _oracle_groups(w, 1, w.seed)
+    budget = 150.0 / (args.steps + args.warmup)
+    groups = max(1, min(w.Hkv, int(budget // max(t_group, 1e-6))))
     for _ in range(args.warmup):
-        _oracle_sample(w, heads, w.seed)
+        _oracle_groups(w, groups, w.seed)
     total_t, total_f = 0.0, 0.0
     for _ in range(args.steps):
-        dt, fl = _oracle_sample(w, heads, w.seed)
+        dt, fl, _ = _oracle_groups(w, groups, w.seed)
         total_t += dt
         total_f += fl
     value = total_f / total_t / 1e12
-    sample = (f"batch row 0, query heads 0..{heads - 1} of {w.name} (fwd"
-              f"{'+bwd' if w.backward else ''}), fp64 oracle, per step")
+    cpu = _cpu_baseline_line(w, total_t / args.steps, total_f / args.steps, groups, cores, "per step")
+    cpu["value"] = value
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total_t / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(w, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                         "sample": sample},
+        "cpu_baseline": cpu,
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -339,6 +457,7 @@ def run_reference_varlen(args, w):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     import oracle
+    oracle.use_build("native")
     cores = _cores()
     oracle.set_threads(cores)
     t1, f1 = _oracle_varlen_sample(w, 1)
@@ -417,7 +536,6 @@ def run_ours_varlen(args, w):
     if fa.fa_device_status(None) != fa.FA_OK:
         raise SystemExit("device status not clean after warm-up")
     sampler = ClockSampler(local)
-    time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -486,6 +604,7 @@ def run_ours_varlen(args, w):
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         import oracle
+        oracle.use_build("native")
         cores = _cores()
         oracle.set_threads(cores)
         dt, fl = _oracle_varlen_sample(w, 2)
@@ -498,18 +617,42 @@ def run_ours_varlen(args, w):
     return 0
 
 
+def _parts(w, world: int, rank: int, scaling: str):
+    """This rank's share of the work as (host tensors, block mask, batch rows, query heads,
+    K/V heads) parts.  Weak scaling: one part, the whole workload drawn with the rank's own
+    seed.  Strong scaling: the workload itself (one seed on every rank) split by
+    (batch row, K/V head) groups, one part per contiguous segment of this rank's groups."""
+    from exact_io_aware_83_b200.inputs import draw
+    from exact_io_aware_83_b200.shard import rank_seed, segment_slices, shard_groups
+    bmh = w.block_mask()
+    if scaling == "weak":
+        host = draw(w.B, w.Hq, w.Hkv, w.N, w.d, rank_seed(w.seed, rank), w.q_std)
+        return [(host, bmh, w.B, w.Hq, w.Hkv)]
+    full = draw(w.B, w.Hq, w.Hkv, w.N, w.d, w.seed, w.q_std)
+    g = w.Hq // w.Hkv
+    parts = []
+    for seg in shard_groups(w.B, w.Hkv, world, rank):
+        qh_, kvh_, bs = segment_slices(seg, g)
+        host = tuple(t[bs, qh_ if t.shape[1] == w.Hq else kvh_].contiguous() for t in full)
+        bm = None if bmh is None else bmh[bs, qh_].contiguous()
+        parts.append((host, bm, seg.b_hi - seg.b_lo, (seg.kv_hi - seg.kv_lo) * g, seg.kv_hi - seg.kv_lo))
+    return parts
+
+
 def run_ours(args, w):
     import torch
     import torch.distributed as dist
     from exact_io_aware_83_b200 import fa
-    from exact_io_aware_83_b200.inputs import draw
-    from exact_io_aware_83_b200.shard import max_over_ranks, rank_seed
+    from exact_io_aware_83_b200.shard import max_over_ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if args.scaling == "strong" and w.dropout_p:
+        raise SystemExit("--scaling strong: the dropout mask is a function of the global head "
+                         "index, so a split problem would draw a different mask")
     torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", timeout=_dt.timedelta(seconds=120),
@@ -520,26 +663,32 @@ def run_ours(args, w):
             dist.barrier()
 
     fa.load()
-    qh, kh, vh, doh = draw(w.B, w.Hq, w.Hkv, w.N, w.d, rank_seed(w.seed, rank), w.q_std)
-    q, k, v, do = (t.cuda() for t in (qh, kh, vh, doh))
-    o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.Hq, w.N), dtype=torch.float32, device="cuda")
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d), dtype=torch.uint8,
-                     device="cuda")
-    bmh = w.block_mask()
-    bmd = None if bmh is None else bmh.cuda()
+    # Per part: device inputs [q, k, v, (dO), (mask)] and outputs [o, lse, (dq, dk, dv)],
+    # one backward workspace per part.
+    parts = []
+    for host, bmh, B, Hq, Hkv in _parts(w, world, rank, args.scaling):
+        ins = list(host[:3]) + ([host[3]] if w.backward else []) + ([] if bmh is None else [bmh])
+        dev = [t.cuda() for t in ins]
+        q = dev[0]
+        outs = [torch.empty_like(q), torch.empty((B, Hq, w.N), dtype=torch.float32, device="cuda")]
+        if w.backward:
+            outs += [torch.empty_like(q), torch.empty_like(dev[1]), torch.empty_like(dev[2])]
+        ws = torch.empty(fa.fa_bwd_workspace_bytes(B, Hq, Hkv, w.N, w.d), dtype=torch.uint8, device="cuda")
+        parts.append({"host": ins, "dev": dev, "outs": outs, "ws": ws, "mask": bmh is not None})
 
-    def run(q, k, v, do, o, lse, dq, dk, dv, bm):
-        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=o, lse=lse, window=w.window,
+    def run(part, dev, outs):
+        q, k, v = dev[0], dev[1], dev[2]
+        bm = dev[-1] if part["mask"] else None
+        fa.fwd(q, k, v, causal=w.causal, scale=w.scale, out=outs[0], lse=outs[1], window=w.window,
                dropout_p=w.dropout_p, seed=w.dropout_seed, block_mask=bm)
         if w.backward:
-            fa.bwd(q, k, v, o, lse, do, causal=w.causal, scale=w.scale, workspace=ws, dq=dq,
-                   dk=dk, dv=dv, window=w.window, dropout_p=w.dropout_p, seed=w.dropout_seed,
-                   block_mask=bm)
+            fa.bwd(q, k, v, outs[0], outs[1], dev[3], causal=w.causal, scale=w.scale, workspace=part["ws"],
+                   dq=outs[2], dk=outs[3], dv=outs[4], window=w.window, dropout_p=w.dropout_p,
+                   seed=w.dropout_seed, block_mask=bm)
 
     def step():
-        run(q, k, v, do, o, lse, dq, dk, dv, bmd)
+        for part in parts:
+            run(part, part["dev"], part["outs"])
 
     for _ in range(args.warmup):
         step()
@@ -548,7 +697,6 @@ def run_ours(args, w):
         raise SystemExit("device status not clean after warm-up")
 
     sampler = ClockSampler(local)
-    time.sleep(0.3)  # let nvidia-smi start sampling
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -560,8 +708,8 @@ def run_ours(args, w):
         step()
     e1.record()
     torch.cuda.synchronize()
-    barrier()
     sampler.stop()
+    barrier()
     fa.fa_kernel_timing(False)
     ms_local = e0.elapsed_time(e1)
     ms = max_over_ranks(ms_local)
@@ -572,63 +720,75 @@ def run_ours(args, w):
         raise SystemExit(f"device status {status} after the timed region")
     clocks = sampler.summary()
 
-    step_flops = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
-    value = step_flops * args.steps * world / (ms / 1e3) / 1e12
+    # FLOPs of one step on this rank (weak: the whole workload; strong: its share), and of
+    # the whole job per step.
+    share = sum(p["dev"][0].shape[0] * p["dev"][0].shape[1] for p in parts) / (w.B * w.Hq)
+    step_flops_full = w.fwd_flops() + (w.bwd_flops() if w.backward else 0.0)
+    job_flops = step_flops_full * (world if args.scaling == "weak" else 1)
+    value = job_flops * args.steps / (ms / 1e3) / 1e12
 
     # ---- end to end through the public API: pinned host inputs in, results back to host
-    pin = lambda t: t.pin_memory()
-    ins = [qh, kh, vh] + ([doh] if w.backward else []) + ([] if bmh is None else [bmh])
-    host_in = [pin(t) for t in ins]
-    outs = [o, lse] + ([dq, dk, dv] if w.backward else [])
-    dev_in = [[q, k, v] + ([do] if w.backward else []) + ([] if bmd is None else [bmd]),
-              [torch.empty_like(t, device="cuda") for t in ins]]
-    dev_out = [outs, [torch.empty_like(t) for t in outs]]
-    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs] for _ in range(2)]
+    host_in = [t.pin_memory() for p in parts for t in p["host"]]
+    dev_in = [[t for p in parts for t in p["dev"]],
+              [torch.empty_like(t) for p in parts for t in p["dev"]]]
+    dev_out = [[t for p in parts for t in p["outs"]],
+               [torch.empty_like(t) for p in parts for t in p["outs"]]]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out[0]] for _ in range(2)]
 
     def compute(sl):
-        di, do_ = dev_in[sl], dev_out[sl]
-        qq, kk, vv = di[0], di[1], di[2]
-        dd = di[3] if w.backward else None
-        bm = di[-1] if bmd is not None else None
-        if w.backward:
-            run(qq, kk, vv, dd, do_[0], do_[1], do_[2], do_[3], do_[4], bm)
-        else:
-            run(qq, kk, vv, None, do_[0], do_[1], None, None, None, bm)
+        i_in = i_out = 0
+        for p in parts:
+            n_in, n_out = len(p["dev"]), len(p["outs"])
+            run(p, dev_in[sl][i_in:i_in + n_in], dev_out[sl][i_out:i_out + n_out])
+            i_in += n_in
+            i_out += n_out
 
     e2e_steps = max(8, args.steps // 10)
     e2e_ms = max_over_ranks(_e2e_pipelined(host_in, dev_in, dev_out, host_out, compute, e2e_steps, 2,
                                            barrier))
     nbytes = lambda *ts: sum(t.numel() * t.element_size() for t in ts)
     h2d = nbytes(*dev_in[0])
-    d2h = nbytes(*outs)
-    e2e_value = step_flops * e2e_steps * world / (e2e_ms / 1e3) / 1e12
+    d2h = nbytes(*dev_out[0])
+    e2e_value = job_flops * e2e_steps / (e2e_ms / 1e3) / 1e12
 
     peaks, peak_src = _peaks()
-    # Dominant kernel: the backward main kernel (or the forward when there is no backward).
-    if w.backward and nbwd:
-        dom_name, dom_ms, dom_n, dom_flops = "fa_bwd_main_kernel", bwd_ms, nbwd, w.bwd_flops()
-    else:
-        dom_name, dom_ms, dom_n, dom_flops = "fa_fwd_kernel", fwd_ms, nfwd, w.fwd_flops()
-    achieved = dom_flops / (dom_ms / dom_n / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
-    traffic = _profile_traffic(dom_name, w.name)
+    # Secondary bound: one exponential per visible score in each pass (the backward
+    # recomputes them), at 16 per clock per SM on the MUFU unit.
+    sms = torch.cuda.get_device_properties(local).multi_processor_count
+    mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
+    exp_rate = 16.0 * sms * mhz * 1e6
     kernels = {}
-    if nfwd:
-        kernels["fa_fwd_kernel"] = {"ms_per_launch": fwd_ms / nfwd,
-                                    "tflops": w.fwd_flops() / (fwd_ms / nfwd / 1e3) / 1e12}
-    if nbwd:
-        kernels["fa_bwd_main_kernel"] = {"ms_per_launch": bwd_ms / nbwd,
-                                         "tflops": w.bwd_flops() / (bwd_ms / nbwd / 1e3) / 1e12}
+    for kname, kms, kn, kflops in (("fa_fwd_kernel", fwd_ms, nfwd, w.fwd_flops() * share / max(len(parts), 1)),
+                                   ("fa_bwd_main_kernel", bwd_ms, nbwd, w.bwd_flops() * share / max(len(parts), 1))):
+        if not kn:
+            continue
+        per = kms / kn
+        exps = w.score_pairs() * share / len(parts)
+        kernels[kname] = {"ms_per_launch": per, "tflops": kflops / (per / 1e3) / 1e12,
+                          "tensor_bound_ms": kflops / (peak * 1e12) * 1e3,
+                          "exp2_per_launch": exps,
+                          "mufu_bound_ms": exps / exp_rate * 1e3,
+                          "mufu_bound_note": (f"all exponentials on MUFU ex2 at 16/clk/SM x {sms} SMs x "
+                                              f"{mhz:.0f} MHz (the forward runs 1/16 of them on the FMA pipe)")}
     for kname, kd in kernels.items():
         kd["frac_of_burst_peak"] = kd["tflops"] / peak
         kd["frac_of_sustained_peak"] = kd["tflops"] / float(peaks["bf16_tflops_sustained"])
         kd["frac_of_nominal_peak"] = kd["tflops"] / NOMINAL_BF16_TFLOPS
+    # Dominant kernel: the backward main kernel (or the forward when there is no backward).
+    dom_name = "fa_bwd_main_kernel" if "fa_bwd_main_kernel" in kernels else "fa_fwd_kernel"
+    achieved = kernels[dom_name]["tflops"]
+    traffic = _profile_traffic(dom_name, w.name) if args.scaling == "weak" else None
 
+    cfg = _config(w, world)
+    if args.scaling == "strong":
+        cfg.update(B_per_gpu=None, global_batch=w.B, parallelism=f"groups{world}",
+                   groups_per_gpu=sum(p["dev"][1].shape[0] * p["dev"][1].shape[1] for p in parts))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": _config(w, world),
+        "scaling": args.scaling, "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": cfg,
         "frac_of_peak": value / world / peak,
         "roofline": {"bound": "tensor", "kernel": dom_name, "achieved": achieved, "peak": peak,
                      "unit": "TFLOP/s", "frac": achieved / peak, "traffic": traffic,
@@ -636,19 +796,16 @@ def run_ours(args, w):
         "kernels": kernels,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps, "overlap": E2E_OVERLAP},
-        "gpu_launches": args.steps * (1 + (3 if w.backward else 0)),
+        "gpu_launches": args.steps * len(parts) * (1 + (3 if w.backward else 0)),
         "clocks": clocks,
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         import oracle
+        oracle.use_build("native")
         cores = _cores()
         oracle.set_threads(cores)
-        heads = max(1, min(w.Hq, args.sample_heads))
-        dt, fl = _oracle_sample(w, heads, w.seed)
-        line["cpu_baseline"] = {
-            "value": fl / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"batch row 0, query heads 0..{heads - 1} of {w.name}, fp64 oracle "
-                      f"fwd{'+bwd' if w.backward else ''}, one pass, {dt:.1f} s wall"}
+        dt, fl, groups = _oracle_groups(w, w.Hkv, w.seed, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = _cpu_baseline_line(w, dt, fl, groups, cores, "wall, one pass")
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -678,6 +835,7 @@ def run_reference_decode(args, w):
     if int(os.environ.get("RANK", "0")) != 0:
         return 0
     import oracle
+    oracle.use_build("native")
     cores = _cores()
     oracle.set_threads(cores)
     t1, _ = _oracle_decode_sample(w, 1)
@@ -745,7 +903,6 @@ def run_ours_decode(args, w):
     if fa.fa_device_status(None) != fa.FA_OK:
         raise SystemExit("device status not clean after warm-up")
     sampler = ClockSampler(local)
-    time.sleep(0.3)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -804,6 +961,7 @@ def run_ours_decode(args, w):
     }
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         import oracle
+        oracle.use_build("native")
         cores = _cores()
         oracle.set_threads(cores)
         dt, nbytes = _oracle_decode_sample(w, 1)
@@ -820,12 +978,15 @@ def run_ours_decode(args, w):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="gpt_2k_causal")
+    ap.add_argument("--workload", default="long_8k_causal")
+    ap.add_argument("--scaling", choices=("weak", "strong"), default="weak",
+                    help="weak: each rank runs the whole workload on its own batch; strong: the "
+                         "workload's (batch row, K/V head) groups are split across the ranks")
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--sample-heads", type=int, default=4,
-                    help="query heads in the oracle's bounded CPU sample")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle time in the CPU-baseline sample (whole K/V-head groups)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -99,6 +99,14 @@ class Workload:
         """2.5 x the forward count."""
         return 2.5 * self.fwd_flops()
 
+    def score_pairs(self) -> float:
+        """(query, key) pairs whose score is visible, i.e. exponentials per pass (the
+        forward evaluates one per pair, the backward recomputes each once)."""
+        if self.block_density or self.window is not None:
+            return self.fwd_flops() / (4.0 * self.d)
+        per_head = self.N * (self.N + 1) / 2 if self.causal else float(self.N) * self.N
+        return self.B * self.Hq * per_head
+
 
 WORKLOADS = {
     w.name: w

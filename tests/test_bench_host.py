@@ -47,8 +47,8 @@ def test_committed_traffic_entries_name_existing_sources():
             assert os.path.exists(os.path.join(bench.ROOT, src)), src
 
 
-def test_clock_summary_keeps_the_timed_region_only(tmp_path):
-    s = bench.ClockSampler.__new__(bench.ClockSampler)
+def test_smi_clock_summary_keeps_the_timed_region_only(tmp_path):
+    s = bench._SmiSampler.__new__(bench._SmiSampler)
     s.file = open(tmp_path / "c.csv", "w+")
     s.proc = object()  # stands for the nvidia-smi process
     t0 = dt.datetime(2026, 1, 1, 12, 0, 0)
@@ -68,6 +68,77 @@ def test_clock_summary_keeps_the_timed_region_only(tmp_path):
     assert out["sm_mhz"] == 1930
     assert out["sm_max_mhz"] == 1965
     assert out["reasons"] == ["sw_power_cap"]
+
+
+class _FakeNvml:
+    """Read-only NVML queries with scripted answers (no GPU involved)."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwPowerBrakeSlowdown = 0x80
+
+    def __init__(self, clocks, reasons):
+        self.clocks, self.reasons, self.i = clocks, reasons, 0
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        return self.clocks[min(self.i, len(self.clocks) - 1)]
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 950000
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        r = self.reasons[min(self.i, len(self.reasons) - 1)]
+        self.i += 1
+        return r
+
+
+def test_nvml_clock_sampler_polls_during_the_region():
+    import threading
+    import time
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.period = 0.001
+    s.samples = []
+    s.source = "nvml"
+    s.nvml = _FakeNvml([1965, 1950, 1940], [0x0, 0x4, 0x0])
+    s.handle = None
+    s.max_mhz = 1965.0
+    s._stop = threading.Event()
+    s._thread = None
+    s.start()
+    time.sleep(0.05)
+    s.stop()
+    out = s.summary()
+    assert out["samples"] >= 3
+    assert out["sm_max_mhz"] == 1965.0 and out["sm_mhz"] == 1940
+    assert out["reasons"] == ["sw_power_cap"]
+    assert out["power_w_max"] == 950.0
+
+
+def test_default_workload_is_the_long_context_target():
+    # the parser's default, read from the source of main() without running it
+    import inspect
+    assert WORKLOADS["long_8k_causal"].N == 8192
+    assert 'default="long_8k_causal"' in inspect.getsource(bench.main)
+
+
+def test_exponential_counts_of_the_workloads():
+    w = WORKLOADS["long_8k_causal"]
+    assert w.score_pairs() == 2 * 16 * 8192 * 8193 / 2
+    assert WORKLOADS["d256_4k_stress"].score_pairs() == 2 * 8 * 4096 * 4096
+    win = WORKLOADS["window_8k_1k"]
+    assert win.score_pairs() == win.fwd_flops() / (4 * win.d)
+
+
+def test_strong_scaling_parts_cover_the_workload():
+    w = WORKLOADS["long_8k_causal"]
+    seen = []
+    for rank in range(8):
+        for host, bm, B, Hq, Hkv in bench._parts(w, 8, rank, "strong"):
+            assert host[0].shape == (B, Hq, w.N, w.d) and host[1].shape == (B, Hkv, w.N, w.d)
+            seen.append(B * Hkv)
+    assert sum(seen) == w.B * w.Hkv
 
 
 def test_config_names_the_workload():
