@@ -11,12 +11,14 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "fa.h"
 #include "fa_common.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd_d256.cuh"
+#include "fa_fwd_persist.cuh"
 #include "fa_bwd.cuh"
 #include "fa_decode.cuh"
 
@@ -67,6 +69,7 @@ EncodeTiledFn encode_fn() {
 struct DeviceState {
   std::once_flag once;
   bool ok = false;
+  int sms = 148;  // multiprocessors: the persistent kernels launch one CTA per SM
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -89,6 +92,11 @@ bool set_smem(K kernel, int bytes) {
                           "cudaFuncSetAttribute(max dynamic shared memory)");
   if (!ok && debug_enabled()) std::fprintf(stderr, "[fa]   requested %d bytes\n", bytes);
   return ok;
+}
+
+int current_sms() {
+  int dev = 0;
+  return (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices) ? g_dev[dev].sms : 148;
 }
 
 bool device_ready() {
@@ -167,6 +175,25 @@ bool device_ready() {
     ok = ok && set_smem(fa::fa_decode_kernel<256, 16>, fa::DecodeLayout<256, 16>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<256, 32>, fa::DecodeLayout<256, 32>::kSmemBytes);
     ok = ok && set_smem(fa::fa_decode_kernel<256, 64>, fa::DecodeLayout<256, 64>::kSmemBytes);
+    using fa::FwdPLayout;
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<64, fa::kAttnFull>, FwdPLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<64, fa::kAttnCausal>, FwdPLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<128, fa::kAttnFull>, FwdPLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<128, fa::kAttnCausal>, FwdPLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<64, fa::kAttnFull, true>, FwdPLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<64, fa::kAttnCausal, true>, FwdPLayout<64>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<128, fa::kAttnFull, true>, FwdPLayout<128>::kSmemBytes);
+    ok = ok && set_smem(fa::fa_fwd_persist_kernel<128, fa::kAttnCausal, true>, FwdPLayout<128>::kSmemBytes);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<64, fa::kAttnFull>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<64, fa::kAttnCausal>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<128, fa::kAttnFull>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<128, fa::kAttnCausal>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<64, fa::kAttnFull, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<64, fa::kAttnCausal, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<128, fa::kAttnFull, true>, fa::kFwdRegsLaunch);
+    ok = ok && regs_at_least(fa::fa_fwd_persist_kernel<128, fa::kAttnCausal, true>, fa::kFwdRegsLaunch);
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0) st.sms = sms;
     if (!ok && debug_enabled()) std::fprintf(stderr, "[fa] device setup failed\n");
     st.ok = ok;
   });
@@ -355,9 +382,36 @@ void launch_fwd_d(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMa
                                        s>>>(tq, tk, tv, to, p);
 }
 
+// Forward scheduler for dense full and causal attention (d = 64, 128): the persistent
+// kernel (one CTA per SM walking the units) or one CTA per unit.  fa_set_fwd_scheduler.
+std::atomic<int> g_fwd_persistent{[] {
+  const char *e = std::getenv("FA_FWD_PERSISTENT");  // "0": start with one CTA per unit
+  return (e && e[0] == '0') ? 0 : 1;
+}()};
+std::atomic<unsigned> g_unit_slot{0};
+
+template <int D, int MODE, bool DROP>
+void launch_fwd_persist(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
+                        const FwdParams &p, unsigned units, cudaStream_t s) {
+  const unsigned sms = static_cast<unsigned>(current_sms());
+  const unsigned grid = units < sms ? units : sms;
+  const int slot = static_cast<int>(g_unit_slot.fetch_add(1u) % fa::kUnitSlots);
+  fa::fa_fwd_persist_kernel<D, MODE, DROP><<<grid, fa::kFwdThreads, fa::FwdPLayout<D>::kSmemBytes, s>>>(
+      tq, tk, tv, to, p, static_cast<int>(units), slot);
+}
+
 template <int D>
 void launch_fwd_mode(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv, const CUtensorMap &to,
                      const FwdParams &p, unsigned units, int mode, bool drop, cudaStream_t s) {
+  if constexpr (D != 256) {
+    if (g_fwd_persistent.load() && (mode == fa::kAttnFull || mode == fa::kAttnCausal)) {
+      if (drop && mode == fa::kAttnCausal) launch_fwd_persist<D, fa::kAttnCausal, true>(tq, tk, tv, to, p, units, s);
+      else if (drop) launch_fwd_persist<D, fa::kAttnFull, true>(tq, tk, tv, to, p, units, s);
+      else if (mode == fa::kAttnCausal) launch_fwd_persist<D, fa::kAttnCausal, false>(tq, tk, tv, to, p, units, s);
+      else launch_fwd_persist<D, fa::kAttnFull, false>(tq, tk, tv, to, p, units, s);
+      return;
+    }
+  }
   if (drop && mode == fa::kAttnCausal) launch_fwd_d<D, fa::kAttnCausal, true>(tq, tk, tv, to, p, units, s);
   else if (drop) launch_fwd_d<D, fa::kAttnFull, true>(tq, tk, tv, to, p, units, s);
   else if (mode == fa::kAttnGeneral) launch_fwd_d<D, fa::kAttnGeneral, false>(tq, tk, tv, to, p, units, s);
@@ -767,6 +821,11 @@ int fa_bwd_blocksparse(const void *q, const void *k, const void *v, const void *
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
                         static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop, nullptr, nullptr,
                         block_mask);
+}
+
+int fa_set_fwd_scheduler(int persistent) {
+  if (persistent != 0 && persistent != 1) return FA_ERR_INVALID_ARG;
+  return g_fwd_persistent.exchange(persistent);
 }
 
 int fa_kernel_timing(int enable) {

@@ -126,6 +126,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_kernel_time_ms.argtypes = [ci, ctypes.POINTER(ctypes.c_float),
                                           ctypes.POINTER(ctypes.c_int)]
         lib.fa_kernel_time_ms.restype = ci
+        lib.fa_set_fwd_scheduler.argtypes = [ci]
+        lib.fa_set_fwd_scheduler.restype = ci
         _lib = lib
         return lib
 
@@ -258,6 +260,15 @@ def fa_watchdog_selftest(limit_us: int, stream=None) -> None:
 
 def fa_kernel_timing(enable: bool) -> None:
     _check(load().fa_kernel_timing(1 if enable else 0), "fa_kernel_timing")
+
+
+def fa_set_fwd_scheduler(persistent: bool) -> bool:
+    """Choose the dense forward's tile scheduler (True: persistent CTAs with dynamic unit
+    assignment, False: one CTA per unit); returns the previous choice."""
+    prev = load().fa_set_fwd_scheduler(1 if persistent else 0)
+    if prev < 0:
+        _check(prev, "fa_set_fwd_scheduler")
+    return bool(prev)
 
 
 def fa_kernel_time_ms(which: int):

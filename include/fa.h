@@ -343,6 +343,24 @@ int fa_kernel_timing(int enable);
 int fa_kernel_time_ms(int which, float *ms, int *launches);
 
 /*
+ * Forward tile scheduler for dense full and causal attention with d = 64 or 128 (fa_fwd,
+ * fa_fwd_window with bands (-1, -1) / (-1, 0), fa_fwd_dropout).  The FlashAttention-2
+ * page ("Better Parallelism") parallelises over batch x heads x query blocks; here a work
+ * unit is two 128-row query tiles, numbered heaviest first under a causal mask.
+ *   persistent = 1 (default): one CTA per SM walks the units, taking each next unit from a
+ *       device counter (dynamic assignment), so one unit's epilogue overlaps the next
+ *       unit's loads and first products.
+ *   persistent = 0: one CTA per unit, started by the hardware in unit order.
+ * The environment variable FA_FWD_PERSISTENT=0, read when the library loads, makes
+ * one CTA per unit the starting choice.
+ * Both compute bit-identical O and LSE.  Other variants (d = 256, other bands, packed
+ * sequences, block masks) always use one CTA per unit.  Affects later calls of this
+ * process; returns the previous setting, or FA_ERR_INVALID_ARG.  Not synchronised with
+ * calls running on other host threads.
+ */
+int fa_set_fwd_scheduler(int persistent);
+
+/*
  * Watchdog self-test: launches one thread that waits, with a limit of `limit_us`
  * microseconds (1 .. 10^7), on a pipeline barrier that nothing ever signals - the same
  * bounded-wait code every attention kernel uses.  The wait expires, the kernel records
