@@ -14,7 +14,8 @@ import torch
 import oracle
 from exact_io_aware_83_b200 import fa
 from exact_io_aware_83_b200.inputs import draw
-from test_gpu_parity import GRAD_TOL, LSE_TOL, _f64, _rel_fro, o_tolerance
+from test_gpu_parity import (GRAD_TOL, LSE_TOL, _f64, _rel_fro, causal_visible, o_tolerance,
+                             p_allowance)
 
 pytestmark = pytest.mark.gpu
 
@@ -31,9 +32,16 @@ def run(q, k, v, do, causal, scale, p, seed):
 
 def check(res, q, k, v, do, causal, scale, p, seed):
     o, lse, dq, dk, dv = res
-    o_r, lse_r = oracle.attention_fwd_dropout(_f64(q), _f64(k), _f64(v), causal, scale, p, seed)
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    o_r, lse_r = oracle.attention_fwd_dropout(q64, k64, v64, causal, scale, p, seed)
     assert np.isfinite(_f64(o)).all()
-    assert float(np.max(np.abs(_f64(o) - o_r) - o_tolerance(o_r))) <= 0.0
+    # the allowance's weights: the keep mask times the inverse keep probability
+    B, Hq, N, _ = q.shape
+    keep = oracle.dropout_keep_mask(B * Hq, N, p, seed).astype(np.float64)
+    inv_keep = 65536.0 / (65536.0 - math.floor(p * 65536.0))
+    allow = p_allowance(q64, k64, v64, o_r, lse_r, scale, causal_visible(N, causal),
+                        weight=lambda b, h, i: keep[b * Hq + h, i] * inv_keep)
+    assert float(np.max(np.abs(_f64(o) - o_r) - o_tolerance(o_r, allow))) <= 0.0
     assert float(np.abs(lse.double().numpy() - lse_r).max()) <= LSE_TOL
     refs = oracle.attention_bwd_dropout(_f64(q), _f64(k), _f64(v), _f64(do), causal, scale, p, seed)
     for name, x, ref in zip(("dQ", "dK", "dV"), (dq, dk, dv), refs):

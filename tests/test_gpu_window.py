@@ -2,9 +2,9 @@
 
 Key j is visible to query i iff i - left <= j <= i + right (-1 = unlimited on that side);
 the "FlashAttention1" Q&A's scaling question (item 4) proposes pairing the method with
-local attention.  Same tolerances as the dense tests: |O - O_ref| <= max(1e-2, one bf16
-spacing of O_ref), |LSE - LSE_ref| <= 1e-3, relative Frobenius error <= 2e-2 for dQ, dK,
-dV, guard bands intact, no NaN/Inf.  Exact checks: the windows that equal full and causal
+local attention.  Same tolerances as the dense tests (the O bound with the allowance for
+the bf16 probabilities computed over each row's window), |LSE - LSE_ref| <= 1e-3,
+relative Frobenius error <= 2e-2 for dQ, dK, dV, guard bands intact, no NaN/Inf.  Exact checks: the windows that equal full and causal
 attention reproduce fa_fwd / fa_bwd bit for bit, and a zero-width window returns V itself.
 """
 import math
@@ -17,7 +17,7 @@ import oracle
 from exact_io_aware_83_b200 import fa
 from exact_io_aware_83_b200.inputs import draw
 from test_gpu_parity import (GRAD_TOL, LSE_TOL, SENT_BF16, SENT_F32, _f64, _finite, _guarded,
-                             _guards_intact, _rel_fro, o_tolerance)
+                             _guards_intact, _rel_fro, o_tolerance, p_allowance)
 
 pytestmark = pytest.mark.gpu
 
@@ -53,11 +53,18 @@ def run_bwd_w(q, k, v, o, lse, do, window, scale):
 
 
 def check_fwd_w(o, lse, q, k, v, window, scale):
-    o_ref, lse_ref = oracle.attention_fwd_window(_f64(q), _f64(k), _f64(v), window[0], window[1],
-                                                 scale)
+    q64, k64, v64 = _f64(q), _f64(k), _f64(v)
+    o_ref, lse_ref = oracle.attention_fwd_window(q64, k64, v64, window[0], window[1], scale)
     _finite(o, lse)
     diff = np.abs(_f64(o) - o_ref)
-    excess = float(np.max(diff - o_tolerance(o_ref)))
+    keys = np.arange(q.shape[2])
+    left, right = window
+
+    def visible(b, h, i):
+        return (((keys >= i - left) if left >= 0 else True) & ((keys <= i + right) if right >= 0 else True)
+                & np.ones(len(keys), dtype=bool))
+
+    excess = float(np.max(diff - o_tolerance(o_ref, p_allowance(q64, k64, v64, o_ref, lse_ref, scale, visible))))
     err_l = float(np.max(np.abs(lse.double().numpy() - lse_ref)))
     assert excess <= 0.0, f"|O-O_ref| above tolerance by {excess}"
     assert err_l <= LSE_TOL, f"max|LSE-LSE_ref| = {err_l}"
