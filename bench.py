@@ -758,8 +758,13 @@ def run_ours(args, w):
     sms = torch.cuda.get_device_properties(local).multi_processor_count
     mhz = clocks.get("sm_mhz") or clocks.get("sm_max_mhz") or 1965.0
     exp_rate = 16.0 * sms * mhz * 1e6
+    # The forward kernel that ran: the persistent one for dense full / causal attention
+    # with d <= 128 (and its dropout form) when that scheduler is selected.
+    dense = w.block_density == 0 and w.window is None
+    fwd_name = ("fa_fwd_d256_kernel" if w.d == 256 else
+                "fa_fwd_persist_kernel" if dense and fa.fa_get_fwd_scheduler() else "fa_fwd_kernel")
     kernels = {}
-    for kname, kms, kn, kflops in (("fa_fwd_kernel", fwd_ms, nfwd, w.fwd_flops() * share / max(len(parts), 1)),
+    for kname, kms, kn, kflops in ((fwd_name, fwd_ms, nfwd, w.fwd_flops() * share / max(len(parts), 1)),
                                    ("fa_bwd_main_kernel", bwd_ms, nbwd, w.bwd_flops() * share / max(len(parts), 1))):
         if not kn:
             continue
@@ -776,7 +781,7 @@ def run_ours(args, w):
         kd["frac_of_sustained_peak"] = kd["tflops"] / float(peaks["bf16_tflops_sustained"])
         kd["frac_of_nominal_peak"] = kd["tflops"] / NOMINAL_BF16_TFLOPS
     # Dominant kernel: the backward main kernel (or the forward when there is no backward).
-    dom_name = "fa_bwd_main_kernel" if "fa_bwd_main_kernel" in kernels else "fa_fwd_kernel"
+    dom_name = "fa_bwd_main_kernel" if "fa_bwd_main_kernel" in kernels else fwd_name
     achieved = kernels[dom_name]["tflops"]
     traffic = _profile_traffic(dom_name, w.name) if args.scaling == "weak" else None
 

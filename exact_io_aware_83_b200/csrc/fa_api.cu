@@ -828,6 +828,8 @@ int fa_set_fwd_scheduler(int persistent) {
   return g_fwd_persistent.exchange(persistent);
 }
 
+int fa_get_fwd_scheduler(void) { return g_fwd_persistent.load(); }
+
 int fa_kernel_timing(int enable) {
   if (enable != 0 && enable != 1) return FA_ERR_INVALID_ARG;
   g_timer.enabled = enable != 0;

@@ -128,6 +128,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
         lib.fa_kernel_time_ms.restype = ci
         lib.fa_set_fwd_scheduler.argtypes = [ci]
         lib.fa_set_fwd_scheduler.restype = ci
+        lib.fa_get_fwd_scheduler.argtypes = []
+        lib.fa_get_fwd_scheduler.restype = ci
         _lib = lib
         return lib
 
@@ -269,6 +271,11 @@ def fa_set_fwd_scheduler(persistent: bool) -> bool:
     if prev < 0:
         _check(prev, "fa_set_fwd_scheduler")
     return bool(prev)
+
+
+def fa_get_fwd_scheduler() -> bool:
+    """True when the dense forward uses the persistent scheduler."""
+    return bool(load().fa_get_fwd_scheduler())
 
 
 def fa_kernel_time_ms(which: int):

@@ -359,6 +359,8 @@ int fa_kernel_time_ms(int which, float *ms, int *launches);
  * calls running on other host threads.
  */
 int fa_set_fwd_scheduler(int persistent);
+/* The current choice (1: persistent, 0: one CTA per unit). */
+int fa_get_fwd_scheduler(void);
 
 /*
  * Watchdog self-test: launches one thread that waits, with a limit of `limit_us`
