@@ -442,3 +442,16 @@ def test_persistent_forward_over_many_launches():
     assert fa.fa_device_status(None) == fa.FA_OK
     for o, lse in outs:
         assert torch.equal(o, ref_o) and torch.equal(lse, ref_l)
+
+
+def test_two_key_row_that_no_bf16_probability_kernel_can_hold_to_1e2():
+    """The constructed row of tests/test_o_bound_reading.py (|O| = 2.18, two keys, the second
+    probability 0.506 rounding to bf16 with relative error 0.0038): the kernel is held to the
+    derived bound, which the ideal bf16-probability computation also needs."""
+    from test_o_bound_reading import two_key_row
+    q64, k64, v64 = two_key_row()
+    q, k, v = (torch.from_numpy(t).to(torch.bfloat16) for t in (q64, k64, v64))
+    for causal in (False, True):
+        o, lse = run_fwd(q, k, v, causal, 1.0)
+        err_o, _ = check_fwd(o, lse, q, k, v, causal, 1.0)
+        print(f"two-key row, causal={causal}: max|O - O_ref| = {err_o:.4f}")
