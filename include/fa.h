@@ -349,7 +349,11 @@ int fa_kernel_time_ms(int which, float *ms, int *launches);
  * unit is two 128-row query tiles, numbered heaviest first under a causal mask.
  *   persistent = 1 (default): one CTA per SM walks the units, taking each next unit from a
  *       device counter (dynamic assignment), so one unit's epilogue overlaps the next
- *       unit's loads and first products.
+ *       unit's loads and first products.  The counter is one of 64 library-owned launch
+ *       slots, taken in turn by successive launches and reset by each launch's last CTA;
+ *       a launch captured in a CUDA graph keeps its slot, so replays of that graph must
+ *       not run on the GPU at the same time as the launch that takes the same slot 64
+ *       launches later.
  *   persistent = 0: one CTA per unit, started by the hardware in unit order.
  * The environment variable FA_FWD_PERSISTENT=0, read when the library loads, makes
  * one CTA per unit the starting choice.

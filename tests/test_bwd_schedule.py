@@ -34,7 +34,7 @@ class ScheduleError(AssertionError):
 
 
 def simulate(T, QS=3, NB=1, seed=0, dp_early=False, dpfree_wait=True, dsempty_wait=True,
-             ds_barrier_per_buffer=True, dqempty_wait=True):
+             ds_barrier_per_buffer=True, dqempty_wait=True, dp_after_dk=False):
     rnd = random.Random(seed)
     done = {}
     state = {"S": None, "dP": None, "dQ": None, "dS": [None] * NB, "stage": [None] * QS}
@@ -97,6 +97,9 @@ def simulate(T, QS=3, NB=1, seed=0, dp_early=False, dpfree_wait=True, dsempty_wa
             while not ready(ds_bar(db), du if ds_barrier_per_buffer else i):
                 yield
             engine.append(("dK", i))
+            if dp_after_dk and not dp_early and i + 1 < T:
+                engine.append(("dP", i + 1))
+                engine.append(("commit", ("DP",)))
             if i > 0 and dqempty_wait:
                 while not ready(("DQE",), i - 1):
                     yield
@@ -104,7 +107,7 @@ def simulate(T, QS=3, NB=1, seed=0, dp_early=False, dpfree_wait=True, dsempty_wa
             engine.append(("commit", ("DQ",)))
             engine.append(("commit", ("DSE", db)))
             engine.append(("commit", ("QE", st)))
-            if not dp_early and i + 1 < T:
+            if not dp_early and not dp_after_dk and i + 1 < T:
                 engine.append(("dP", i + 1))
                 engine.append(("commit", ("DP",)))
             yield
@@ -223,6 +226,12 @@ def simulate(T, QS=3, NB=1, seed=0, dp_early=False, dpfree_wait=True, dsempty_wa
 def test_backward_schedule_is_race_free(T):
     for seed in range(80):
         simulate(T, seed=seed)
+
+
+@pytest.mark.parametrize("T", [1, 2, 5, 16])
+def test_dp_between_dk_and_dq_is_race_free(T):
+    for seed in range(80):
+        simulate(T, seed=seed, dp_after_dk=True)
 
 
 @pytest.mark.parametrize("T", [2, 7])
