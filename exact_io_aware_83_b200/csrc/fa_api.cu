@@ -429,24 +429,29 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   if (mode != fa::kAttnSparse) p.bmask = nullptr;
   const int tslot = timer_start(0, s);
   // Unit order (unit_order), chosen from B200 measurements (forward TFLOP/s): dense causal
-  // attention runs its heavy units first - every level alone up to 16 query blocks, two
-  // tiers beyond (gpt_2k 660 -> 724, 8k causal 984 -> 1040, GQA 4k 983 -> 1006); a band or a
-  // block mask goes level by level (window_8k_1k 578 -> 611, blocksparse_8k 560 -> 614);
+  // attention runs its heavy units first up to 16 query blocks, every level alone (gpt_2k
+  // 660 -> 724; 826 against 777 for the head-major order below, persistent kernel); beyond,
+  // head-major with an eighth of the heads level by level at the end (persistent kernel:
+  // 8k causal 1066 -> 1090 and GQA 4k 1038 -> 1067 against two tiers of levels); a band or
+  // a block mask goes level by level (window_8k_1k 578 -> 611, blocksparse_8k 560 -> 614);
   // full attention and packed sequences stay head-major (packed: 680 head-major, 669-679
   // tiered).
   auto order = [&](int levels) {
-    if (mode == fa::kAttnCausal) return p.nqb <= 16 ? 1 : (levels + 1) / 2;
+    if (mode == fa::kAttnCausal) return p.nqb <= 16 ? 1 : levels;
     if (mode == fa::kAttnSparse || (mode == fa::kAttnGeneral && p.cu_q == nullptr)) return 1;
     return levels;
   };
+  p.tail = 0;
   if (d == 256) {
     p.pair_heads = 0;
     p.tsz = order(p.nqb);
+    if (mode == fa::kAttnCausal && p.nqb > 16) p.tail = p.B * p.Hq / 8;
     const unsigned units = static_cast<unsigned>(p.B) * p.Hq * p.nqb;
     launch_fwd_mode<256>(tq, tk, tv, to, p, units, mode, drop != nullptr, s);
   } else {
     p.pair_heads = (g % 2 == 0) ? 1 : 0;
     p.tsz = order(p.pair_heads ? p.nqb : (p.nqb + 1) / 2);
+    if (mode == fa::kAttnCausal && p.nqb > 16) p.tail = (p.pair_heads ? p.B * (p.Hq / 2) : p.B * p.Hq) / 8;
     const unsigned units = p.pair_heads ? static_cast<unsigned>(p.B) * (p.Hq / 2) * p.nqb
                                         : static_cast<unsigned>(p.B) * p.Hq * ((p.nqb + 1) / 2);
     if (d == 64)
@@ -495,17 +500,21 @@ bool normalise_window_varlen(int w, int max_q, int max_k, int *out) {
   return true;
 }
 
-// Backward unit order (tiers of key-block levels for unit_order), from B200 measurements.
-// Dense causal attention over at most 16 key blocks runs in three tiers, heavy first, so
-// no heavy unit starts last: gpt_2k main kernel 615 -> 649 TFLOP/s, at the price of DRAM
-// traffic 628 -> 977 MB per launch (each tier streams every head's Q / dO / dQ rows
-// again); at 8k the tiers were 2% slower, so longer sequences stay head-major (one head's
-// CTAs together in L2).  A band goes level by level (window_8k_1k backward call 518 -> 541);
+// Backward unit order (unit_order), from B200 measurements.  Dense causal attention runs
+// head-major - one (b, kv head) row's key blocks heaviest first, its CTAs together in L2 -
+// except for the last heads, which go level by level so that the grid ends on the lightest
+// units: half of the heads up to 16 key blocks, an eighth beyond (main kernel TFLOP/s:
+// gpt_2k 678 -> 696 and DRAM 977 -> ~630 MB per launch against three tiers of levels over
+// all heads, which stream every head's Q / dO / dQ rows once per tier; 8k causal 800 -> 832
+// against head-major).  A band goes level by level (window_8k_1k backward call 518 -> 541);
 // full attention and (in the callers) block masks and packed sequences stay head-major.
-int bwd_tiers(int N, int left, int right) {
-  if (left < 0 && right < 0) return 1;
-  if (left < 0 && right == 0) return (N + 127) / 128 <= 16 ? 3 : 1;
-  return 1 << 20;
+fa::BwdOrder bwd_order(int B, int Hkv, int N, int left, int right) {
+  if (left < 0 && right < 0) return {1, 0};
+  if (left < 0 && right == 0) {
+    const int heads = B * Hkv;
+    return {1, (N + 127) / 128 <= 16 ? heads / 2 : heads / 8};
+  }
+  return {1 << 20, 0};
 }
 
 // Block-sparse limits: the forward keeps each CTA's key-block list in shared memory (at most
@@ -664,7 +673,7 @@ int fa_bwd_window(const void *q, const void *k, const void *v, const void *o, co
   if (!device_ready()) return FA_ERR_CUDA;
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, left, right,
                         scale, static_cast<cudaStream_t>(stream), encode_fn(), &timer_start,
-                        &timer_stop, nullptr, nullptr, nullptr, bwd_tiers(N, left, right));
+                        &timer_stop, nullptr, nullptr, nullptr, bwd_order(B, Hkv, N, left, right));
 }
 
 size_t fa_bwd_varlen_workspace_bytes(int Hq, int total_q, int d) {
@@ -767,7 +776,7 @@ int fa_bwd_dropout(const void *q, const void *k, const void *v, const void *o, c
   // N = 1 with causal is full attention (normalise_window's rule); the mask is the same.
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
                         static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop, nullptr, &drop,
-                        nullptr, bwd_tiers(N, -1, causal ? 0 : -1));
+                        nullptr, bwd_order(B, Hkv, N, -1, causal ? 0 : -1));
 }
 
 int fa_fwd_blocksparse(const void *q, const void *k, const void *v, void *o, float *lse,
@@ -869,7 +878,7 @@ int fa_bwd_noalloc(const void *q, const void *k, const void *v, const void *o, c
   if (!scratch) return FA_ERR_CUDA;
   return fa::bwd_launch(q, k, v, o, lse, dout, dq, dk, dv, scratch, B, Hq, Hkv, N, d, -1, causal ? 0 : -1, scale,
                         static_cast<cudaStream_t>(stream), encode_fn(), &timer_start, &timer_stop, nullptr,
-                        nullptr, nullptr, bwd_tiers(N, -1, causal ? 0 : -1));
+                        nullptr, nullptr, bwd_order(B, Hkv, N, -1, causal ? 0 : -1));
 }
 
 int fa_watchdog_selftest(int limit_us, void *stream) {

@@ -110,6 +110,7 @@ struct BwdParams {
   DropCfg drop;           // dropout (kernels instantiated with DROP only)
   const uint8_t *bmask;   // block-sparse: [B, Hq, nkb, nkb] 0/1 over 128 x 128 blocks
   int tsz;                // unit order: key-block levels per tier (see unit_order)
+  int tail;               // unit order: heads taken level by level at the end
 };
 
 // D: head dimension (contraction of S^T and dP^T); DH: output columns owned by a CTA
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   // mask) first
   const int half = static_cast<int>(blockIdx.x) % kHalves;
   int head, kb;
-  unit_order(static_cast<int>(blockIdx.x) / kHalves, p.B * p.Hkv, p.nkb, p.tsz, head, kb);
+  unit_order(static_cast<int>(blockIdx.x) / kHalves, p.B * p.Hkv, p.nkb, p.tsz, p.tail, head, kb);
   const int kvh = head % p.Hkv;
   const int b = head / p.Hkv;
   const int g = p.Hq / p.Hkv;
@@ -804,12 +805,18 @@ inline void bwd_launch_main(const CUtensorMap &tq, const CUtensorMap &tk, const 
 typedef int (*TimerStartFn)(int, cudaStream_t);
 typedef void (*TimerStopFn)(int, int, cudaStream_t);
 
+// Unit order of a backward launch: tiers of key-block levels (1: head-major) and the
+// number of (b, kv head) rows taken level by level at the end of the grid.
+struct BwdOrder {
+  int tiers, tail;
+};
+
 template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                         int Hkv, int N, int left, int right, float scale, cudaStream_t s, EncodeTiledFnBwd enc,
                         TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk, const DropCfg *drop,
-                        const uint8_t *bmask, int tiers) {
+                        const uint8_t *bmask, BwdOrder order) {
   const long long rows = pk ? static_cast<long long>(pk->total_q) * Hq : static_cast<long long>(B) * Hq * N;
   float *delta = static_cast<float *>(workspace);
   float *dqacc = reinterpret_cast<float *>(static_cast<char *>(workspace) + pad256(static_cast<size_t>(rows) * 4));
@@ -856,8 +863,12 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.sl2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   p.drop = drop ? *drop : DropCfg{};
   p.bmask = bmask;
-  // Unit order (unit_order): `tiers` tiers of key-block levels (1: head-major).
+  // Unit order (unit_order): `order.tiers` tiers of key-block levels (1: head-major), the
+  // last `order.tail` (b, kv head) rows level by level.
+  const int tiers = order.tiers < 1 ? 1 : order.tiers;
   p.tsz = (p.nkb + tiers - 1) / tiers;
+  const int heads = B * Hkv;
+  p.tail = order.tail < 0 ? 0 : (order.tail < heads ? order.tail : heads - 1);
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
   if (grid > 0) {
@@ -889,16 +900,16 @@ inline int bwd_launch(const void *q, const void *k, const void *v, const void *o
                       const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
                       int Hkv, int N, int d, int left, int right, float scale, cudaStream_t s, Enc enc,
                       TimerStartFn tstart, TimerStopFn tstop, const PackedSeqs *pk = nullptr,
-                      const DropCfg *drop = nullptr, const uint8_t *bmask = nullptr, int tiers = 1) {
+                      const DropCfg *drop = nullptr, const uint8_t *bmask = nullptr, BwdOrder order = {1, 0}) {
   const EncodeTiledFnBwd e = reinterpret_cast<EncodeTiledFnBwd>(enc);
   if (d == 64)
     return bwd_launch_d<64, 64, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk, drop, bmask, tiers < 1 ? 1 : tiers);
+                                    scale, s, e, tstart, tstop, pk, drop, bmask, order);
   if (d == 128)
     return bwd_launch_d<128, 128, 64>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                      scale, s, e, tstart, tstop, pk, drop, bmask, tiers < 1 ? 1 : tiers);
+                                      scale, s, e, tstart, tstop, pk, drop, bmask, order);
   return bwd_launch_d<256, 128, 32>(q, k, v, o, lse, dout, dq, dk, dv, workspace, B, Hq, Hkv, N, left, right,
-                                    scale, s, e, tstart, tstop, pk, drop, bmask, tiers < 1 ? 1 : tiers);
+                                    scale, s, e, tstart, tstop, pk, drop, bmask, order);
 }
 
 }  // namespace fa

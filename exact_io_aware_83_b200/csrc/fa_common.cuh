@@ -116,9 +116,19 @@ constexpr int kAttnFull = 0, kAttnCausal = 1, kAttnGeneral = 2, kAttnSparse = 3;
 // levels; the tiers run heaviest first, and inside a tier one head's units are consecutive,
 // so the CTAs that run together share that head's K/V (or Q/dO) in L2.  tsz = levels is
 // head-major order, tsz = 1 pure heaviest-first.  The hardware starts CTAs in index order,
-// so heavy units never start last and leave a long tail.
-__device__ __forceinline__ void unit_order(int u, int heads, int levels, int tsz, int &head, int &level) {
-  const int per_tier = heads * tsz;
+// so heavy units never start last and leave a long tail.  With tail > 0 the last `tail`
+// heads come after all the others, level by level (heaviest first): only the end of the
+// grid gives up head locality, and it ends on the lightest units.
+__host__ __device__ __forceinline__ void unit_order(int u, int heads, int levels, int tsz, int tail,
+                                                    int &head, int &level) {
+  const int front = (heads - tail) * levels;
+  if (u >= front) {
+    const int v = u - front;
+    level = v / tail;
+    head = heads - tail + v % tail;
+    return;
+  }
+  const int per_tier = (heads - tail) * tsz;
   const int t = u / per_tier;
   const int v = u - t * per_tier;
   const int cnt = min(tsz, levels - t * tsz);

@@ -55,6 +55,7 @@ struct FwdParams {
   DropCfg drop;           // dropout (kernels instantiated with DROP only)
   const uint8_t *bmask;   // block-sparse: [B, Hq, nqb, nqb] 0/1 over 128 x 128 blocks
   int tsz;                // unit order: levels per tier (see unit_order)
+  int tail;               // unit order: heads taken level by level at the end
 };
 
 // Blocks of KB keys [lo, hi] that some row q0 .. min(q0 + 127, Lq - 1) of a query tile can
@@ -304,7 +305,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     int head, level;
     if (p.pair_heads) {
       const int hp_count = p.Hq / 2;
-      unit_order(u, p.B * hp_count, p.nqb, p.tsz, head, level);
+      unit_order(u, p.B * hp_count, p.nqb, p.tsz, p.tail, head, level);
       const int q = p.nqb - 1 - level;
       const int hp = head % hp_count;
       b = head / hp_count;
@@ -314,7 +315,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       valid[0] = valid[1] = true;
     } else {
       const int npairs = (p.nqb + 1) / 2;
-      unit_order(u, p.B * p.Hq, npairs, p.tsz, head, level);
+      unit_order(u, p.B * p.Hq, npairs, p.tsz, p.tail, head, level);
       const int pi = npairs - 1 - level;
       h[0] = h[1] = head % p.Hq;
       b = head / p.Hq;

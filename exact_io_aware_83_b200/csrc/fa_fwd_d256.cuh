@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kFwdD256Threads, 1)
   // ---- unit = (b, h, query block), ordered by unit_order (last query blocks, the longest
   // under a causal mask, are level 0)
   int head, level;
-  unit_order(blockIdx.x, p.B * p.Hq, p.nqb, p.tsz, head, level);
+  unit_order(blockIdx.x, p.B * p.Hq, p.nqb, p.tsz, p.tail, head, level);
   const int qb = p.nqb - 1 - level;
   const int h = head % p.Hq;
   const int b = head / p.Hq;

@@ -88,7 +88,7 @@ __device__ __forceinline__ void fwd_unit(const FwdParams &p, int u, bool causal,
   bool v1 = true;
   if (p.pair_heads) {
     const int hp_count = p.Hq / 2;
-    unit_order(u, p.B * hp_count, p.nqb, p.tsz, head, level);
+    unit_order(u, p.B * hp_count, p.nqb, p.tsz, p.tail, head, level);
     const int hp = head % hp_count;
     x.b = head / hp_count;
     x.h[0] = 2 * hp;
@@ -96,7 +96,7 @@ __device__ __forceinline__ void fwd_unit(const FwdParams &p, int u, bool causal,
     x.qb[0] = x.qb[1] = p.nqb - 1 - level;
   } else {
     const int npairs = (p.nqb + 1) / 2;
-    unit_order(u, p.B * p.Hq, npairs, p.tsz, head, level);
+    unit_order(u, p.B * p.Hq, npairs, p.tsz, p.tail, head, level);
     const int pi = npairs - 1 - level;
     x.h[0] = x.h[1] = head % p.Hq;
     x.b = head / p.Hq;
