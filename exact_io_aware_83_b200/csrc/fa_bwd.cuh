@@ -811,6 +811,11 @@ struct BwdOrder {
   int tiers, tail;
 };
 
+// Dense d = 256 backward main kernel as a two-CTA cluster (fa_bwd_pair.cuh).
+template <int MODE>
+bool bwd_launch_pair(EncodeTiledFnBwd enc, const void *q, const void *k, const void *v, const void *dout, void *dk,
+                     void *dv, float *dqacc, int B, int Hq, int Hkv, int N, const BwdParams &p, cudaStream_t s);
+
 template <int D, int DH, int BQ>
 inline int bwd_launch_d(const void *q, const void *k, const void *v, const void *o, const float *lse,
                         const void *dout, void *dq, void *dk, void *dv, void *workspace, int B, int Hq,
@@ -871,7 +876,17 @@ inline int bwd_launch_d(const void *q, const void *k, const void *v, const void 
   p.tail = order.tail < 0 ? 0 : (order.tail < heads ? order.tail : heads - 1);
   const unsigned grid = static_cast<unsigned>(B) * Hkv * p.nkb * (D / DH);
   const int tslot = tstart(1, s);
-  if (grid > 0) {
+  // Dense full and causal attention at d = 256 run as CTA pairs that split the work by role.
+  const bool pair = D == 256 && !pk && !drop && !bmask && left < 0 && right <= 0;
+  if (pair && grid > 0) {
+    const bool launched =
+        right == 0 ? bwd_launch_pair<kAttnCausal>(enc, q, k, v, dout, dk, dv, dqacc, B, Hq, Hkv, N, p, s)
+                   : bwd_launch_pair<kAttnFull>(enc, q, k, v, dout, dk, dv, dqacc, B, Hq, Hkv, N, p, s);
+    if (!launched) {
+      tstop(1, tslot, s);
+      return FA_ERR_CUDA;
+    }
+  } else if (grid > 0) {
     // Dense full and causal attention have their own variants; packed sequences and other
     // bands take the general one.
     if (bmask)  // block-sparse: dense layout, causal or not (right = 0 or -1)

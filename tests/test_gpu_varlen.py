@@ -120,7 +120,7 @@ def test_varlen_heads_and_groups(Hq, Hkv):
 @pytest.mark.parametrize("d", [64, 128, 256])
 def test_one_sequence_equals_the_dense_call(d):
     # A single sequence packed as [N, H, d] runs the same tiles as the dense [1, H, N, d]
-    # call: the forward is bitwise identical, dK and dV too.
+    # call: the forward is bitwise identical, dK and dV too (d = 64, 128).
     N, H = 384, 4
     q, k, v, do = draw(1, H, H, N, d, seed=17)
     scale = 1.0 / math.sqrt(d)
@@ -137,6 +137,12 @@ def test_one_sequence_equals_the_dense_call(d):
         g2 = fa.bwd_varlen(pack(q), pack(k), pack(v), o2, l2, pack(do), cu, cu, N, N,
                            causal=causal, scale=scale)
         torch.cuda.synchronize()
+        if d == 256:
+            # Dense d = 256 runs its backward as CTA pairs (64-row steps, P^T exchanged as
+            # bf16); packed sequences take the single-CTA d-split kernel: equal to rounding.
+            for a1, a2 in zip(g1, g2):
+                assert _rel_fro(_f64(a1[0].transpose(0, 1)), _f64(a2)) < 1e-2
+            continue
         assert torch.equal(g1[1][0].transpose(0, 1), g2[1])
         assert torch.equal(g1[2][0].transpose(0, 1), g2[2])
         assert _rel_fro(_f64(g1[0][0].transpose(0, 1)), _f64(g2[0])) < 1e-3
