@@ -770,9 +770,11 @@ def run_ours(args, w):
     dense = w.block_density == 0 and w.window is None
     fwd_name = ("fa_fwd_d256_kernel" if w.d == 256 else
                 "fa_fwd_persist_kernel" if dense and fa.fa_get_fwd_scheduler() else "fa_fwd_kernel")
+    # The backward main kernel: dense d = 256 attention without dropout runs as CTA pairs.
+    bwd_name = "fa_bwd_pair_kernel" if w.d == 256 and dense and not w.dropout_p else "fa_bwd_main_kernel"
     kernels = {}
     for kname, kms, kn, kflops in ((fwd_name, fwd_ms, nfwd, w.fwd_flops() * share / max(len(parts), 1)),
-                                   ("fa_bwd_main_kernel", bwd_ms, nbwd, w.bwd_flops() * share / max(len(parts), 1))):
+                                   (bwd_name, bwd_ms, nbwd, w.bwd_flops() * share / max(len(parts), 1))):
         if not kn:
             continue
         per = kms / kn
@@ -788,7 +790,7 @@ def run_ours(args, w):
         kd["frac_of_sustained_peak"] = kd["tflops"] / float(peaks["bf16_tflops_sustained"])
         kd["frac_of_nominal_peak"] = kd["tflops"] / NOMINAL_BF16_TFLOPS
     # Dominant kernel: the backward main kernel (or the forward when there is no backward).
-    dom_name = "fa_bwd_main_kernel" if "fa_bwd_main_kernel" in kernels else fwd_name
+    dom_name = bwd_name if bwd_name in kernels else fwd_name
     achieved = kernels[dom_name]["tflops"]
     traffic = _profile_traffic(dom_name, w.name) if args.scaling == "weak" else None
 

@@ -506,16 +506,17 @@ bool normalise_window_varlen(int w, int max_q, int max_k, int *out) {
 // Backward unit order (unit_order), from B200 measurements.  Dense causal attention runs
 // head-major - one (b, kv head) row's key blocks heaviest first, its CTAs together in L2 -
 // except for the last heads, which go level by level so that the grid ends on the lightest
-// units: half of the heads up to 16 key blocks, an eighth beyond (main kernel TFLOP/s:
-// gpt_2k 678 -> 696 and DRAM 977 -> ~630 MB per launch against three tiers of levels over
-// all heads, which stream every head's Q / dO / dQ rows once per tier; 8k causal 800 -> 832
-// against head-major).  A band goes level by level (window_8k_1k backward call 518 -> 541);
-// full attention and (in the callers) block masks and packed sequences stay head-major.
+// units: a quarter of the heads up to 16 key blocks, an eighth beyond (main kernel TFLOP/s:
+// gpt_2k 678 -> 694 and DRAM 977 -> 629 MB per launch against three tiers of levels over
+// all heads, which stream every head's Q / dO / dQ rows once per tier - half of the heads
+// in the tail ran as fast with 955 MB; 8k causal 800 -> 832 against head-major).  A band
+// goes level by level (window_8k_1k backward call 518 -> 541); full attention and (in the
+// callers) block masks and packed sequences stay head-major.
 fa::BwdOrder bwd_order(int B, int Hkv, int N, int left, int right) {
   if (left < 0 && right < 0) return {1, 0};
   if (left < 0 && right == 0) {
     const int heads = B * Hkv;
-    return {1, (N + 127) / 128 <= 16 ? heads / 2 : heads / 8};
+    return {1, (N + 127) / 128 <= 16 ? heads / 4 : heads / 8};
   }
   return {1 << 20, 0};
 }
