@@ -158,7 +158,11 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  *        heads that share each K/V head)
  *   workspace: device scratch of at least fa_bwd_workspace_bytes() bytes, 16-byte
  *        aligned; its contents on entry do not matter and on return are unspecified.
- * The score tiles are recomputed from Q, K and LSE (nothing N x N is stored).
+ * The score tiles are recomputed from Q, K and LSE (nothing N x N is stored).  At d = 256
+ * the main kernel runs as clusters of two CTAs on two SMs (one forms P, the other dS; the
+ * bf16 tiles cross through distributed shared memory), so dQ, dK and dV of this entry point
+ * and of fa_bwd_window with a causal or unlimited band agree with the d = 256 paths of the
+ * other entry points (packed, windowed, block-sparse, dropout) to rounding, not bit for bit.
  */
 int fa_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
            const void *dout, void *dq, void *dk, void *dv, void *workspace,
