@@ -434,11 +434,13 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   // Unit order (unit_order), chosen from B200 measurements (forward TFLOP/s): dense causal
   // attention runs its heavy units first up to 16 query blocks, every level alone (gpt_2k
   // 660 -> 724; 826 against 777 for the head-major order below, persistent kernel); beyond,
-  // head-major with an eighth of the heads level by level at the end (persistent kernel:
-  // 8k causal 1066 -> 1090 and GQA 4k 1038 -> 1067 against two tiers of levels); a band or
-  // a block mask goes level by level (window_8k_1k 578 -> 611, blocksparse_8k 560 -> 614);
-  // full attention and packed sequences stay head-major (packed: 680 head-major, 669-679
-  // tiered).
+  // head-major with half of the head pairs level by level at the end (persistent kernel, 8k
+  // causal: two tiers of levels 1066, a tail of an eighth 1090-1095, a quarter 1098, 3/8
+  // 1115, a half 1124-1141, 5/8 1134-1136, 3/4 1132; GQA 4k: an eighth 1072, a quarter to 5/8
+  // 1086-1102, 3/4 1094); a band or a block mask goes level by level (window_8k_1k 578 ->
+  // 611, blocksparse_8k 560 -> 614); full attention and packed sequences stay head-major
+  // (packed: 680 head-major, 669-679 tiered).  The d = 256 forward keeps an eighth
+  // (causal d = 256 was not measured).
   auto order = [&](int levels) {
     if (mode == fa::kAttnCausal) return p.nqb <= 16 ? 1 : levels;
     if (mode == fa::kAttnSparse || (mode == fa::kAttnGeneral && p.cu_q == nullptr)) return 1;
@@ -454,7 +456,7 @@ int launch_fwd(const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &
   } else {
     p.pair_heads = (g % 2 == 0) ? 1 : 0;
     p.tsz = order(p.pair_heads ? p.nqb : (p.nqb + 1) / 2);
-    if (mode == fa::kAttnCausal && p.nqb > 16) p.tail = (p.pair_heads ? p.B * (p.Hq / 2) : p.B * p.Hq) / 8;
+    if (mode == fa::kAttnCausal && p.nqb > 16) p.tail = (p.pair_heads ? p.B * (p.Hq / 2) : p.B * p.Hq) / 2;
     const unsigned units = p.pair_heads ? static_cast<unsigned>(p.B) * (p.Hq / 2) * p.nqb
                                         : static_cast<unsigned>(p.B) * p.Hq * ((p.nqb + 1) / 2);
     if (d == 64)
@@ -506,17 +508,18 @@ bool normalise_window_varlen(int w, int max_q, int max_k, int *out) {
 // Backward unit order (unit_order), from B200 measurements.  Dense causal attention runs
 // head-major - one (b, kv head) row's key blocks heaviest first, its CTAs together in L2 -
 // except for the last heads, which go level by level so that the grid ends on the lightest
-// units: a quarter of the heads up to 16 key blocks, an eighth beyond (main kernel TFLOP/s:
+// units: a quarter of the heads up to 16 key blocks, 3/8 beyond (main kernel TFLOP/s:
 // gpt_2k 678 -> 694 and DRAM 977 -> 629 MB per launch against three tiers of levels over
 // all heads, which stream every head's Q / dO / dQ rows once per tier - half of the heads
-// in the tail ran as fast with 955 MB; 8k causal 800 -> 832 against head-major).  A band
-// goes level by level (window_8k_1k backward call 518 -> 541); full attention and (in the
+// in the tail ran as fast with 955 MB; 8k causal against head-major 800, with 4 of its 32
+// heads in the tail 831, 6 843, 8 851, 12 853-855, 16 853, 20 847, 24 830).  A band goes
+// level by level (window_8k_1k backward call 518 -> 541); full attention and (in the
 // callers) block masks and packed sequences stay head-major.
 fa::BwdOrder bwd_order(int B, int Hkv, int N, int left, int right) {
   if (left < 0 && right < 0) return {1, 0};
   if (left < 0 && right == 0) {
     const int heads = B * Hkv;
-    return {1, (N + 127) / 128 <= 16 ? heads / 4 : heads / 8};
+    return {1, (N + 127) / 128 <= 16 ? heads / 4 : heads * 3 / 8};
   }
   return {1 << 20, 0};
 }
