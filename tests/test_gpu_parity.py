@@ -292,6 +292,15 @@ def test_bwd_d256_heads_and_lengths(Hq, Hkv, N, causal):
     check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
 
 
+def test_bwd_d256_causal_long_gqa():
+    # The cluster backward over 16 key blocks per head with causal masking: every cluster
+    # walks two query heads and up to 64 steps, with the diagonal blocks masked.
+    q, k, v, do = draw(1, 4, 2, 2048, 256, seed=4500)
+    o, lse = run_fwd(q, k, v, True, 0.0625)
+    dq, dk, dv = run_bwd(q, k, v, o, lse, do, True, 0.0625)
+    check_bwd(dq, dk, dv, q, k, v, do, True, 0.0625)
+
+
 def test_softmax_stress_large_scores_d256():
     q, k, v, do = draw(1, 2, 1, 520, 256, seed=78, q_std=4.0)
     for causal in (False, True):
