@@ -770,8 +770,11 @@ def run_ours(args, w):
     dense = w.block_density == 0 and w.window is None
     fwd_name = ("fa_fwd_d256_kernel" if w.d == 256 else
                 "fa_fwd_persist_kernel" if dense and fa.fa_get_fwd_scheduler() else "fa_fwd_kernel")
-    # The backward main kernel: dense d = 256 attention without dropout runs as CTA pairs.
-    bwd_name = "fa_bwd_pair_kernel" if w.d == 256 and dense and not w.dropout_p else "fa_bwd_main_kernel"
+    # The backward main kernel: dense attention without dropout runs as CTA pairs at
+    # d = 256 and with 128-query steps at d = 128 from N = 4096 on (the library's dispatch).
+    plain = dense and not w.dropout_p
+    bwd_name = ("fa_bwd_pair_kernel" if plain and w.d == 256 else
+                "fa_bwd_q128_kernel" if plain and w.d == 128 and w.N >= 4096 else "fa_bwd_main_kernel")
     kernels = {}
     for kname, kms, kn, kflops in ((fwd_name, fwd_ms, nfwd, w.fwd_flops() * share / max(len(parts), 1)),
                                    (bwd_name, bwd_ms, nbwd, w.bwd_flops() * share / max(len(parts), 1))):

@@ -21,6 +21,7 @@
 #include "fa_fwd_persist.cuh"
 #include "fa_bwd.cuh"
 #include "fa_bwd_pair.cuh"
+#include "fa_bwd_q128.cuh"
 #include "fa_decode.cuh"
 
 namespace {
@@ -161,6 +162,8 @@ bool device_ready() {
     ok = ok && set_smem(fa_bwd_main_kernel<256, 128, 32, fa::kAttnGeneral>, BwdLayout<256, 128, 32>::kSmemBytes);
     ok = ok && set_smem(fa::fa_bwd_pair_kernel<fa::kAttnFull>, fa::PairLayout::kSmemBytes);
     ok = ok && set_smem(fa::fa_bwd_pair_kernel<fa::kAttnCausal>, fa::PairLayout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_bwd_q128_kernel<fa::kAttnFull>, fa::Q128Layout::kSmemBytes);
+    ok = ok && set_smem(fa::fa_bwd_q128_kernel<fa::kAttnCausal>, fa::Q128Layout::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnFull, true>, BwdLayout<64, 64, 64>::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<64, 64, 64, fa::kAttnCausal, true>, BwdLayout<64, 64, 64>::kSmemBytes);
     ok = ok && set_smem(fa_bwd_main_kernel<128, 128, 64, fa::kAttnFull, true>, BwdLayout<128, 128, 64>::kSmemBytes);

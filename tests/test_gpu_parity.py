@@ -280,6 +280,21 @@ def test_bwd_heads_and_groups(Hq, Hkv, causal):
     check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,N", [(1, 2, 1, 4096), (1, 2, 2, 4133), (1, 4, 1, 4200),
+                                         (1, 3, 3, 4351), (2, 2, 1, 4160)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bwd_long_128_query_steps(B, Hq, Hkv, N, causal):
+    # From N = 4096 on, the dense d = 128 backward takes 128-query steps, with dQ^T sharing
+    # tensor memory with dP^T and the dQ rows reduced in two 64-row halves: whole blocks,
+    # ragged last blocks whose second half is empty (37 rows), partial (104) or one row
+    # short (127), query-head groups of 1 to 4, two batches.
+    q, k, v, do = draw(B, Hq, Hkv, N, 128, seed=6000 + B * 1000 + Hq * 100 + N)
+    scale = 0.0883883461356163
+    o, lse = run_fwd(q, k, v, causal, scale)
+    dq, dk, dv = run_bwd(q, k, v, o, lse, do, causal, scale)
+    check_bwd(dq, dk, dv, q, k, v, do, causal, scale)
+
+
 @pytest.mark.parametrize("Hq,Hkv,N", [(4, 4, 200), (8, 2, 640), (3, 1, 333), (2, 2, 1000)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_bwd_d256_heads_and_lengths(Hq, Hkv, N, causal):
