@@ -322,43 +322,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       tc_fence_after_sync();
       const float4 *lse4 = reinterpret_cast<const float4 *>(lse_s + st * BQ + c0);
       const float4 *dl4 = reinterpret_cast<const float4 *>(delta_s + c0);
-      // P^T half by half (32 query columns each): exponentials, masks (key rows past N and,
-      // causal, queries before this key; query rows past N already have P = 0), then the
-      // bf16 pairs into the first 16 columns of that half's S^T, which it has just read.
-      float pr[HC];
+      // P^T over the warpgroup's 64 columns from one TMEM load: exponentials, masks (key
+      // rows past N and, causal, queries before this key; query rows past N already have
+      // P = 0), then the bf16 pairs into the first 32 of its S^T columns.  The packed pairs
+      // are also P for this step's dS: 64 fp32 values would leave too few of a thread's 128
+      // registers to load dP^T in one piece.
+      uint32_t pk[HC / 2];
+      {
+        uint32_t rr[HC];
+        tmem_ld_x64(tS, rr);
+        const bool diag = MODE == kAttnCausal && q0 < kv;
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t rr[32];
-        tmem_ld_x32(tS + h2 * 32, rr);
+        for (int c4 = 0; c4 < HC / 4; ++c4) {
+          const float4 l = lse4[c4];
+          float e[4];
+          e[0] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 0]), sl2, -l.x));
+          e[1] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 1]), sl2, -l.y));
+          e[2] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 2]), sl2, -l.z));
+          e[3] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 3]), sl2, -l.w));
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 l = lse4[h2 * 8 + c4];
-          pr[h2 * 32 + 4 * c4 + 0] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 0]), sl2, -l.x));
-          pr[h2 * 32 + 4 * c4 + 1] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 1]), sl2, -l.y));
-          pr[h2 * 32 + 4 * c4 + 2] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 2]), sl2, -l.z));
-          pr[h2 * 32 + 4 * c4 + 3] = ex2_approx(fmaf(__uint_as_float(rr[4 * c4 + 3]), sl2, -l.w));
+          for (int j = 0; j < 4; ++j)
+            if (!row_live || (diag && q0 + 4 * c4 + j < kv)) e[j] = 0.f;
+          pk[2 * c4] = pack_bf16x2(e[0], e[1]);
+          pk[2 * c4 + 1] = pack_bf16x2(e[2], e[3]);
         }
-        const int qh = q0 + h2 * 32;
-        if (!row_live) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pr[h2 * 32 + c] = 0.f;
-        } else if (MODE == kAttnCausal && qh < kv) {
-#pragma unroll
-          for (int c = 0; c < 32; ++c)
-            if (qh + c < kv) pr[h2 * 32 + c] = 0.f;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) pk[c] = pack_bf16x2(pr[h2 * 32 + 2 * c], pr[h2 * 32 + 2 * c + 1]);
-        tmem_st_x16(tS + h2 * 16, pk);
+        tmem_st_x32(tS, pk);
       }
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kBarP));
 
-      // dS^T = P^T o (dP^T - Delta), written half by half into this row of shared memory
-      // (128-byte swizzled) once the previous step's dK and dQ^T have read dS^T.
+      // dS^T = P^T o (dP^T - Delta) into this row of shared memory (128-byte swizzled), once
+      // the previous step's dK and dQ^T have read dS^T.
       if (!(ok = warp_wait_bounded(bar(L::kBarDSEmpty), (i & 1) ^ 1, abort_flag,
                                    wait_site(kSite, L::kBarDSEmpty, i))))
         break;
@@ -367,25 +363,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         break;
       if (!(ok = warp_wait_bounded(bar(L::kBarDP), i & 1, abort_flag, wait_site(kSite, L::kBarDP, i)))) break;
       tc_fence_after_sync();
+      {
+        uint32_t rr[HC];
+        tmem_ld_x64(tDP, rr);
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        uint32_t rr[32];
-        tmem_ld_x32(tDP + h2 * 32, rr);
-        uint32_t dsk[16];
+        for (int uu = 0; uu < HC / 8; ++uu) {  // 16-byte unit uu: columns 8uu .. 8uu + 7
+          uint32_t w[4];
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 dd = dl4[h2 * 8 + c4];
-          const int c = h2 * 32 + 4 * c4;
-          dsk[2 * c4] = pack_bf16x2(pr[c + 0] * (__uint_as_float(rr[4 * c4 + 0]) - dd.x),
-                                    pr[c + 1] * (__uint_as_float(rr[4 * c4 + 1]) - dd.y));
-          dsk[2 * c4 + 1] = pack_bf16x2(pr[c + 2] * (__uint_as_float(rr[4 * c4 + 2]) - dd.z),
-                                        pr[c + 3] * (__uint_as_float(rr[4 * c4 + 3]) - dd.w));
-        }
-#pragma unroll
-        for (int uu = 0; uu < 4; ++uu) {
-          const int unit = h2 * 4 + uu;
-          st_shared_v4(rowp + ((unit ^ (r & 7)) * 16), dsk[4 * uu], dsk[4 * uu + 1], dsk[4 * uu + 2],
-                       dsk[4 * uu + 3]);
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * uu + e;  // pair j: columns 2j (low half) and 2j + 1
+            const float4 dd = dl4[j / 2];
+            const float d0 = (j & 1) ? dd.z : dd.x, d1 = (j & 1) ? dd.w : dd.y;
+            const float p0 = __uint_as_float(pk[j] << 16), p1 = __uint_as_float(pk[j] & 0xFFFF0000u);
+            w[e] = pack_bf16x2(p0 * (__uint_as_float(rr[2 * j]) - d0), p1 * (__uint_as_float(rr[2 * j + 1]) - d1));
+          }
+          st_shared_v4(rowp + ((uu ^ (r & 7)) * 16), w[0], w[1], w[2], w[3]);
         }
       }
       fence_proxy_async_smem();
