@@ -75,6 +75,23 @@ def _peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+# The library takes 128-query backward steps for dense d = 128 attention from this sequence
+# length on (kQ128MinN in exact_io_aware_83_b200/csrc/fa_bwd.cuh).
+Q128_MIN_N = 4096
+
+
+def _bwd_kernel_name(w) -> str:
+    """The backward main kernel the library's dispatch runs for workload `w`: dense
+    attention without dropout runs as CTA pairs at d = 256 and with 128-query steps at
+    d = 128 from Q128_MIN_N on; everything else runs fa_bwd_main_kernel."""
+    plain = w.block_density == 0 and w.window is None and not w.dropout_p
+    if plain and w.d == 256:
+        return "fa_bwd_pair_kernel"
+    if plain and w.d == 128 and w.N >= Q128_MIN_N:
+        return "fa_bwd_q128_kernel"
+    return "fa_bwd_main_kernel"
+
+
 def _profile_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu capture
     (profiles/dram_traffic.json), or None when there is none or a source file of the
@@ -770,11 +787,7 @@ def run_ours(args, w):
     dense = w.block_density == 0 and w.window is None
     fwd_name = ("fa_fwd_d256_kernel" if w.d == 256 else
                 "fa_fwd_persist_kernel" if dense and fa.fa_get_fwd_scheduler() else "fa_fwd_kernel")
-    # The backward main kernel: dense attention without dropout runs as CTA pairs at
-    # d = 256 and with 128-query steps at d = 128 from N = 4096 on (the library's dispatch).
-    plain = dense and not w.dropout_p
-    bwd_name = ("fa_bwd_pair_kernel" if plain and w.d == 256 else
-                "fa_bwd_q128_kernel" if plain and w.d == 128 and w.N >= 4096 else "fa_bwd_main_kernel")
+    bwd_name = _bwd_kernel_name(w)
     kernels = {}
     for kname, kms, kn, kflops in ((fwd_name, fwd_ms, nfwd, w.fwd_flops() * share / max(len(parts), 1)),
                                    (bwd_name, bwd_ms, nbwd, w.bwd_flops() * share / max(len(parts), 1))):

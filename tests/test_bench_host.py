@@ -151,3 +151,16 @@ def test_config_names_the_workload():
     assert c["window"] == [1023, 0]
     c = bench._config(DECODE_WORKLOADS["decode_64k_gqa"], 1)
     assert c["cache_len"] == 65536 and c["passes"] == "decode"
+
+
+def test_backward_kernel_names_follow_the_library_dispatch():
+    import re
+    src = open(os.path.join(os.path.dirname(bench.__file__), "exact_io_aware_83_b200", "csrc",
+                            "fa_bwd.cuh")).read()
+    assert int(re.search(r"constexpr int kQ128MinN = (\d+);", src).group(1)) == bench.Q128_MIN_N
+    expect = {"gpt_2k_causal": "fa_bwd_main_kernel", "long_8k_causal": "fa_bwd_q128_kernel",
+              "gqa_4k_causal_fwd": "fa_bwd_q128_kernel", "d256_4k_stress": "fa_bwd_pair_kernel",
+              "window_8k_1k": "fa_bwd_main_kernel", "dropout_8k_causal": "fa_bwd_main_kernel",
+              "blocksparse_8k_causal": "fa_bwd_main_kernel"}
+    for name, kernel in expect.items():
+        assert bench._bwd_kernel_name(WORKLOADS[name]) == kernel, name
