@@ -148,11 +148,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_load_3d(sV + c * L::kChunk, &tm_v, bar(L::kBarKV), c * 64, kv0, kv_c2);
       }
     }
+    // A step's LSE and Delta values (4 of each a lane) are read from global memory one
+    // iteration early, so that their latency overlaps this iteration's waits instead of
+    // delaying the next Q load.  Query rows past N get LSE = +inf, so their probabilities
+    // (and dS) are exactly 0.
+    auto fetch = [&](int k, float (&lv)[4], float (&dv)[4]) {
+      const int qk = step_q0(k);
+      const size_t rk = static_cast<size_t>(b * p.Hq + step_head(k)) * p.N;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = qk + lane + 32 * u;
+        lv[u] = q < p.N ? p.lse[rk + q] * 1.4426950408889634f : INFINITY;
+        dv[u] = q < p.N ? p.delta[rk + q] : 0.f;
+      }
+    };
+    float lse_c[4], dl_c[4];
+    fetch(0, lse_c, dl_c);
     int issued_q = 0, issued_do = 0;
     for (int i = 0; ok && i < T; ++i) {
       const int st = i & 1;
       const int h = step_head(i), q0 = step_q0(i);
       const int c2 = b * p.Hq + h;
+      float lse_n[4], dl_n[4];
+      if (i + 1 < T) fetch(i + 1, lse_n, dl_n);
       ok = warp_wait_bounded(bar(L::kBarQEmpty + st), ((i >> 1) & 1) ^ 1, abort_flag,
                              wait_site(kSite, L::kBarQEmpty + st, i));
       if (!ok) break;
@@ -162,12 +180,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int c = 0; c < 2; ++c)
           tma_load_3d(sQ + st * L::kTile + c * L::kChunk, &tm_q, bar(L::kBarQFull + st), c * 64, q0, c2);
       }
-      const size_t row0 = static_cast<size_t>(c2) * p.N;
-      for (int c = lane; c < BQ; c += 32) {
-        // Query rows past N get LSE = +inf, so their probabilities (and dS) are exactly 0.
-        const int q = q0 + c;
-        lse_s[st * BQ + c] = q < p.N ? p.lse[row0 + q] * 1.4426950408889634f : INFINITY;
-      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) lse_s[st * BQ + lane + 32 * u] = lse_c[u];
       // The stores above are ordered before lane 0's arrival by the warp barrier; the
       // phase completes only when that arrival and the TMA bytes are both in.
       __syncwarp();
@@ -187,15 +201,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const bool ds_ok =
           i == 0 || warp_wait_bounded(bar(L::kBarDS), (i - 1) & 1, abort_flag, wait_site(kSite, L::kBarDS, i - 1));
       if (ds_ok) {
-        for (int c = lane; c < BQ; c += 32) {
-          const int q = q0 + c;
-          delta_s[c] = q < p.N ? p.delta[row0 + q] : 0.f;
-        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) delta_s[lane + 32 * u] = dl_c[u];
       }
       // Arrive even after an abort, so that the phase completes once the bytes are in.
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(L::kBarDOFull));
       if (!(ok = ds_ok)) break;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        lse_c[u] = lse_n[u];
+        dl_c[u] = dl_n[u];
+      }
     }
     // Loads still in flight after an abort land before the CTA exits: the last two Q
     // stages and the last dO load (each earlier one was consumed before the next issued).
